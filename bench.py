@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Benchmark: MoE-layer tokens/s and achieved HBM GB/s (4-bit experts, K=4, batch 1).
+
+Workload: one MoE layer shaped like the Qwen3.5-397B layer the pages run
+(hidden 4096, 512 experts, top-4, expert intermediate 1024, 4-bit group-64
+experts with bf16 scale/bias, a bf16 shared expert of the same size), one
+token per step, router bias Zipf(1.1)-skewed.  All inputs are seeded
+synthetic data.  A step is one call of moe_layer_forward (router, top-K,
+routed experts, shared expert, combine, residual, RMSNorm) on one token.
+
+L2 guard: R=8 independent replicas of the layer (3.6 GB of experts each,
+29 GB in all) are used round-robin, so no step finds its weights in the
+126 MB L2 from an earlier step.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--bits 4|2] [--impl ours|reference]
+
+For N > 1 run under torch.distributed.run: every rank runs its own replica
+of the workload (replicas only: the layer has no exchange step), the timed
+region is bracketed by barriers, and the time is the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth as S  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and achieved HBM GB/s (4-bit experts, K=4, batch 1)"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["moe_decode.cu", "moe_phases.cuh", "moe_device.cuh", "moe_layout.h", "moe_kernels.h"]
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--bits", type=int, default=4, choices=(4, 2))
+    p.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    p.add_argument("--replicas", type=int, default=8)
+    p.add_argument("--e2e-steps", type=int, default=300)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-graph", action="store_true")
+    return p.parse_args(argv)
+
+
+def workload(bits):
+    return S.QWEN_4BIT if bits == 4 else S.QWEN_2BIT
+
+
+def algorithmic_bytes(s, T=1):
+    """Bytes one launch must move at least: the K chosen experts' packed blobs,
+    the bf16 shared expert, the bf16 router, bias, gamma, activations in and
+    out."""
+    import quantized_expert_ffn_03_b200 as M
+    cfg = M.config(s.hidden, s.inter, s.n_experts, s.top_k, bits=s.bits)
+    experts = T * s.top_k * M.moe_packed_expert_bytes(cfg)  # distinct experts per token
+    shared = 3 * s.hidden * s.inter * 2 if s.has_shared else 0
+    router = s.n_experts * s.hidden * 2 + s.n_experts * 4
+    small = s.hidden * 2 + 4 * T * s.hidden * 2 + 2 * T * s.top_k * 4
+    return experts + shared + router + small
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "quantized_expert_ffn_03_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(bits):
+    """dram bytes per launch from a committed ncu summary, if it was taken on
+    the kernel as it is now."""
+    path = os.path.join(ROOT, "profiles", "moe_decode_kernel_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        ent = d.get("%dbit" % bits)
+        if ent and ent.get("src_sha") == kernel_source_hash():
+            return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---- distributed plumbing (replicas only) -------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def aggregate(elapsed_ms, units, group_backend_device=None):
+    """Max of elapsed over ranks and sum of units over ranks (all ranks call)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized():
+        return elapsed_ms, units
+    dev = group_backend_device or "cpu"
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    u = torch.tensor([units], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ---- clocks -------------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+        "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index, period_s=0.005):
+        self.dev, self.period = device_index, period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        for k, bit in self.REASONS.items():
+                            if r & bit:
+                                self.reasons.add(k)
+                    except Exception:
+                        pass
+                    time.sleep(self.period)
+
+            self._t = threading.Thread(target=run, daemon=True)
+            self._t.start()
+        except Exception:
+            self.ok = False
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---- CPU oracle timing ------------------------------------------------------------------
+
+def oracle_token_rate(s, n_tokens, seconds_cap=None):
+    """Time the plain C oracle (single-threaded) on n_tokens tokens of the
+    workload; expert generation and quantisation are done first, untimed."""
+    import oracle as O
+    oc = O.cfg(s.hidden, s.inter, s.n_experts, s.top_k, bits=s.bits, eps=s.eps, has_shared=s.has_shared)
+    d = S.dense_weights(s, 0)
+    toks = [S.activations(s, step=k) for k in range(n_tokens)]
+    need = set()
+    for x, _ in toks:
+        _, idx, _ = O.router(oc, x, d["wr"], d["bias"])
+        need |= set(idx.ravel().tolist())
+    blobs = {e: O.quantize_expert(oc, *S.expert_weights(s, e)) for e in sorted(need)}
+    first = blobs[min(blobs)]
+    lst = [blobs.get(e, first) for e in range(s.n_experts)]
+    done, t0 = 0, time.perf_counter()
+    for x, res in toks:
+        O.layer_forward(oc, lst, d["wr"], d["bias"], d["shared_gate"], d["shared_up"], d["shared_down"],
+                        d["gamma"], x, res)
+        done += 1
+        if seconds_cap is not None and time.perf_counter() - t0 > seconds_cap:
+            break
+    dt = time.perf_counter() - t0
+    return done / dt, done, dt
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    s = workload(args.bits)
+    # each step is one token through the oracle; the run is capped so that the
+    # whole --steps/--warmup invocation ends within a few minutes
+    rate1, _, t1 = oracle_token_rate(s, 1)
+    n = max(1, min(args.steps, int(150.0 / max(t1, 1e-3))))
+    rate, done, dt = oracle_token_rate(s, n, seconds_cap=150.0)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": done, "warmup": 1, "ms_per_step": 1e3 * dt / done, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": s.name, "hidden": s.hidden, "inter": s.inter, "n_experts": s.n_experts,
+                   "top_k": s.top_k, "bits": s.bits, "tokens_per_step": 1},
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": "%d tokens of the workload through the single-threaded C oracle "
+                                   "(fp64, dequantise-then-dot), experts generated and quantised "
+                                   "before timing" % done},
+        "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- GPU run ----------------------------------------------------------------------------
+
+def build_replica(M, s, replica, T, chunk=32):
+    import torch
+    cfg = M.config(s.hidden, s.inter, s.n_experts, s.top_k, bits=s.bits, eps=s.eps, has_shared=s.has_shared)
+    nb = M.moe_packed_expert_bytes(cfg)
+    pool = torch.empty(s.n_experts * nb, dtype=torch.uint8, device="cuda")
+    for e0 in range(0, s.n_experts, chunk):
+        n = min(chunk, s.n_experts - e0)
+        wg, wu, wd = S.torch_expert_weights(s, e0, n, replica, "cuda")
+        M.moe_pack_experts_device(cfg, wg, wu, wd, pool[e0 * nb:(e0 + n) * nb])
+        del wg, wu, wd
+    ptrs = (torch.arange(s.n_experts, dtype=torch.int64, device="cuda") * nb + pool.data_ptr()).contiguous()
+    d = S.dense_weights(s, replica)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+    r = dict(pool=pool, ptrs=ptrs, wr=dev(d["wr"]), bias=torch.from_numpy(d["bias"]).cuda(),
+             sg=dev(d["shared_gate"]), su=dev(d["shared_up"]), sd=dev(d["shared_down"]), gamma=dev(d["gamma"]))
+    r["wts"] = M.layer_weights(r["ptrs"], r["wr"], r["bias"], r["sg"], r["su"], r["sd"], r["gamma"])
+    r["ws"] = torch.zeros(M.moe_layer_host_workspace_bytes(cfg, T), dtype=torch.uint8, device="cuda")
+    M.moe_workspace_init(r["ws"])
+    r["cfg"] = cfg
+    return r
+
+
+def run_ours(args):
+    import torch
+    import quantized_expert_ffn_03_b200 as M
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev_index = torch.cuda.current_device()
+    s = workload(args.bits)
+    T = 1
+    R = max(1, args.replicas)
+    reps = [build_replica(M, s, rr + 17 * rank, T) for rr in range(R)]
+    torch.cuda.synchronize()
+
+    # token pool: fresh N(0,1) bf16 activations per step
+    P = min(args.steps + args.warmup, 4096)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1234 + rank)
+    xs = torch.randn((P, T, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
+    rs = torch.randn((P, T, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
+    h_out = torch.empty((R, T, s.hidden), dtype=torch.int16, device="cuda")
+    y_out = torch.empty((R, T, s.hidden), dtype=torch.int16, device="cuda")
+    cfg = reps[0]["cfg"]
+
+    def step(i):
+        r = reps[i % R]
+        k = i % P
+        M.moe_layer_forward(cfg, r["wts"], xs[k], rs[k], h_out[i % R], y_out[i % R], workspace=r["ws"])
+
+    stream = torch.cuda.Stream()
+    used_graph = False
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize()
+        graph = None
+        if not args.no_graph:
+            try:
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=stream):
+                    for i in range(args.steps):
+                        step(args.warmup + i)
+                graph.replay()  # untimed: uploads the graph
+                torch.cuda.synchronize()
+                used_graph = True
+            except Exception as e:  # capture not possible: time direct launches
+                print("graph capture failed (%s); timing direct launches" % e, file=sys.stderr)
+                graph = None
+                torch.cuda.synchronize()
+        st, detail = M.moe_device_error(reps[0]["ws"])
+        assert st == 0, (st, detail)
+
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(dev_index) as clk:
+            start.record(stream)
+            if graph is not None:
+                graph.replay()
+            else:
+                for i in range(args.steps):
+                    step(args.warmup + i)
+            stop.record(stream)
+            torch.cuda.synchronize()
+        barrier()
+        local_ms = start.elapsed_time(stop)
+        for r in reps:
+            st, detail = M.moe_device_error(r["ws"])
+            assert st == 0, ("device error after timed run", st, detail)
+
+        # L2-assisted (single replica, warm) figure, for context
+        warm = None
+        if graph is not None:
+            g1 = torch.cuda.CUDAGraph()
+            n1 = min(args.steps, 500)
+            with torch.cuda.graph(g1, stream=stream):
+                for i in range(n1):
+                    M.moe_layer_forward(cfg, reps[0]["wts"], xs[i % P], rs[i % P], h_out[0], y_out[0],
+                                        workspace=reps[0]["ws"])
+            g1.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g1.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            warm = e0.elapsed_time(e1) / n1
+            del g1
+
+    elapsed_ms, units = aggregate(local_ms, float(args.steps * T), "cuda" if world > 1 else None)
+    ms_per_step = elapsed_ms / args.steps
+    value = units / (elapsed_ms / 1e3)
+
+    # end to end through the host-buffer entry point: H2D of the step's inputs
+    # from pinned memory and D2H of its outputs inside the timed region
+    ne = min(args.e2e_steps, P)
+    xh = xs[:ne].cpu().pin_memory()
+    rh = rs[:ne].cpu().pin_memory()
+    hh = torch.empty((T, s.hidden), dtype=torch.int16).pin_memory()
+    yh = torch.empty((T, s.hidden), dtype=torch.int16).pin_memory()
+    for i in range(5):
+        M.moe_layer_forward_host(cfg, reps[i % R]["wts"], xh[i], rh[i], hh, yh, reps[i % R]["ws"], stream=stream)
+    barrier()
+    t0 = time.perf_counter()
+    for i in range(ne):
+        r = reps[i % R]
+        M.moe_layer_forward_host(cfg, r["wts"], xh[i], rh[i], hh, yh, r["ws"], stream=stream)
+    e2e_ms = (time.perf_counter() - t0) * 1e3
+    barrier()
+    e2e_ms, e2e_units = aggregate(e2e_ms, float(ne * T), "cuda" if world > 1 else None)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, done, dt = oracle_token_rate(s, 6, seconds_cap=30.0)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": "%d tokens of this workload through the single-threaded C oracle (fp64 "
+                         "dequantise-then-dot, %.1f s); experts generated and quantised before timing"
+                         % (done, dt)}
+
+    peak, peak_src = measured_peaks()
+    abytes = algorithmic_bytes(s, T)
+    achieved = abytes / (ms_per_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": s.name, "hidden": s.hidden, "inter": s.inter, "n_experts": s.n_experts,
+                   "top_k": s.top_k, "bits": s.bits, "group": s.group, "tokens_per_step": T,
+                   "shared_expert": "bf16", "router_bias": "zipf1.1", "replicas": R,
+                   "l2": "inputs larger than L2: %d replicas round-robin, %.1f GB of experts" %
+                         (R, R * s.n_experts * M.moe_packed_expert_bytes(cfg) / 1e9),
+                   "cuda_graph": used_graph, "parallelism": "replicas" if world > 1 else "single"},
+        "hbm_gbs": achieved,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(args.bits),
+                     "peak_source": peak_src, "algorithmic_bytes_per_launch": abytes,
+                     "kernel": "moe_decode_kernel"},
+        "e2e": {"value": e2e_units / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": 2 * T * s.hidden * 2, "d2h_bytes_per_step": 2 * T * s.hidden * 2},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "l2_warm_tokens_per_s": (T / (warm * 1e-3)) if warm else None,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

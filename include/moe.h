@@ -1,0 +1,199 @@
+/*
+ * moe.h -- C ABI of libmoe: the per-token Mixture-of-Experts layer of a
+ * "streaming experts" decoder, on NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes (the pages describe the Flash-MoE engine that runs
+ * Qwen3.5-397B-A17B with experts streamed from SSD):
+ *   1. router: logits = x . Wr^T + bias; the top K of E experts per token,
+ *      weights = softmax over E renormalised over the K chosen
+ *      ("Streaming experts: как запустить триллионную модель на MacBook"
+ *      (toolarium.ru), section "Mixture of Experts и почему SSD достаточно":
+ *      4 of 512 experts per token; "Flash-MoE: ラップトップでの397Bパラメータ
+ *      モデルの実行" (hakusoku.com), section "パイプライン概要": CPU
+ *      softmax/top-K after the GPU router projection);
+ *   2. for each chosen expert, a SwiGLU FFN whose weights are 4- or 2-bit
+ *      group-affine codes, dequantised as q*scale + bias and multiplied in the
+ *      fused form fma(q, scale*x, bias*x) (toolarium, section "Оптимизации,
+ *      которые сработали"; hakusoku, section "主要技術": FMA dequant kernel,
+ *      4/2-bit dequant matvec, SwiGLU);
+ *   3. a shared expert (bf16 SwiGLU FFN, weight 1) (hakusoku, section
+ *      "モデルアーキテクチャ": K=4 plus a shared expert);
+ *   4. combine + residual + RMSNorm in one kernel (toolarium, section
+ *      "Оптимизации, которые сработали"; hakusoku, section "主要技術").
+ *
+ * Conventions for every call:
+ *   - Pointers are owned by the caller.  Device pointers are CUDA global
+ *     memory on the current device; host pointers are ordinary host memory
+ *     (pinned where stated).  The library allocates device memory only inside
+ *     a streaming-cache handle (moe_stream_create).
+ *   - Device calls are asynchronous on the given stream and do not
+ *     synchronise unless stated.  Inputs are never modified.
+ *   - Every call returns a moe_status.  On MOE_OK all outputs are fully
+ *     written (once the stream reaches them); on an error they are
+ *     unspecified.  moe_last_error() gives a message for the last failing
+ *     call on the calling host thread.
+ *   - bf16 tensors are passed as 16-bit patterns (void*), row-major.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad index */
+  MOE_ERR_UNSUPPORTED = 2, /* bits not 2/4, group not 64, H or I not a multiple of 64, K > E, T too large for the path */
+  MOE_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the size query says */
+  MOE_ERR_CUDA = 4,        /* a CUDA runtime call failed (message has the CUDA error) */
+  MOE_ERR_OOM = 5,         /* a device or pinned-host allocation failed */
+  MOE_ERR_TIMEOUT = 6,     /* a bounded device-side wait expired (see moe_device_error) */
+  MOE_ERR_IO = 7,          /* a host-store copy of the streaming tier failed */
+  MOE_ERR_DEVICE = 8       /* a device-side check failed (misaligned expert pointer, bad expert id) */
+} moe_status;
+
+/* Layer shape.  hidden H, inter I (expert intermediate size), n_experts E,
+ * top_k K, bits b (4 or 2), group G (64), eps of the RMSNorm (1e-6 in the
+ * synthetic workloads), has_shared (1 = a bf16 shared expert of the same I). */
+typedef struct {
+  int hidden, inter, n_experts, top_k, bits, group;
+  float eps;
+  int has_shared;
+} moe_config;
+
+/* Thread-local message for the last failing call ("" if none). */
+const char* moe_last_error(void);
+
+/* ------------------------------------------------------------------------
+ * Packed expert format (this library's; the pages fix only the size, ~6.75 MB
+ * per 4-bit expert at H=4096, toolarium, section "Flash-MoE: чистый C, Metal и
+ * никакого Python").  One blob per expert, six sections each starting on a
+ * 256-byte boundary:
+ *   0 gate codes [I][H*b/8]   1 up codes [I][H*b/8]   2 down codes [H][I*b/8]
+ *   3 gate scales [I][H/G]    4 up scales [I][H/G]    5 down scales [H][I/G]
+ * Codes: row-major; little-endian 32-bit words; word j of a row holds columns
+ * j*(32/b) .. j*(32/b)+32/b-1, column j*(32/b)+n at bits n*b .. n*b+b-1.
+ * Scale word (uint32): bf16 scale s in bits 0..15, bf16 bias beta in bits
+ * 16..31; weight = q*s + beta.  Groups run along the input (reduction) dim.
+ * Quantiser (round-to-nearest affine, single precision):
+ *   s = bf16_rne((max-min)/(2^b-1)), beta = bf16_rne(min),
+ *   q = clamp(rint((w - beta)/s), 0, 2^b-1), q = 0 when s == 0.
+ * Blob size: moe_packed_expert_bytes (7,077,888 B at H=4096, I=1024, 4-bit;
+ * 3,932,160 B at 2-bit).  Blobs handed to the device calls must start on a
+ * 256-byte boundary.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of one packed expert; 0 if cfg is unsupported. */
+size_t moe_packed_expert_bytes(const moe_config* cfg);
+
+/* Byte offsets of the six sections inside a blob. */
+moe_status moe_packed_layout(const moe_config* cfg, size_t offsets[6]);
+
+/* Host packer (the pages' offline repacking scripts for 4-bit and 2-bit
+ * experts, hakusoku, section "プロジェクト構成").  w_gate, w_up: fp32
+ * [*][I][H]; w_down: fp32 [*][H][I] (host).  Packs experts e_begin ..
+ * e_begin+e_count-1 of those arrays into out (host, e_count consecutive blobs
+ * of moe_packed_expert_bytes each; out_bytes must be at least that).
+ * Inputs must be finite.  Synchronous, multi-threaded over experts. */
+moe_status moe_pack_experts(const moe_config* cfg, const float* w_gate, const float* w_up,
+                            const float* w_down, int e_begin, int e_count, void* out,
+                            size_t out_bytes);
+
+/* Device packer: the same format and bit-identical output as
+ * moe_pack_experts, computed on the GPU.  w_gate, w_up: fp32 [e_count][I][H],
+ * w_down: fp32 [e_count][H][I] (device); out: device, e_count blobs. */
+moe_status moe_pack_experts_device(const moe_config* cfg, const float* w_gate,
+                                   const float* w_up, const float* w_down, int e_count,
+                                   void* out, size_t out_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Router (toolarium, section "Mixture of Experts и почему SSD достаточно";
+ * hakusoku, section "パイプライン概要").
+ *   logits[t][e] = sum_h x[t][h]*Wr[e][h] (fp32 accumulation) + bias[e]
+ *   idx[t][0..K-1]: the K largest logits, descending, ties to the lower index
+ *     (a NaN logit ranks as -inf)
+ *   w[t][k] = exp(l_k - l_max) / sum_j exp(l_j - l_max) over the K chosen
+ *     (= softmax over E renormalised over the K).
+ * x_bf16 [T][H], wr_bf16 [E][H], bias fp32 [E] or NULL, idx int32 [T][K],
+ * w fp32 [T][K], logits_out fp32 [T][E] or NULL: all device.  If logits_out
+ * is NULL the logits go to workspace (moe_router_workspace_bytes). */
+size_t moe_router_workspace_bytes(const moe_config* cfg, int T);
+moe_status moe_router_topk(const moe_config* cfg, const void* x_bf16, const void* wr_bf16,
+                           const float* bias, int T, int32_t* idx, float* w,
+                           float* logits_out, void* workspace, size_t ws_bytes,
+                           cudaStream_t stream);
+
+/* Top-K and weights from given fp32 logits [T][E] (device), same rules. */
+moe_status moe_topk_from_logits(const moe_config* cfg, const float* logits, int T,
+                                int32_t* idx, float* w, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Whole layer.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const void* const* expert_ptr; /* device array [E] of device pointers, one packed blob per expert (256-B aligned) */
+  const void* router_w;          /* bf16 [E][H] */
+  const float* router_bias;      /* fp32 [E] or NULL */
+  const void* shared_gate;       /* bf16 [I][H]; ignored when has_shared == 0 */
+  const void* shared_up;         /* bf16 [I][H] */
+  const void* shared_down;       /* bf16 [H][I] */
+  const void* gamma;             /* bf16 [H], RMSNorm weight */
+} moe_layer_weights;
+
+/* Workspace for moe_layer_forward with T tokens (device memory, 256-B
+ * aligned).  It must be zero-filled once before its first use
+ * (moe_workspace_init); the layer leaves it ready for the next call.  One
+ * workspace serves one call at a time: calls that overlap on the GPU must use
+ * different workspaces. */
+size_t moe_layer_workspace_bytes(const moe_config* cfg, int T);
+moe_status moe_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* One MoE layer for T tokens (device pointers):
+ *   h_out[t]  = residual[t] + sum_k w[t][k] * expert_{idx[t][k]}(x[t]) + shared(x[t])
+ *   y_norm[t] = h_out[t] / sqrt(mean(h_out[t]^2) + eps) * gamma
+ * expert_e(x) = Wd_e (silu(Wg_e x) * (Wu_e x)) with dequantised weights.
+ * x_bf16, residual_bf16 [T][H]; h_out_bf16, y_norm_bf16 [T][H] (y_norm is
+ * computed from the fp32 sum, before h_out is rounded to bf16); idx_out
+ * int32 [T][K] and w_out fp32 [T][K] may be NULL.  T == 0 is a no-op.
+ * T <= 8 runs the fused single-launch decode kernel.  A bounded device wait
+ * that expires leaves MOE_ERR_TIMEOUT in the workspace (moe_device_error). */
+moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts,
+                             const void* x_bf16, const void* residual_bf16, int T,
+                             void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
+                             float* w_out, void* workspace, size_t ws_bytes,
+                             cudaStream_t stream);
+
+/* The same call with HOST activations: copies x and residual (host, pinned
+ * for asynchronous copies) to device staging inside the workspace, runs the
+ * layer, copies h_out and y_norm back to host, and synchronises the stream
+ * before returning.  Workspace size: moe_layer_host_workspace_bytes. */
+size_t moe_layer_host_workspace_bytes(const moe_config* cfg, int T);
+moe_status moe_layer_forward_host(const moe_config* cfg, const moe_layer_weights* wts,
+                                  const void* x_bf16_host, const void* residual_bf16_host,
+                                  int T, void* h_out_bf16_host, void* y_norm_bf16_host,
+                                  void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Read (synchronising the stream) and clear the device-side error word of a
+ * layer workspace.  Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE;
+ * *detail (may be NULL) gets the raw code. */
+moe_status moe_device_error(void* workspace, uint32_t* detail, cudaStream_t stream);
+
+/* Self-test of the bounded device-side wait (no counterpart on the pages):
+ * launches a tiny kernel that waits, with the given limit in nanoseconds, on
+ * a counter of the workspace that nothing increments.  The wait must give up,
+ * record MOE_ERR_TIMEOUT in the workspace's error word (read it with
+ * moe_device_error) and return, leaving the GPU context usable.  The first
+ * 256 bytes of the workspace must be zero (moe_workspace_init). */
+moe_status moe_selftest_bounded_wait(void* workspace, size_t ws_bytes, uint64_t timeout_ns,
+                                     cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

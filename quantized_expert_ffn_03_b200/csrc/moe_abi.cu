@@ -1,0 +1,366 @@
+// moe_abi.cu -- the extern "C" entry points of libmoe: argument checks,
+// workspace carving and kernel launches.  See include/moe.h for the contract.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/moe.h"
+#include "moe_kernels.h"
+
+namespace moe {
+void pack_host(const Layout& L, const float* wg, const float* wu, const float* wd, int e_begin,
+               int e_count, uint8_t* out);
+}
+
+using namespace moe;
+
+namespace {
+
+thread_local std::string g_err;
+
+moe_status fail(moe_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+moe_status bad_shape(const moe_config* cfg) {
+  if (!cfg) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  return fail(MOE_ERR_UNSUPPORTED,
+              "unsupported shape: bits=%d (2 or 4), group=%d (64), hidden=%d and inter=%d "
+              "(positive multiples of 64)",
+              cfg->bits, cfg->group, cfg->hidden, cfg->inter);
+}
+
+moe_status ok() {
+  g_err.clear();
+  return MOE_OK;
+}
+
+#define CUDA_TRY(call)                                                                       \
+  do {                                                                                       \
+    cudaError_t e_ = (call);                                                                 \
+    if (e_ != cudaSuccess)                                                                   \
+      return fail(MOE_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));             \
+  } while (0)
+
+constexpr int kMaxGrid = 1024;
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status check_cfg(const moe_config* cfg, Layout* L) {
+  if (!cfg) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->n_experts <= 0 || cfg->top_k <= 0)
+    return fail(MOE_ERR_INVALID_ARG, "n_experts and top_k must be positive");
+  if (!make_layout(cfg->hidden, cfg->inter, cfg->n_experts, cfg->top_k, cfg->bits, cfg->group,
+                   cfg->has_shared, cfg->eps, L))
+    return fail(MOE_ERR_UNSUPPORTED,
+                "unsupported shape: bits=%d (2 or 4), group=%d (64), hidden=%d and inter=%d "
+                "(positive multiples of 64)",
+                cfg->bits, cfg->group, cfg->hidden, cfg->inter);
+  if (cfg->top_k > cfg->n_experts) return fail(MOE_ERR_UNSUPPORTED, "top_k > n_experts");
+  if (cfg->top_k > kMaxK) return fail(MOE_ERR_UNSUPPORTED, "top_k > %d", kMaxK);
+  if (cfg->hidden > 16384 || cfg->inter > 16384)
+    return fail(MOE_ERR_UNSUPPORTED, "hidden and inter must be <= 16384");
+  return MOE_OK;
+}
+
+int team_warps(int cols) {
+  int need = (cols + 1023) / 1024, tw = 1;
+  while (tw < need) tw *= 2;
+  return tw;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+};
+
+moe_status device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev].sms == 0) {
+    int sms = 0;
+    CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    cache[dev].sms = sms;
+  }
+  *out = cache[dev];
+  return MOE_OK;
+}
+
+struct WsPlan {
+  size_t logits, hs, he, ss, total;
+};
+
+WsPlan ws_plan(const Layout& L, int T) {
+  WsPlan w;
+  size_t pos = 256;
+  w.logits = pos;
+  pos = round_up_256(pos + sizeof(float) * (size_t)T * L.E);
+  w.hs = pos;
+  pos = round_up_256(pos + sizeof(float) * (size_t)T * L.I);
+  w.he = pos;
+  pos = round_up_256(pos + sizeof(float) * (size_t)T * L.K * L.I);
+  w.ss = pos;
+  pos = round_up_256(pos + sizeof(float) * (size_t)T * kMaxGrid);
+  w.total = pos;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_err.c_str(); }
+
+size_t moe_packed_expert_bytes(const moe_config* cfg) {
+  Layout L;
+  if (!cfg || !make_layout(cfg->hidden, cfg->inter, 1, 1, cfg->bits, cfg->group, 0, 0.f, &L)) return 0;
+  return (size_t)L.blob_bytes;
+}
+
+moe_status moe_packed_layout(const moe_config* cfg, size_t offsets[6]) {
+  Layout L;
+  if (!offsets) return fail(MOE_ERR_INVALID_ARG, "offsets is NULL");
+  if (!cfg || !make_layout(cfg->hidden, cfg->inter, 1, 1, cfg->bits, cfg->group, 0, 0.f, &L))
+    return bad_shape(cfg);
+  for (int m = 0; m < 3; ++m) {
+    offsets[m] = L.off_codes[m];
+    offsets[3 + m] = L.off_scales[m];
+  }
+  return ok();
+}
+
+moe_status moe_pack_experts(const moe_config* cfg, const float* w_gate, const float* w_up,
+                            const float* w_down, int e_begin, int e_count, void* out,
+                            size_t out_bytes) {
+  Layout L;
+  if (!cfg || !make_layout(cfg->hidden, cfg->inter, 1, 1, cfg->bits, cfg->group, 0, 0.f, &L))
+    return bad_shape(cfg);
+  if (e_begin < 0 || e_count < 0) return fail(MOE_ERR_INVALID_ARG, "negative expert range");
+  if (e_count == 0) return ok();
+  if (!w_gate || !w_up || !w_down || !out) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (out_bytes < (size_t)L.blob_bytes * e_count)
+    return fail(MOE_ERR_INVALID_ARG, "out_bytes %zu < %zu", out_bytes, (size_t)L.blob_bytes * e_count);
+  pack_host(L, w_gate, w_up, w_down, e_begin, e_count, static_cast<uint8_t*>(out));
+  return ok();
+}
+
+moe_status moe_pack_experts_device(const moe_config* cfg, const float* w_gate,
+                                   const float* w_up, const float* w_down, int e_count,
+                                   void* out, size_t out_bytes, cudaStream_t stream) {
+  Layout L;
+  if (!cfg || !make_layout(cfg->hidden, cfg->inter, 1, 1, cfg->bits, cfg->group, 0, 0.f, &L))
+    return bad_shape(cfg);
+  if (e_count < 0) return fail(MOE_ERR_INVALID_ARG, "negative expert count");
+  if (e_count == 0) return ok();
+  if (!w_gate || !w_up || !w_down || !out) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) || !aligned(out, 16))
+    return fail(MOE_ERR_INVALID_ARG, "device packer pointers must be 16-byte aligned");
+  if (out_bytes < (size_t)L.blob_bytes * e_count)
+    return fail(MOE_ERR_INVALID_ARG, "out_bytes %zu < %zu", out_bytes, (size_t)L.blob_bytes * e_count);
+  CUDA_TRY(launch_pack(L, w_gate, w_up, w_down, e_count, static_cast<uint8_t*>(out), stream));
+  return ok();
+}
+
+size_t moe_router_workspace_bytes(const moe_config* cfg, int T) {
+  if (!cfg || T < 0 || cfg->n_experts <= 0) return 0;
+  return (size_t)round_up_256(sizeof(float) * (size_t)T * cfg->n_experts);
+}
+
+moe_status moe_topk_from_logits(const moe_config* cfg, const float* logits, int T, int32_t* idx,
+                                float* w, cudaStream_t stream) {
+  if (!cfg) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->n_experts <= 0 || cfg->top_k <= 0 || T < 0) return fail(MOE_ERR_INVALID_ARG, "bad sizes");
+  if (cfg->top_k > cfg->n_experts || cfg->top_k > kMaxK) return fail(MOE_ERR_UNSUPPORTED, "top_k");
+  if (T == 0) return ok();
+  if (!logits || !idx || !w) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  CUDA_TRY(launch_topk(logits, T, cfg->n_experts, cfg->top_k, idx, w, stream));
+  return ok();
+}
+
+moe_status moe_router_topk(const moe_config* cfg, const void* x_bf16, const void* wr_bf16,
+                           const float* bias, int T, int32_t* idx, float* w, float* logits_out,
+                           void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  Layout L;
+  moe_status s = check_cfg(cfg, &L);
+  if (s != MOE_OK) return s;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+  if (T == 0) return ok();
+  if (!x_bf16 || !wr_bf16 || !idx || !w) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(x_bf16, 16) || !aligned(wr_bf16, 16))
+    return fail(MOE_ERR_INVALID_ARG, "x and router weights must be 16-byte aligned");
+  float* logits = logits_out;
+  if (!logits) {
+    if (!workspace || ws_bytes < moe_router_workspace_bytes(cfg, T))
+      return fail(MOE_ERR_WORKSPACE, "router workspace too small (need %zu)",
+                  moe_router_workspace_bytes(cfg, T));
+    logits = static_cast<float*>(workspace);
+  }
+  DeviceInfo di;
+  if ((s = device_info(&di)) != MOE_OK) return s;
+  const int tw = team_warps(L.H);
+  const int rows_per_block = (kThreads / 32 / tw) * 4;
+  int grid = (L.E + rows_per_block - 1) / rows_per_block;
+  if (grid > di.sms) grid = di.sms;
+  CUDA_TRY(launch_router_logits(static_cast<const uint16_t*>(x_bf16), static_cast<const uint16_t*>(wr_bf16),
+                                bias, T, L.H, L.E, tw, grid, logits, stream));
+  CUDA_TRY(launch_topk(logits, T, L.E, L.K, idx, w, stream));
+  return ok();
+}
+
+size_t moe_layer_workspace_bytes(const moe_config* cfg, int T) {
+  Layout L;
+  if (!cfg || T < 0 || cfg->n_experts <= 0 || cfg->top_k <= 0) return 0;
+  if (!make_layout(cfg->hidden, cfg->inter, cfg->n_experts, cfg->top_k, cfg->bits, cfg->group,
+                   cfg->has_shared, cfg->eps, &L))
+    return 0;
+  return ws_plan(L, T).total;
+}
+
+moe_status moe_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!workspace || ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace missing or < 256 bytes");
+  CUDA_TRY(cudaMemsetAsync(workspace, 0, ws_bytes, stream));
+  return ok();
+}
+
+moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts,
+                             const void* x_bf16, const void* residual_bf16, int T,
+                             void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out, float* w_out,
+                             void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  Layout L;
+  moe_status s = check_cfg(cfg, &L);
+  if (s != MOE_OK) return s;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+  if (T == 0) return ok();
+  if (T > kMaxTokensFused)
+    return fail(MOE_ERR_UNSUPPORTED, "T=%d: the fused decode path takes at most %d tokens", T,
+                kMaxTokensFused);
+  if (T * L.K > 64) return fail(MOE_ERR_UNSUPPORTED, "T*top_k must be <= 64");
+  if (!wts || !wts->expert_ptr || !wts->router_w || !wts->gamma || !x_bf16 || !residual_bf16 ||
+      !h_out_bf16 || !y_norm_bf16)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (L.has_shared && (!wts->shared_gate || !wts->shared_up || !wts->shared_down))
+    return fail(MOE_ERR_INVALID_ARG, "has_shared=1 but a shared-expert pointer is NULL");
+  const void* a16[] = {x_bf16, residual_bf16, h_out_bf16, y_norm_bf16, wts->router_w, wts->gamma};
+  for (const void* p : a16)
+    if (!aligned(p, 16)) return fail(MOE_ERR_INVALID_ARG, "bf16 arrays must be 16-byte aligned");
+  if (L.has_shared && (!aligned(wts->shared_gate, 16) || !aligned(wts->shared_up, 16) ||
+                       !aligned(wts->shared_down, 16)))
+    return fail(MOE_ERR_INVALID_ARG, "shared-expert weights must be 16-byte aligned");
+  const WsPlan wp = ws_plan(L, T);
+  if (!workspace || ws_bytes < wp.total || !aligned(workspace, 256))
+    return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned and >= %zu bytes", wp.total);
+  DeviceInfo di;
+  if ((s = device_info(&di)) != MOE_OK) return s;
+  const int grid = di.sms < kMaxGrid ? di.sms : kMaxGrid;
+  const int nrows_max = (L.H + grid - 1) / grid;
+  const size_t smem = decode_smem_bytes(T, L.K, nrows_max);
+  if (smem > 200 * 1024) return fail(MOE_ERR_UNSUPPORTED, "shape needs %zu B of shared memory", smem);
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeParams p;
+  p.L = L;
+  p.T = T;
+  p.tw_h = team_warps(L.H);
+  p.tw_i = team_warps(L.I);
+  p.expert_ptr = wts->expert_ptr;
+  p.wr = static_cast<const uint16_t*>(wts->router_w);
+  p.bias = wts->router_bias;
+  p.sg = static_cast<const uint16_t*>(wts->shared_gate);
+  p.su = static_cast<const uint16_t*>(wts->shared_up);
+  p.sd = static_cast<const uint16_t*>(wts->shared_down);
+  p.gamma = static_cast<const uint16_t*>(wts->gamma);
+  p.x = static_cast<const uint16_t*>(x_bf16);
+  p.res = static_cast<const uint16_t*>(residual_bf16);
+  p.h_out = static_cast<uint16_t*>(h_out_bf16);
+  p.y_norm = static_cast<uint16_t*>(y_norm_bf16);
+  p.idx_out = idx_out;
+  p.w_out = w_out;
+  p.ctr = reinterpret_cast<uint32_t*>(ws);
+  p.err = reinterpret_cast<uint32_t*>(ws + 64);
+  p.logits = reinterpret_cast<float*>(ws + wp.logits);
+  p.hs = reinterpret_cast<float*>(ws + wp.hs);
+  p.he = reinterpret_cast<float*>(ws + wp.he);
+  p.ss = reinterpret_cast<float*>(ws + wp.ss);
+  p.timeout_ns = kTimeoutNs;
+  CUDA_TRY(launch_decode(p, grid, smem, stream));
+  return ok();
+}
+
+size_t moe_layer_host_workspace_bytes(const moe_config* cfg, int T) {
+  const size_t base = moe_layer_workspace_bytes(cfg, T);
+  if (base == 0) return 0;
+  const size_t act = (size_t)round_up_256(2ull * (size_t)T * cfg->hidden);
+  return base + 4 * act;
+}
+
+moe_status moe_layer_forward_host(const moe_config* cfg, const moe_layer_weights* wts,
+                                  const void* x_bf16_host, const void* residual_bf16_host, int T,
+                                  void* h_out_bf16_host, void* y_norm_bf16_host, void* workspace,
+                                  size_t ws_bytes, cudaStream_t stream) {
+  if (!cfg) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+  if (T == 0) return ok();
+  if (!x_bf16_host || !residual_bf16_host || !h_out_bf16_host || !y_norm_bf16_host)
+    return fail(MOE_ERR_INVALID_ARG, "NULL host pointer");
+  const size_t base = moe_layer_workspace_bytes(cfg, T);
+  const size_t need = moe_layer_host_workspace_bytes(cfg, T);
+  if (base == 0) return bad_shape(cfg);
+  if (!workspace || ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "host-path workspace must be >= %zu bytes", need);
+  const size_t bytes = 2ull * (size_t)T * cfg->hidden;
+  const size_t act = (size_t)round_up_256(bytes);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* dx = ws + base;
+  void* dr = ws + base + act;
+  void* dh = ws + base + 2 * act;
+  void* dy = ws + base + 3 * act;
+  CUDA_TRY(cudaMemcpyAsync(dx, x_bf16_host, bytes, cudaMemcpyHostToDevice, stream));
+  CUDA_TRY(cudaMemcpyAsync(dr, residual_bf16_host, bytes, cudaMemcpyHostToDevice, stream));
+  moe_status s = moe_layer_forward(cfg, wts, dx, dr, T, dh, dy, nullptr, nullptr, workspace, base, stream);
+  if (s != MOE_OK) return s;
+  CUDA_TRY(cudaMemcpyAsync(h_out_bf16_host, dh, bytes, cudaMemcpyDeviceToHost, stream));
+  CUDA_TRY(cudaMemcpyAsync(y_norm_bf16_host, dy, bytes, cudaMemcpyDeviceToHost, stream));
+  CUDA_TRY(cudaStreamSynchronize(stream));
+  return ok();
+}
+
+moe_status moe_device_error(void* workspace, uint32_t* detail, cudaStream_t stream) {
+  if (!workspace) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  uint32_t code = 0;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  CUDA_TRY(cudaMemcpyAsync(&code, ws + 64, 4, cudaMemcpyDeviceToHost, stream));
+  CUDA_TRY(cudaStreamSynchronize(stream));
+  if (code != 0) {
+    CUDA_TRY(cudaMemsetAsync(ws + 64, 0, 4, stream));
+    CUDA_TRY(cudaStreamSynchronize(stream));
+  }
+  if (detail) *detail = code;
+  if (code == 0) return ok();
+  if (code == 1) return fail(MOE_ERR_TIMEOUT, "a bounded device-side wait expired");
+  return fail(MOE_ERR_DEVICE, "device-side check failed (code %u: bad or misaligned expert pointer)", code);
+}
+
+moe_status moe_selftest_bounded_wait(void* workspace, size_t ws_bytes, uint64_t timeout_ns,
+                                     cudaStream_t stream) {
+  if (!workspace || ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace missing or < 256 bytes");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  CUDA_TRY(launch_barrier_timeout_probe(reinterpret_cast<uint32_t*>(ws), reinterpret_cast<uint32_t*>(ws + 64),
+                                        timeout_ns, stream));
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// moe_kernels.h -- host-side declarations of the kernels' launch wrappers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe_layout.h"
+
+namespace moe {
+
+// Workspace of a layer call: counters and error word first, then fp32
+// intermediates.  ctr[0] router, [1] shared gate/up, [2] routed gate/up,
+// [3] down, [4] blocks that exited, [5] abort flag of the running launch.
+struct DecodeParams {
+  Layout L;
+  int T;
+  int tw_h, tw_i;  // warps per team for H-wide and I-wide rows
+  const void* const* expert_ptr;
+  const uint16_t* wr;
+  const float* bias;
+  const uint16_t* sg;
+  const uint16_t* su;
+  const uint16_t* sd;
+  const uint16_t* gamma;
+  const uint16_t* x;
+  const uint16_t* res;
+  uint16_t* h_out;
+  uint16_t* y_norm;
+  int32_t* idx_out;
+  float* w_out;
+  uint32_t* ctr;
+  uint32_t* err;
+  float* logits;  // [T][E]
+  float* hs;      // [T][I]
+  float* he;      // [T][K][I]
+  float* ss;      // [grid][T]
+  uint64_t timeout_ns;
+};
+
+size_t decode_smem_bytes(int T, int K, int nrows);
+cudaError_t launch_decode(const DecodeParams& p, int grid, size_t smem, cudaStream_t st);
+cudaError_t decode_occupancy(int bits, size_t smem, int* blocks_per_sm);
+cudaError_t launch_barrier_timeout_probe(uint32_t* ctr, uint32_t* err, uint64_t timeout_ns,
+                                         cudaStream_t st);
+
+// Stand-alone router: logits into `logits` ([T][E]), then top-K.
+cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* wr, const float* bias, int T,
+                                 int H, int E, int tw, int grid, float* logits, cudaStream_t st);
+cudaError_t launch_topk(const float* logits, int T, int E, int K, int32_t* idx, float* w,
+                        cudaStream_t st);
+
+// Device packer: e_count experts, fp32 weights [e][I][H], [e][I][H], [e][H][I].
+cudaError_t launch_pack(const Layout& L, const float* wg, const float* wu, const float* wd,
+                        int e_count, uint8_t* out, cudaStream_t st);
+
+}  // namespace moe
