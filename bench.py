@@ -50,6 +50,8 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=300)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-graph", action="store_true")
+    p.add_argument("--trace", action="store_true",
+                   help="also print per-phase timestamps of a few traced layer calls")
     return p.parse_args(argv)
 
 
@@ -262,6 +264,41 @@ def build_replica(M, s, replica, T, chunk=32):
     return r
 
 
+TRACE_NAMES = ["start", "router_done", "shared_gu_done", "expert_gu_done", "wait_S_done", "wait_E_done",
+               "tiles_done", "wait_D_done", "exit", "producer_topk", "producer_last_copy"]
+
+
+def print_trace(M, reps, cfg, xs, rs, h_out, y_out, stream, P, R, calls=16):
+    """Per-phase timestamps (median over blocks, then over calls), relative
+    to the earliest block start of each call; printed to stderr."""
+    import torch
+    nb = M.moe_layer_trace_blocks()
+    tr = torch.zeros((calls, nb, 64), dtype=torch.int64, device="cuda")
+    with torch.cuda.stream(stream):
+        for i in range(calls):
+            r = reps[i % R]
+            M.moe_layer_forward_traced(cfg, r["wts"], xs[i % P], rs[i % P], h_out[0], y_out[0], tr[i],
+                                       r["ws"], stream=stream)
+        torch.cuda.synchronize()
+    t = tr.cpu().numpy().astype(np.float64)
+    rel = t - t[:, :, 0:1].min(axis=1, keepdims=True)
+    out = {}
+    for k, name in enumerate(TRACE_NAMES):
+        v = rel[:, :, k]
+        out[name] = {"median_us": float(np.median(np.median(v, axis=1)) / 1e3),
+                     "max_us": float(np.median(v.max(axis=1)) / 1e3)}
+    print("trace " + json.dumps(out), file=sys.stderr, flush=True)
+    # per-tile view of block 0 of the last call: (ready, released) per tile
+    # and the producer's publish times, in us after that block's start
+    b0 = t[-1, 0]
+    tiles = [(round((b0[16 + 2 * n] - b0[0]) / 1e3, 2), round((b0[17 + 2 * n] - b0[0]) / 1e3, 2))
+             for n in range(16) if b0[16 + 2 * n] > 0]
+    pub = [round((b0[48 + n] - b0[0]) / 1e3, 2) for n in range(16) if b0[48 + n] > 0]
+    print("trace_block0 tiles=%s publish=%s" % (tiles, pub), file=sys.stderr, flush=True)
+    probe = [round((b0[k] - b0[0]) / 1e3, 3) for k in range(11, 16)]
+    print("trace_block0 first routed gate/up row: %s" % probe, file=sys.stderr, flush=True)
+
+
 def run_ours(args):
     import torch
     import quantized_expert_ffn_03_b200 as M
@@ -355,6 +392,9 @@ def run_ours(args):
             torch.cuda.synchronize()
             warm = e0.elapsed_time(e1) / n1
             del g1
+
+    if args.trace and rank == 0:
+        print_trace(M, reps, cfg, xs, rs, h_out, y_out, stream, P, R)
 
     elapsed_ms, units = aggregate(local_ms, float(args.steps * T), "cuda" if world > 1 else None)
     ms_per_step = elapsed_ms / args.steps

@@ -169,6 +169,24 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts
                              float* w_out, void* workspace, size_t ws_bytes,
                              cudaStream_t stream);
 
+/* Per-phase timing of one layer call, in the spirit of the pages' per-layer
+ * --timing breakdown ("Flash-MoE: ...", section "パイプライン概要"): the same
+ * computation as moe_layer_forward (idx/w outputs omitted), and every block
+ * of the fused kernel writes global-timer stamps in ns to trace[block*64 + k]
+ * (device memory, moe_layer_trace_blocks()*64 entries):
+ * k = 0 start, 1 router rows done, 2 shared gate/up done, 3 routed gate/up
+ * done, 4 shared wait done, 5 routed wait done, 6 last tile done, 7 norm wait
+ * done, 8 exit, 9 producer top-K done, 10 producer issued its last copy;
+ * 16+2n / 17+2n: shared-memory tile n (n < 16) ready / released by the
+ * consumers; 48+n: producer publishes tile n.  Unused entries are left as
+ * they were.  Timestamps perturb nothing else. */
+int moe_layer_trace_blocks(void);
+moe_status moe_layer_forward_traced(const moe_config* cfg, const moe_layer_weights* wts,
+                                    const void* x_bf16, const void* residual_bf16, int T,
+                                    void* h_out_bf16, void* y_norm_bf16, void* workspace,
+                                    size_t ws_bytes, uint64_t* trace, size_t trace_entries,
+                                    cudaStream_t stream);
+
 /* The same call with HOST activations: copies x and residual (host, pinned
  * for asynchronous copies) to device staging inside the workspace, runs the
  * layer, copies h_out and y_norm back to host, and synchronises the stream

@@ -1,7 +1,7 @@
 """Python binding of libmoe: the streaming-experts MoE layer on B200.
 
 Argument marshalling only.  Every computation of the layer runs in the CUDA
-library (``libmoe.so``, built by ``python -m quantized_expert_ffn_03_b200.build``);
+library (``libmoe.so``, built by ``python quantized_expert_ffn_03_b200/build.py``);
 if the library is missing, importing this package raises ImportError.
 Device arguments are torch CUDA tensors (bf16 tensors may be torch.bfloat16
 or 16-bit integer views); host arguments of the host packer are numpy arrays.
@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        "libmoe.so is not built (%s); run `python -m quantized_expert_ffn_03_b200.build`" % LIB_PATH)
+        "libmoe.so is not built (%s); run `python quantized_expert_ffn_03_b200/build.py`" % LIB_PATH)
 
 _lib = C.CDLL(LIB_PATH)
 
@@ -66,6 +66,10 @@ EXPORTS = {
     "moe_layer_host_workspace_bytes": (C.c_size_t, [C.c_void_p, C.c_int]),
     "moe_layer_forward_host": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                          C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "moe_layer_trace_blocks": (C.c_int, []),
+    "moe_layer_forward_traced": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                           C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p,
+                                           C.c_size_t, C.c_void_p]),
     "moe_device_error": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
     "moe_selftest_bounded_wait": (C.c_int, [C.c_void_p, C.c_size_t, C.c_uint64, C.c_void_p]),
 }
@@ -196,6 +200,19 @@ def moe_layer_forward(cfg, wts, x, residual, h_out, y_norm, idx_out=None, w_out=
     _check(_lib.moe_layer_forward(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T, _ptr(h_out),
                                   _ptr(y_norm), _ptr(idx_out), _ptr(w_out), _ptr(workspace),
                                   workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_layer_trace_blocks():
+    return _lib.moe_layer_trace_blocks()
+
+
+def moe_layer_forward_traced(cfg, wts, x, residual, h_out, y_norm, trace, workspace, stream=None):
+    """trace: int64 CUDA tensor of moe_layer_trace_blocks()*16 entries."""
+    T = x.shape[0]
+    _check(_lib.moe_layer_forward_traced(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T,
+                                         _ptr(h_out), _ptr(y_norm), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _ptr(trace),
+                                         trace.numel(), _stream(stream)))
 
 
 def moe_layer_forward_host(cfg, wts, x, residual, h_out, y_norm, workspace, stream=None):

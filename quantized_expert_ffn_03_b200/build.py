@@ -1,6 +1,6 @@
 """Build libmoe.so (CUDA, sm_100a) in the package directory.
 
-    python -m quantized_expert_ffn_03_b200.build [--force]
+    python quantized_expert_ffn_03_b200/build.py [--force]
 
 nvcc cross-compiles for sm_100a without a GPU; the library links the CUDA
 runtime statically so it does not depend on the runtime version loaded by

@@ -236,10 +236,13 @@ moe_status moe_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t str
   return ok();
 }
 
-moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts,
-                             const void* x_bf16, const void* residual_bf16, int T,
-                             void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out, float* w_out,
-                             void* workspace, size_t ws_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weights* wts,
+                                     const void* x_bf16, const void* residual_bf16, int T,
+                                     void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
+                                     float* w_out, void* workspace, size_t ws_bytes,
+                                     void* trace, size_t trace_entries, cudaStream_t stream) {
   Layout L;
   moe_status s = check_cfg(cfg, &L);
   if (s != MOE_OK) return s;
@@ -267,8 +270,11 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts
   if ((s = device_info(&di)) != MOE_OK) return s;
   const int grid = di.sms < kMaxGrid ? di.sms : kMaxGrid;
   const int nrows_max = (L.H + grid - 1) / grid;
-  const size_t smem = decode_smem_bytes(T, L.K, nrows_max);
-  if (smem > 200 * 1024) return fail(MOE_ERR_UNSUPPORTED, "shape needs %zu B of shared memory", smem);
+  const uint32_t slot_bytes = decode_slot_bytes(L, T, nrows_max);
+  if (slot_bytes == 0)
+    return fail(MOE_ERR_UNSUPPORTED, "shape does not fit the fused kernel's shared memory (H=%d, I=%d, T=%d)",
+                L.H, L.I, T);
+  const size_t smem = decode_smem_bytes(L, T, nrows_max, slot_bytes);
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   DecodeParams p;
@@ -295,9 +301,39 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts
   p.hs = reinterpret_cast<float*>(ws + wp.hs);
   p.he = reinterpret_cast<float*>(ws + wp.he);
   p.ss = reinterpret_cast<float*>(ws + wp.ss);
+  if (trace && trace_entries < (size_t)grid * 64)
+    return fail(MOE_ERR_INVALID_ARG, "trace needs %d entries", grid * 64);
   p.timeout_ns = kTimeoutNs;
+  p.slot_bytes = slot_bytes;
+  p.trace = static_cast<uint64_t*>(trace);
   CUDA_TRY(launch_decode(p, grid, smem, stream));
   return ok();
+}
+
+extern "C" {
+
+moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts,
+                             const void* x_bf16, const void* residual_bf16, int T,
+                             void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out, float* w_out,
+                             void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  return layer_forward_impl(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out,
+                            workspace, ws_bytes, nullptr, 0, stream);
+}
+
+int moe_layer_trace_blocks(void) {
+  DeviceInfo di;
+  if (device_info(&di) != MOE_OK) return -1;
+  return di.sms < kMaxGrid ? di.sms : kMaxGrid;
+}
+
+moe_status moe_layer_forward_traced(const moe_config* cfg, const moe_layer_weights* wts,
+                                    const void* x_bf16, const void* residual_bf16, int T,
+                                    void* h_out_bf16, void* y_norm_bf16, void* workspace,
+                                    size_t ws_bytes, uint64_t* trace, size_t trace_entries,
+                                    cudaStream_t stream) {
+  if (!trace) return fail(MOE_ERR_INVALID_ARG, "trace is NULL");
+  return layer_forward_impl(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, nullptr, nullptr,
+                            workspace, ws_bytes, trace, trace_entries, stream);
 }
 
 size_t moe_layer_host_workspace_bytes(const moe_config* cfg, int T) {

@@ -65,53 +65,67 @@ __device__ __forceinline__ void lane_constants(LaneX& lx) {
   lx.corr = c;
 }
 
-// Sum over 32 columns of (2^e + q_i) * x_i for one 4-bit fragment.
+// Sum over 32 columns of (2^e + q_i) * x_i for one 4-bit fragment.  The two
+// codes a rotation exposes multiply two adjacent activations, so each pair is
+// one packed fp32 FMA (fma.rn.f32x2): lane x[2i] pairs with the 256+q code of
+// its word position, x[2i+1] with the 16+q code.
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
 __device__ __forceinline__ float codes_dot_q4(const uint4 q, const LaneX& lx) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-  float a0 = 0.f, a1 = 0.f;
+  float2 acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       const uint32_t r = rotl(w[j], (15 - 8 * p) & 31);
-      a0 = fmaf(magic(r, 0x00078000u, 0x43800000u), lx.x[8 * j + 2 * p], a0);
-      a1 = fmaf(magic(r, 0x00780000u, 0x41800000u), lx.x[8 * j + 2 * p + 1], a1);
+      const float2 c = f2(magic(r, 0x00078000u, 0x43800000u), magic(r, 0x00780000u, 0x41800000u));
+      const float2 xx = f2(lx.x[8 * j + 2 * p], lx.x[8 * j + 2 * p + 1]);
+      if (p & 1)
+        acc1 = __ffma2_rn(c, xx, acc1);
+      else
+        acc0 = __ffma2_rn(c, xx, acc0);
     }
   }
-  return a0 + a1;
+  return (acc0.x + acc1.x) + (acc0.y + acc1.y);
 }
 
-// Same for a 2-bit fragment (two words, 32 codes).
+// Same for a 2-bit fragment (two words, 32 codes): codes 4p..4p+3 of a word
+// sit at bits 15, 17, 19, 21 after one rotation (256+q, 64+q, 16+q, 4+q).
 __device__ __forceinline__ float codes_dot_q2(const uint2 q, const LaneX& lx) {
   const uint32_t w[2] = {q.x, q.y};
-  float a0 = 0.f, a1 = 0.f;
+  float2 acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       const uint32_t r = rotl(w[j], (15 - 8 * p) & 31);
       const float* xx = lx.x + 16 * j + 4 * p;
-      a0 = fmaf(magic(r, 0x00018000u, 0x43800000u), xx[0], a0);
-      a1 = fmaf(magic(r, 0x00060000u, 0x42800000u), xx[1], a1);
-      a0 = fmaf(magic(r, 0x00180000u, 0x41800000u), xx[2], a0);
-      a1 = fmaf(magic(r, 0x00600000u, 0x40800000u), xx[3], a1);
+      acc0 = __ffma2_rn(f2(magic(r, 0x00018000u, 0x43800000u), magic(r, 0x00060000u, 0x42800000u)),
+                        f2(xx[0], xx[1]), acc0);
+      acc1 = __ffma2_rn(f2(magic(r, 0x00180000u, 0x41800000u), magic(r, 0x00600000u, 0x40800000u)),
+                        f2(xx[2], xx[3]), acc1);
     }
   }
-  return a0 + a1;
+  return (acc0.x + acc1.x) + (acc0.y + acc1.y);
 }
 
 __device__ __forceinline__ float bf16_dot(const uint4 (&q)[4], const LaneX& lx) {
-  float a0 = 0.f, a1 = 0.f;
+  float2 acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      a0 = fmaf(__uint_as_float(w[m] << 16), lx.x[8 * j + 2 * m], a0);
-      a1 = fmaf(__uint_as_float(w[m] & 0xffff0000u), lx.x[8 * j + 2 * m + 1], a1);
+      const float2 c = f2(__uint_as_float(w[m] << 16), __uint_as_float(w[m] & 0xffff0000u));
+      const float2 xx = f2(lx.x[8 * j + 2 * m], lx.x[8 * j + 2 * m + 1]);
+      if (m & 1)
+        acc1 = __ffma2_rn(c, xx, acc1);
+      else
+        acc0 = __ffma2_rn(c, xx, acc0);
     }
   }
-  return a0 + a1;
+  return (acc0.x + acc1.x) + (acc0.y + acc1.y);
 }
 
 // ---------------------------------------------------------------------------
@@ -339,7 +353,7 @@ __device__ __forceinline__ bool ranks_before(float ka, int ia, float kb, int ib)
 
 // logits: [E] for this token (read through L2).  Writes idx[K], w[K] from
 // lane 0..K-1 (any memory space).
-__device__ __forceinline__ void warp_topk(const float* logits, int E, int K, int32_t* idx, float* w) {
+static __device__ __noinline__ void warp_topk(const float* logits, int E, int K, int32_t* idx, float* w) {
   const int lane = threadIdx.x & 31;
   float prev_k = INFINITY;
   int prev_i = -1;
@@ -354,6 +368,7 @@ __device__ __forceinline__ void warp_topk(const float* logits, int E, int K, int
       vals[m] = e < E ? rank_key(__ldcg(logits + e)) : -INFINITY;
     }
   }
+#pragma unroll 1
   for (int k = 0; k < K; ++k) {
     // best element of this lane that ranks strictly after the previous pick
     float bk = -INFINITY;
@@ -386,7 +401,9 @@ __device__ __forceinline__ void warp_topk(const float* logits, int E, int K, int
   // weights, computed redundantly by every lane; lane k writes entry k
   const float lmax = sel_k[0];
   float den = 0.f;
+#pragma unroll 1
   for (int k = 0; k < K; ++k) den += expf(sel_k[k] - lmax);
+#pragma unroll 1
   for (int k = 0; k < K; ++k) {
     if (lane == (k & 31)) {
       idx[k] = sel_i[k];
@@ -409,6 +426,105 @@ __device__ __forceinline__ void l2_prefetch(const void* p, size_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
     a += n;
   }
+}
+
+// ---------------------------------------------------------------------------
+// Shared-memory barriers (mbarrier) and bulk copies global -> shared.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// try_wait that lets the hardware suspend the thread for up to hint_ns while
+// the phase is incomplete (it returns as soon as the phase completes), so a
+// waiting warp issues almost no instructions.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for phase `parity` of an mbarrier; false on timeout.
+static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 1023u) == 1023u && globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+}
+
+// Orders this thread's earlier generic-proxy accesses (e.g. an acquire that
+// observed other blocks' stores) before its later bulk copies from global.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Adds `bytes` to the transaction count of the current phase (no arrival).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Bulk copy of `bytes` (multiple of 16) from global `src` (16-byte aligned)
+// to shared `dst` (16-byte aligned); completion is counted on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// L2 policy for data read once per launch: evict it before anything else, so
+// the kernel's code and its small shared data stay in L2 across launches.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// bulk_g2s with an L2 cache-policy hint.
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+      "%4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
 }
 
 }  // namespace moe

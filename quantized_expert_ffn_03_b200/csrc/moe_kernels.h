@@ -36,9 +36,13 @@ struct DecodeParams {
   float* he;      // [T][K][I]
   float* ss;      // [grid][T]
   uint64_t timeout_ns;
+  uint32_t slot_bytes;  // bytes per shared-memory ring slot
+  uint64_t* trace;      // optional [grid][16] phase timestamps (ns), or null
 };
 
-size_t decode_smem_bytes(int T, int K, int nrows);
+constexpr int kDecodeBlockThreads = 512;  // 14 consumer warps, a producer warp, a sync warp
+size_t decode_smem_bytes(const Layout& L, int T, int nrows, uint32_t slot_bytes);
+uint32_t decode_slot_bytes(const Layout& L, int T, int nrows_max);
 cudaError_t launch_decode(const DecodeParams& p, int grid, size_t smem, cudaStream_t st);
 cudaError_t decode_occupancy(int bits, size_t smem, int* blocks_per_sm);
 cudaError_t launch_barrier_timeout_probe(uint32_t* ctr, uint32_t* err, uint64_t timeout_ns,
