@@ -36,7 +36,7 @@ import synth as S  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (4-bit experts, K=4, batch 1)"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["moe_decode.cu", "moe_phases.cuh", "moe_device.cuh", "moe_layout.h", "moe_kernels.h"]
+KERNEL_SOURCES = ["moe_decode.cu", "moe_device.cuh", "moe_layout.h", "moe_kernels.h"]
 
 
 def parse_args(argv=None):
@@ -268,12 +268,16 @@ TRACE_NAMES = ["start", "router_done", "shared_gu_done", "expert_gu_done", "wait
                "tiles_done", "wait_D_done", "exit", "producer_topk", "producer_last_copy"]
 
 
+SPIN_NAMES = ["consumer_slot", "consumer_phase", "consumer_x", "producer_slot", "producer_routing",
+              "sync_arrivals", "sync_grid", "sync_x"]
+
+
 def print_trace(M, reps, cfg, xs, rs, h_out, y_out, stream, P, R, calls=16):
     """Per-phase timestamps (median over blocks, then over calls), relative
     to the earliest block start of each call; printed to stderr."""
     import torch
     nb = M.moe_layer_trace_blocks()
-    tr = torch.zeros((calls, nb, 64), dtype=torch.int64, device="cuda")
+    tr = torch.zeros((calls, nb, 128), dtype=torch.int64, device="cuda")
     with torch.cuda.stream(stream):
         for i in range(calls):
             r = reps[i % R]
@@ -295,8 +299,13 @@ def print_trace(M, reps, cfg, xs, rs, h_out, y_out, stream, P, R, calls=16):
              for n in range(16) if b0[16 + 2 * n] > 0]
     pub = [round((b0[48 + n] - b0[0]) / 1e3, 2) for n in range(16) if b0[48 + n] > 0]
     print("trace_block0 tiles=%s publish=%s" % (tiles, pub), file=sys.stderr, flush=True)
-    probe = [round((b0[k] - b0[0]) / 1e3, 3) for k in range(11, 16)]
-    print("trace_block0 first routed gate/up row: %s" % probe, file=sys.stderr, flush=True)
+    probe = [round((b0[k] - b0[0]) / 1e3, 3) for k in range(11, 15)]
+    print("trace_block0 first routed units (gate/up start, end, down start, end): %s" % probe,
+          file=sys.stderr, flush=True)
+    sync = {k: round(float(np.median(rel[:, :, k])) / 1e3, 3) for k in range(64, 74)}
+    print("trace sync warp (median us): %s" % json.dumps(sync), file=sys.stderr, flush=True)
+    polls = {SPIN_NAMES[k]: float(np.median(t[:, :, 80 + k])) for k in range(8)}
+    print("trace polls per block (median): %s" % json.dumps(polls), file=sys.stderr, flush=True)
 
 
 def run_ours(args):

@@ -26,7 +26,7 @@ static size_t round_up_256(size_t n) { return (n + 255u) & ~(size_t)255u; }
 
 static int cfg_ok(const orc_cfg* c) {
   if (c->bits != 2 && c->bits != 4) return 0;
-  if (c->group <= 0 || c->hidden <= 0 || c->inter <= 0) return 0;
+  if (c->group != 64 || c->hidden <= 0 || c->inter <= 0) return 0; /* layout blocks are 8 x 64 */
   if (c->hidden % c->group || c->inter % c->group) return 0;
   /* whole 32-bit code words per row */
   if ((c->hidden * c->bits) % 32 || (c->inter * c->bits) % 32) return 0;
@@ -128,27 +128,66 @@ static void quantize_group(const float* w, int n, int bits, uint16_t* s_out,
   *b_out = beta;
 }
 
-static void put_code(uint8_t* row, int col, int bits, int q) {
-  int per_word = 32 / bits;
-  int word = col / per_word, n = col % per_word;
+/* Where code (row, col) of a [rows][cols] matrix lives: byte offset of its
+ * 32-bit little-endian word inside the code section, and its bit position.
+ * Blocks of 8 rows x 64 columns, row-block major then column group; a block
+ * holds 64*b bytes, 64*b/32 bytes per "lane" l = 4*(row % 8) + t.  Inside the
+ * group, column c = 16*s + cc (k-step s = 0..3):
+ *   cc in 0..7 : t = cc / 2, e = cc % 2, "first" slot;  cc in 8..15:
+ *   t = (cc - 8) / 2, e = cc % 2, "second" slot.
+ * 4-bit: word h = s / 2 of the lane, j = s % 2; first slot nibble 2j + 4e,
+ *        second slot nibble 2j + 1 + 4e.
+ * 2-bit: the lane's single word; first slot code 2s + 8e, second slot code
+ *        2s + 1 + 8e.
+ * (This places the four codes a lane needs for one 16-column step of a
+ * tensor-core B fragment in one word; the dequantised value is unaffected.) */
+static void code_pos(int bits, int cols, int row, int col, size_t* byte_off, int* shift) {
+  int rb = row / 8, n = row % 8, g = col / 64, cg = col % 64;
+  int s = cg / 16, cc = cg % 16;
+  int second = cc >= 8;
+  int t = (second ? cc - 8 : cc) / 2, e = cc % 2;
+  int lane = 4 * n + t;
+  size_t block = (size_t)rb * (cols / 64) + g;
+  size_t lane_bytes = (size_t)(64 * bits) / 32;
+  size_t off = block * (size_t)(64 * bits) + (size_t)lane * lane_bytes;
+  int m;
+  if (bits == 4) {
+    int h = s / 2, j = s % 2;
+    off += 4 * (size_t)h;
+    m = second ? 2 * j + 1 + 4 * e : 2 * j + 4 * e;
+  } else {
+    m = second ? 2 * s + 1 + 8 * e : 2 * s + 8 * e;
+  }
+  *byte_off = off;
+  *shift = m * bits;
+}
+
+/* Scale word of (row, group): [row block][group][row % 8], 4 bytes each. */
+static size_t scale_pos(int cols, int row, int g) {
+  return (((size_t)(row / 8) * (cols / 64) + g) * 8 + row % 8) * 4;
+}
+
+static void put_code(uint8_t* codes, int cols, int row, int col, int bits, int q) {
+  size_t off;
+  int shift;
+  code_pos(bits, cols, row, col, &off, &shift);
   uint32_t v;
-  memcpy(&v, row + 4 * (size_t)word, 4); /* little-endian host */
-  v |= ((uint32_t)q & ((1u << bits) - 1u)) << (n * bits);
-  memcpy(row + 4 * (size_t)word, &v, 4);
+  memcpy(&v, codes + off, 4); /* little-endian host */
+  v |= ((uint32_t)q & ((1u << bits) - 1u)) << shift;
+  memcpy(codes + off, &v, 4);
 }
 
 static void quantize_matrix(const orc_cfg* c, const float* w, int rows, int cols,
                             uint8_t* codes, uint8_t* scales) {
   int G = c->group, b = c->bits;
-  size_t row_bytes = (size_t)cols * b / 8;
   int* q = (int*)malloc(sizeof(int) * G);
   for (int r = 0; r < rows; ++r) {
     for (int g = 0; g < cols / G; ++g) {
       uint16_t s, beta;
       quantize_group(w + (size_t)r * cols + (size_t)g * G, G, b, &s, &beta, q);
-      for (int i = 0; i < G; ++i) put_code(codes + r * row_bytes, g * G + i, b, q[i]);
+      for (int i = 0; i < G; ++i) put_code(codes, cols, r, g * G + i, b, q[i]);
       uint32_t word = (uint32_t)s | ((uint32_t)beta << 16);
-      memcpy(scales + ((size_t)r * (cols / G) + g) * 4, &word, 4);
+      memcpy(scales + scale_pos(cols, r, g), &word, 4);
     }
   }
   free(q);
@@ -180,16 +219,15 @@ static void mat_shape(const orc_cfg* c, int m, int* rows, int* cols) {
 }
 
 int orc_code(const orc_cfg* c, const uint8_t* blob, int m, int row, int col) {
-  size_t off[6];
-  int rows, cols;
+  size_t off[6], pos;
+  int rows, cols, shift;
   orc_section_offsets(c, off);
   mat_shape(c, m, &rows, &cols);
-  int b = c->bits, per_word = 32 / b;
-  const uint8_t* r = blob + off[m] + (size_t)row * ((size_t)cols * b / 8);
+  int b = c->bits;
+  code_pos(b, cols, row, ORC_MUTANT == 2 ? (col ^ 1) : col, &pos, &shift);
   uint32_t v;
-  memcpy(&v, r + 4 * (size_t)(col / per_word), 4);
-  int n = ORC_MUTANT == 2 ? per_word - 1 - col % per_word : col % per_word;
-  return (int)((v >> (n * b)) & ((1u << b) - 1u));
+  memcpy(&v, blob + off[m] + pos, 4);
+  return (int)((v >> shift) & ((1u << b) - 1u));
 }
 
 /* w = q*s + beta, the "(nibble x scale + bias)" form of [toolarium]
@@ -200,7 +238,7 @@ double orc_dequant(const orc_cfg* c, const uint8_t* blob, int m, int row, int co
   orc_section_offsets(c, off);
   mat_shape(c, m, &rows, &cols);
   uint32_t word;
-  memcpy(&word, blob + off[3 + m] + ((size_t)row * (cols / c->group) + col / c->group) * 4, 4);
+  memcpy(&word, blob + off[3 + m] + scale_pos(cols, row, col / c->group), 4);
   double s = orc_bf16_to_f64((uint16_t)(word & 0xffffu));
   double beta = orc_bf16_to_f64((uint16_t)(word >> 16));
   return (double)orc_code(c, blob, m, row, col) * s + (ORC_MUTANT == 1 ? 0.0 : beta);
@@ -335,7 +373,7 @@ static double fma_form_dot(const orc_cfg* c, const uint8_t* blob, int m, int row
   double acc = 0.0;
   for (int k = 0; k < n; ++k) {
     uint32_t word;
-    memcpy(&word, blob + off[3 + m] + ((size_t)row * (n / c->group) + k / c->group) * 4, 4);
+    memcpy(&word, blob + off[3 + m] + scale_pos(n, row, k / c->group), 4);
     double s = orc_bf16_to_f64((uint16_t)(word & 0xffffu));
     double beta = orc_bf16_to_f64((uint16_t)(word >> 16));
     double q = (double)orc_code(c, blob, m, row, k);

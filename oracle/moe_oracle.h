@@ -27,11 +27,14 @@
  *   0 gate codes  [I][H*b/8]     1 up codes   [I][H*b/8]
  *   2 down codes  [H][I*b/8]     3 gate scales [I][H/G] (uint32)
  *   4 up scales   [I][H/G]       5 down scales [H][I/G]
- * Codes are row-major.  Inside a row, little-endian 32-bit words; word j holds
- * columns j*(32/b) ... j*(32/b)+32/b-1, column j*(32/b)+n at bits n*b..n*b+b-1.
- * A scale word holds the bf16 scale s in bits 0..15 and the bf16 bias beta in
- * bits 16..31.  The dequantised weight is q*s + beta ([toolarium] "Оптимизации,
- * которые сработали": the "(nibble x scale + bias)" form).
+ * Codes come in blocks of 8 rows x 64 columns (row-block major, then column
+ * group), 64*b bytes per block; inside a block the four codes that a
+ * tensor-core B fragment takes for one 16-column step share one 32-bit word
+ * (exact positions: code_pos in moe_oracle.c).  Scale words are stored
+ * [row block][group][row % 8]; a scale word holds the bf16 scale s in bits
+ * 0..15 and the bf16 bias beta in bits 16..31.  The dequantised weight is
+ * q*s + beta ([toolarium] "Оптимизации, которые сработали": the "(nibble x
+ * scale + bias)" form).  Group size 64, H and I multiples of 64.
  */
 #ifndef MOE_ORACLE_H
 #define MOE_ORACLE_H

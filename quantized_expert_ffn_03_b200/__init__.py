@@ -207,7 +207,7 @@ def moe_layer_trace_blocks():
 
 
 def moe_layer_forward_traced(cfg, wts, x, residual, h_out, y_norm, trace, workspace, stream=None):
-    """trace: int64 CUDA tensor of moe_layer_trace_blocks()*16 entries."""
+    """trace: int64 CUDA tensor of moe_layer_trace_blocks()*128 entries."""
     T = x.shape[0]
     _check(_lib.moe_layer_forward_traced(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T,
                                          _ptr(h_out), _ptr(y_norm), _ptr(workspace),

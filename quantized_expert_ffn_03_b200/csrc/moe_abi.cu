@@ -71,13 +71,8 @@ moe_status check_cfg(const moe_config* cfg, Layout* L) {
   if (cfg->top_k > kMaxK) return fail(MOE_ERR_UNSUPPORTED, "top_k > %d", kMaxK);
   if (cfg->hidden > 16384 || cfg->inter > 16384)
     return fail(MOE_ERR_UNSUPPORTED, "hidden and inter must be <= 16384");
+  if (cfg->n_experts > 65536) return fail(MOE_ERR_UNSUPPORTED, "n_experts must be <= 65536");
   return MOE_OK;
-}
-
-int team_warps(int cols) {
-  int need = (cols + 1023) / 1024, tw = 1;
-  while (tw < need) tw *= 2;
-  return tw;
 }
 
 struct DeviceInfo {
@@ -101,7 +96,7 @@ moe_status device_info(DeviceInfo* out) {
 }
 
 struct WsPlan {
-  size_t logits, hs, he, ss, total;
+  size_t logits, hs, hf, hx, ss, total;
 };
 
 WsPlan ws_plan(const Layout& L, int T) {
@@ -111,8 +106,10 @@ WsPlan ws_plan(const Layout& L, int T) {
   pos = round_up_256(pos + sizeof(float) * (size_t)T * L.E);
   w.hs = pos;
   pos = round_up_256(pos + sizeof(float) * (size_t)T * L.I);
-  w.he = pos;
-  pos = round_up_256(pos + sizeof(float) * (size_t)T * L.K * L.I);
+  w.hf = pos;
+  pos = round_up_256(pos + 4ull * (size_t)T * L.K * L.I);
+  w.hx = pos;
+  pos = round_up_256(pos + sizeof(float) * (size_t)T * L.K * (L.I / 8));
   w.ss = pos;
   pos = round_up_256(pos + sizeof(float) * (size_t)T * kMaxGrid);
   w.total = pos;
@@ -211,12 +208,10 @@ moe_status moe_router_topk(const moe_config* cfg, const void* x_bf16, const void
   }
   DeviceInfo di;
   if ((s = device_info(&di)) != MOE_OK) return s;
-  const int tw = team_warps(L.H);
-  const int rows_per_block = (kThreads / 32 / tw) * 4;
-  int grid = (L.E + rows_per_block - 1) / rows_per_block;
-  if (grid > di.sms) grid = di.sms;
+  int grid = (L.E + 15) / 16;
+  if (grid > 4 * di.sms) grid = 4 * di.sms;
   CUDA_TRY(launch_router_logits(static_cast<const uint16_t*>(x_bf16), static_cast<const uint16_t*>(wr_bf16),
-                                bias, T, L.H, L.E, tw, grid, logits, stream));
+                                bias, T, L.H, L.E, grid, logits, stream));
   CUDA_TRY(launch_topk(logits, T, L.E, L.K, idx, w, stream));
   return ok();
 }
@@ -269,19 +264,18 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
   DeviceInfo di;
   if ((s = device_info(&di)) != MOE_OK) return s;
   const int grid = di.sms < kMaxGrid ? di.sms : kMaxGrid;
-  const int nrows_max = (L.H + grid - 1) / grid;
-  const uint32_t slot_bytes = decode_slot_bytes(L, T, nrows_max);
+  const int nrows_max = decode_rows_max(L.H, grid);
+  int nslots = 0;
+  const uint32_t slot_bytes = decode_slot_bytes(L, T, nrows_max, &nslots);
   if (slot_bytes == 0)
     return fail(MOE_ERR_UNSUPPORTED, "shape does not fit the fused kernel's shared memory (H=%d, I=%d, T=%d)",
                 L.H, L.I, T);
-  const size_t smem = decode_smem_bytes(L, T, nrows_max, slot_bytes);
+  const size_t smem = decode_smem_bytes(L, T, nrows_max, nslots, slot_bytes);
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   DecodeParams p;
   p.L = L;
   p.T = T;
-  p.tw_h = team_warps(L.H);
-  p.tw_i = team_warps(L.I);
   p.expert_ptr = wts->expert_ptr;
   p.wr = static_cast<const uint16_t*>(wts->router_w);
   p.bias = wts->router_bias;
@@ -299,12 +293,14 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
   p.err = reinterpret_cast<uint32_t*>(ws + 64);
   p.logits = reinterpret_cast<float*>(ws + wp.logits);
   p.hs = reinterpret_cast<float*>(ws + wp.hs);
-  p.he = reinterpret_cast<float*>(ws + wp.he);
+  p.hf = ws + wp.hf;
+  p.hx = reinterpret_cast<float*>(ws + wp.hx);
   p.ss = reinterpret_cast<float*>(ws + wp.ss);
-  if (trace && trace_entries < (size_t)grid * 64)
-    return fail(MOE_ERR_INVALID_ARG, "trace needs %d entries", grid * 64);
+  if (trace && trace_entries < (size_t)grid * 128)
+    return fail(MOE_ERR_INVALID_ARG, "trace needs %d entries", grid * 128);
   p.timeout_ns = kTimeoutNs;
   p.slot_bytes = slot_bytes;
+  p.nslots = nslots;
   p.trace = static_cast<uint64_t*>(trace);
   CUDA_TRY(launch_decode(p, grid, smem, stream));
   return ok();

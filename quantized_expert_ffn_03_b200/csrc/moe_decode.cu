@@ -4,22 +4,34 @@
 // exactly the weight bytes it owns through a ring of shared-memory slots:
 // a producer warp issues bulk copies (cp.async.bulk, completion counted on an
 // mbarrier per slot) and 14 consumer warps compute from shared memory.  A
-// sync warp does the block's grid-wide arrivals and waits and stages the
-// activation vectors, so consumers never stall on a release fence, on
-// polling global memory, or on block-wide barriers between tiles.
+// sync warp prepares the activations, does the block's grid-wide arrivals and
+// waits, runs the router's top-K and stages the intermediates, so consumers
+// never stall on a release fence, on polling global memory, or on block-wide
+// barriers between tiles.
 // The block's byte stream, in order:
 //   router rows  -> [arrive R]  shared gate/up rows  -> [arrive S]
-//   (producer: wait R, top-K, expert pointers)
-//   routed gate/up rows of the chosen experts  -> [arrive E]
+//   (sync warp: wait R, top-K, expert pointers; producer waits for them)
+//   routed gate/up row blocks of the chosen experts  -> [arrive E]
 //   [wait S]  shared down rows of the block's output rows
-//   [wait E]  routed down rows of the block's output rows
+//   [wait E]  routed down row blocks of the block's output rows
 // then combine + residual, a grid-wide sum of squares, and RMSNorm of the
 // block's rows.  The copies that follow a wait are already in flight while a
-// block waits, so HBM stays busy across the waits.
+// block waits, so HBM stays busy across the waits.  Phase arrivals and waits
+// ride on the data tiles as flags, so they take no ring slot of their own.
 //
-// Consumer work unit: one weight row (or the gate/up pair of one row), done
-// entirely by one warp over 1024-column chunks; rows are dealt round-robin to
-// the consumer warps across tiles, and each warp releases a slot on its own.
+// bf16 rows (router, shared expert) are dotted on the CUDA cores, one row per
+// warp.  Packed expert rows go through the tensor cores: mma.sync m16n8k16
+// with the 4/2-bit codes as the B operand (each code becomes the bf16 number
+// 128 + q with two logic ops), the activations as the A operand, and the
+// group's scale and bias applied to the fp32 result:
+//   sum_k x_k (q_k s + beta) = s * D + (beta - 128 s) * X,
+//   D = sum_k x_k (128 + q_k),  X = sum_k x_k  over the group's 64 columns.
+// A "window" is 8 consecutive groups of one 8-row block: A row m carries the
+// activations of group m of the window (zero in the other groups' steps), so
+// after the window's 32 mma steps lane group m holds group m's D for 8
+// weight rows and the scale epilogue is spread over all 32 lanes.  For the
+// down projection the fp32 intermediate is split into bf16 hi + lo parts in
+// A rows 0..7 and 8..15, so it enters at about 16 bits of precision.
 //
 // This is the single-kernel form of the pages' pipeline: router projection
 // with the shared expert (CMD2), top-K, the K expert reads and the deferred
@@ -31,7 +43,7 @@
 #include <cuda_bf16.h>
 
 #include "moe_kernels.h"
-#include "moe_phases.cuh"
+#include "moe_device.cuh"
 
 namespace moe {
 
@@ -43,81 +55,106 @@ constexpr int kProducerWarp = kConsumerWarps;    // warp 14
 constexpr int kSyncWarp = kConsumerWarps + 1;    // warp 15
 constexpr int kDecodeThreads = kConsumers + 64;
 static_assert(kDecodeThreads == kDecodeBlockThreads, "block size");
-constexpr int kSlots = 4;
+constexpr int kSlots = 4;  // ring slots at most (the launch picks 2..4)
 constexpr int kMaxSeg = 8;
 constexpr int kMaxSlotBytes = 48 * 1024;
-constexpr int kTraceEntries = 64;
+constexpr int kTraceEntries = 128;
+// Routed gate/up: at most this many row blocks per tile, and a ring of
+// accumulator entries large enough for every row block of kSlots tiles.
+constexpr int kMaxRbPerTile = 2;
+constexpr int kAccSlots = kSlots * kMaxRbPerTile;
 
-enum TileType : int {
-  TILE_ROUTER = 0,
-  TILE_SHARED_GU,
-  TILE_EXPERT_GU,
-  TILE_SHARED_DOWN,
-  TILE_EXPERT_DOWN,
-  TILE_ARRIVE_R,
-  TILE_ARRIVE_S,
-  TILE_ARRIVE_E,
-  TILE_WAIT_S,
-  TILE_WAIT_E,
-  TILE_END
+enum TileType : int { TILE_NONE = 0, TILE_ROUTER, TILE_SHARED_GU, TILE_EXPERT_GU, TILE_SHARED_DOWN, TILE_EXPERT_DOWN };
+
+// flags carried by a tile: waits done before its compute, arrivals after it
+enum TileFlag : int {
+  F_WAIT_S = 1,
+  F_WAIT_E = 2,
+  F_ARRIVE_R = 4,
+  F_ARRIVE_S = 8,
+  F_ARRIVE_E = 16,
+  F_END = 32
 };
 
 struct Seg {
-  int pair;  // (token, expert) pair of routed tiles
-  int row0;  // first matrix row
-  int nrows;
+  int pair;   // (token, expert) pair of routed tiles
+  int row0;   // bf16 tiles: first matrix row; routed tiles: first 8-row block
+  int nrows;  // bf16 tiles: rows; routed tiles: row blocks
+  int u0, u1; // routed tiles: units of each row block held in the slot
+  int gbase;  // routed tiles: first group held (0 for whole row blocks)
+  int acc;    // routed gate/up: accumulator entry of the first row block
   uint32_t off[4];  // slot byte offset of each range's first valid byte
 };
 
 struct TileDesc {
   int type;
   int nseg;
+  int pre;   // F_WAIT_* flags
+  int post;  // F_ARRIVE_* / F_END flags
   Seg seg[kMaxSeg];
 };
 
 // barriers consumers -> sync warp (evt) and sync warp -> consumers (go)
 enum { EVT_R = 0, EVT_S, EVT_E, EVT_D, NEVT };
 enum { GO_S = 0, GO_E, GO_D, NGO };
+enum { FLAG_TOPK = NGO };  // flags[] slot: routing valid
 
 // ---- shared-memory plan ------------------------------------------------------
-// xq: x in the quantised-row lane layout, permuted so that lane l's j-th
-// 16-byte piece of 1024-column chunk ch sits at unit ((t*nch + ch)*4 + j)*32 + l;
-// xc: (sum x, sum offset*x) of each lane's 32 columns.
+// xf: x as mma A fragments, [token][group][t][8 words]; word 2s is the bf16
+//     pair at columns 16s + 2t (+1) of the group, word 2s+1 the pair at 16s + 8 + 2t.
+// xsum: per (token, group) sum of x.
+// hf: routed intermediate as A fragments (hi/lo), [pair][group][t][step] x 16 bytes.
+// hx: per (pair, 8-row block of I) sum of hi + lo.
 struct DecodeSmem {
-  size_t ring, bars, desc, xs, xq, xc, hs, he, tk_w, tk_i, eptr, ypart, ys, hacc, inv, flags, total;
+  size_t ring, bars, desc, xs, xf, xsum, hs, hf, hx, zero, part, cnt, tk_w, tk_i, eptr, tkbuf, res, gam, ypart,
+      ys, hacc, inv, flags, spin, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
 
-__host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int H, int I, int nrows,
+__host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int E, int H, int I, int nrows, int nslots,
                                                        uint32_t slot_bytes) {
-  const int nch = (H + 1023) / 1024;
+  const RoutedGeo gi = routed_geo(I);
   DecodeSmem s;
   size_t pos = 0;
   s.ring = pos;
-  pos = align_up(pos + (size_t)kSlots * slot_bytes, 128);
-  s.bars = pos;  // full[kSlots], empty[kSlots], xbar, xcbar, evt[NEVT], go[NGO]
-  pos = align_up(pos + 8 * (2 * kSlots + 2 + NEVT + NGO), 16);
+  pos = align_up(pos + (size_t)nslots * slot_bytes, 128);
+  s.bars = pos;  // full[kSlots], empty[kSlots], xbar, xfbar, topkbar, evt[NEVT], go[NGO]
+  pos = align_up(pos + 8 * (2 * kSlots + 3 + NEVT + NGO), 16);
   s.desc = pos;
   pos = align_up(pos + sizeof(TileDesc) * kSlots, 16);
   s.xs = pos;
   pos = align_up(pos + 2ull * T * H, 16);
-  s.xq = pos;
-  pos = align_up(pos + 16ull * T * nch * 128, 16);
-  s.xc = pos;
-  pos = align_up(pos + 8ull * T * nch * 32, 16);
+  s.xf = pos;
+  pos = align_up(pos + 2ull * T * H, 16);
+  s.xsum = pos;
+  pos = align_up(pos + 4ull * T * (H / 64), 16);
   s.hs = pos;
   pos = align_up(pos + 4ull * T * I, 16);
-  s.he = pos;
+  s.hf = pos;
   pos = align_up(pos + 4ull * T * K * I, 16);
+  s.hx = pos;
+  pos = align_up(pos + 4ull * T * K * (I / 8), 16);
+  s.zero = pos;
+  pos = align_up(pos + 64, 16);
+  s.part = pos;
+  pos = align_up(pos + 4ull * kAccSlots * kMaxUnits * 16, 16);
+  s.cnt = pos;
+  pos = align_up(pos + 4ull * kAccSlots, 16);
   s.tk_w = pos;
   pos = align_up(pos + sizeof(float) * T * K, 16);
   s.tk_i = pos;
   pos = align_up(pos + sizeof(int) * T * K, 16);
   s.eptr = pos;
   pos = align_up(pos + sizeof(void*) * T * K, 16);
+  s.tkbuf = pos;
+  pos = align_up(pos + sizeof(uint64_t) * E, 16);
+  s.res = pos;
+  pos = align_up(pos + 2ull * T * nrows, 16);
+  s.gam = pos;
+  pos = align_up(pos + 2ull * nrows, 16);
   s.ypart = pos;
-  pos = align_up(pos + sizeof(float) * T * K * nrows, 16);
+  pos = align_up(pos + sizeof(float) * T * K * gi.U * nrows, 16);
   s.ys = pos;
   pos = align_up(pos + sizeof(float) * T * nrows, 16);
   s.hacc = pos;
@@ -126,12 +163,14 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int H, int 
   pos = align_up(pos + sizeof(float) * T, 16);
   s.flags = pos;
   pos = align_up(pos + 16 * sizeof(int), 16);
+  s.spin = pos;
+  pos = align_up(pos + 16 * sizeof(uint32_t), 16);
   s.total = pos;
   return s;
 }
 
-size_t decode_smem_bytes(const Layout& L, int T, int nrows, uint32_t slot_bytes) {
-  return decode_smem_plan(T, L.K, L.H, L.I, nrows, slot_bytes).total;
+size_t decode_smem_bytes(const Layout& L, int T, int nrows, int nslots, uint32_t slot_bytes) {
+  return decode_smem_plan(T, L.K, L.E, L.H, L.I, nrows, nslots, slot_bytes).total;
 }
 
 // ---- small helpers ----------------------------------------------------------------
@@ -140,133 +179,293 @@ __device__ __forceinline__ void consumer_sync() { named_sync(1, kConsumers); }
 
 // Warp-wide bounded wait on an mbarrier phase: lane 0 polls, the warp
 // synchronises on the result (other lanes see the data through __syncwarp).
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
+                                          uint32_t* spins = nullptr) {
   int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, timeout_ns) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, timeout_ns, spins) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
   return ok != 0;
 }
 
+// Trace stamp k of this block (traced launches only; the untraced kernel
+// carries no trace code).
+template <bool TRACE>
 __device__ __forceinline__ void trace_mark(const DecodeParams& p, int k) {
-  if (p.trace && k < kTraceEntries) p.trace[(size_t)blockIdx.x * kTraceEntries + k] = globaltimer_ns();
+  if constexpr (TRACE) p.trace[(size_t)blockIdx.x * kTraceEntries + k] = globaltimer_ns();
 }
 
+// Share [a, b) of n items for block c of G (n * G < 2^32 for every caller).
 __device__ __forceinline__ void range_of(int n, int c, int G, int& a, int& b) {
-  a = (int)((long long)n * c / G);
-  b = (int)((long long)n * (c + 1) / G);
+  a = (int)((uint32_t)n * (uint32_t)c / (uint32_t)G);
+  b = (int)((uint32_t)n * (uint32_t)(c + 1) / (uint32_t)G);
 }
 
-__device__ __forceinline__ int cap_rows(uint32_t slot_bytes, uint32_t slack, uint32_t per_row) {
-  const int r = (int)((slot_bytes - slack) / per_row);
-  return max(1, min(r, 1024));
-}
 
 // One grid wait by the calling thread only.
 __device__ __forceinline__ bool grid_wait_thread(const uint32_t* ctr, uint32_t target, uint32_t* abort_flag,
-                                                 uint32_t* err, uint64_t timeout_ns) {
+                                                 uint32_t* err, uint64_t timeout_ns, uint32_t* spins = nullptr) {
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (ld_acquire_gpu(ctr) >= target) return true;
-    if (ld_relaxed_gpu(abort_flag) != 0u) return false;
+  bool ok = true;
+  uint32_t it = 0;
+  for (;; ++it) {
+    if (ld_acquire_gpu(ctr) >= target) break;
+    if (ld_relaxed_gpu(abort_flag) != 0u) {
+      ok = false;
+      break;
+    }
     if ((it & 63u) == 63u && (globaltimer_ns() - t0 > timeout_ns || it > (1u << 28))) {
       atomicCAS(err, 0u, 1u);
       atomicExch(abort_flag, 1u);
-      return false;
+      ok = false;
+      break;
     }
   }
+  if (spins) atomicAdd(spins, it + 1);
+  return ok;
 }
 
-// ---- per-lane chunk loads and dots ----------------------------------------------------
-// Chunk ch of a row covers columns [1024*ch, 1024*ch + 1024).
-// bf16 rows: lane l owns columns 1024*ch + 256*j + 8*l + c (j < 4, c < 8), so
-// each 16-byte read of a row (or of x) is contiguous across the warp.
-// Quantised rows: lane l owns the 32 columns of group-half cidx = 32*ch + l.
-
-__device__ __forceinline__ void x_strided_bf16(float (&x)[32], const uint16_t* v, int ch, int cols) {
+// ---- bf16 rows on the CUDA cores -----------------------------------------------------
+// Dot of one bf16 weight row w0 (and w1, the up row of a gate/up pair, if not
+// null) with up to 4 tokens' activations: bf16 x, or the fp32 shared
+// intermediate (xf32).  Lane l owns columns 256k + 8l .. +7, so each 16-byte
+// read of a row is contiguous across the warp.  acc[m][t]: lane partial sums.
+__device__ __forceinline__ void bf16_dot4(const uint8_t* w0, const uint8_t* w1, int cols, const uint8_t* x,
+                                          uint32_t xstride, bool xf32, int nt, float (&acc)[2][4]) {
   const int lane = threadIdx.x & 31;
+  float2 a[2][4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int c0 = ch * 1024 + 256 * j + 8 * lane;
-    if (c0 < cols) {
-      unpack_bf16x8(*reinterpret_cast<const uint4*>(v + c0), x + 8 * j);
-    } else {
+  for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) x[8 * j + c] = 0.f;
-    }
-  }
-}
-
-__device__ __forceinline__ void x_strided_f32(float (&x)[32], const float* v, int ch, int cols) {
-  const int lane = threadIdx.x & 31;
+    for (int tt = 0; tt < 4; ++tt) a[mm][tt] = make_float2(0.f, 0.f);
+#pragma unroll 1
+  for (int c = 8 * lane; c < cols; c += 256) {
+    uint4 q[2];
+    q[0] = *reinterpret_cast<const uint4*>(w0 + 2 * c);
+    q[1] = w1 ? *reinterpret_cast<const uint4*>(w1 + 2 * c) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int c0 = ch * 1024 + 256 * j + 8 * lane;
-    if (c0 < cols) {
-      const float4 a = *reinterpret_cast<const float4*>(v + c0);
-      const float4 b = *reinterpret_cast<const float4*>(v + c0 + 4);
-      x[8 * j + 0] = a.x;
-      x[8 * j + 1] = a.y;
-      x[8 * j + 2] = a.z;
-      x[8 * j + 3] = a.w;
-      x[8 * j + 4] = b.x;
-      x[8 * j + 5] = b.y;
-      x[8 * j + 6] = b.z;
-      x[8 * j + 7] = b.w;
-    } else {
+    for (int tt = 0; tt < 4; ++tt) {
+      if (tt < nt) {
+        float xx[8];
+        if (xf32) {
+          const float4* xp = reinterpret_cast<const float4*>(x + tt * xstride + 4 * c);
+          const float4 u = xp[0], v = xp[1];
+          xx[0] = u.x, xx[1] = u.y, xx[2] = u.z, xx[3] = u.w, xx[4] = v.x, xx[5] = v.y, xx[6] = v.z, xx[7] = v.w;
+        } else {
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(x + tt * xstride + 2 * c), xx);
+        }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) x[8 * j + c] = 0.f;
-    }
-  }
-}
-
-// bf16 row chunk dot (strided lane layout)
-__device__ __forceinline__ float bf16_chunk(const uint8_t* row, int ch, int cols, const float (&x)[32]) {
-  const int lane = threadIdx.x & 31;
-  float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+        for (int mm = 0; mm < 2; ++mm) {
+          if (mm == 0 || w1) {
+            const uint32_t w[4] = {q[mm].x, q[mm].y, q[mm].z, q[mm].w};
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int c0 = ch * 1024 + 256 * j + 8 * lane;
-    if (c0 < cols) {
-      const uint4 q = *reinterpret_cast<const uint4*>(row + 2 * c0);
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float2 c = make_float2(__uint_as_float(w[m] << 16), __uint_as_float(w[m] & 0xffff0000u));
-        const float2 xx = make_float2(x[8 * j + 2 * m], x[8 * j + 2 * m + 1]);
-        if (m & 1)
-          a1 = __ffma2_rn(c, xx, a1);
-        else
-          a0 = __ffma2_rn(c, xx, a0);
+            for (int k = 0; k < 4; ++k)
+              a[mm][tt] = __ffma2_rn(make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u)),
+                                     make_float2(xx[2 * k], xx[2 * k + 1]), a[mm][tt]);
+          }
+        }
       }
     }
   }
-  return (a0.x + a1.x) + (a0.y + a1.y);
-}
-
-// quantised row chunk dot (contiguous lane layout); lx holds the lane's 32
-// activations and its two constants
-template <int FMT>
-__device__ __forceinline__ float q_chunk(const uint8_t* row, const uint8_t* srow, int cidx, bool active,
-                                         const LaneX& lx) {
-  if (!active) return 0.f;
-  Frag<FMT> f;
-  if constexpr (FMT == FMT_Q4)
-    f.q = *reinterpret_cast<const uint4*>(row + cidx * 16);
-  else
-    f.q = *reinterpret_cast<const uint2*>(row + cidx * 8);
-  f.s = *reinterpret_cast<const uint32_t*>(srow + (cidx >> 1) * 4);
-  return frag_dot<FMT>(f, lx);
-}
-
-// x chunk for quantised rows from the permuted bf16 copy, constants from xc
-__device__ __forceinline__ void xq_chunk(LaneX& lx, const uint4* xq, const float2* xc, int t, int nch, int ch) {
-  const int lane = threadIdx.x & 31;
-  const uint4* u = xq + (size_t)((t * nch + ch) * 4) * 32 + lane;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) unpack_bf16x8(u[32 * j], lx.x + 8 * j);
-  const float2 k = xc[(t * nch + ch) * 32 + lane];
-  lx.xsum = k.x;
-  lx.corr = k.y;
+  for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt) acc[mm][tt] = a[mm][tt].x + a[mm][tt].y;
+}
+
+// ---- packed rows on the tensor cores ----------------------------------------------------
+
+// D += A * B for one m16n8k16 step, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// B fragments of the four 16-column steps of one block from this lane's
+// code bytes: each 16-bit half becomes the bf16 number 128 + q (exponent of
+// 128 OR-ed over a code in the low mantissa bits).  Code positions: see the
+// block layout in moe_layout.h.
+template <int FMT>
+struct LaneCodes;
+template <>
+struct LaneCodes<FMT_Q4> {
+  uint2 w;
+  static constexpr int kBytes = 8;
+  __device__ __forceinline__ void load(const uint8_t* p) { w = *reinterpret_cast<const uint2*>(p); }
+  __device__ __forceinline__ void frags(uint32_t (&b)[4][2]) const {
+    const uint32_t v[2] = {w.x, w.y};
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        b[2 * h + j][0] = ((v[h] >> (8 * j)) & 0x000F000Fu) | 0x43004300u;
+        b[2 * h + j][1] = ((v[h] >> (8 * j + 4)) & 0x000F000Fu) | 0x43004300u;
+      }
+  }
+};
+template <>
+struct LaneCodes<FMT_Q2> {
+  uint32_t w;
+  static constexpr int kBytes = 4;
+  __device__ __forceinline__ void load(const uint8_t* p) { w = *reinterpret_cast<const uint32_t*>(p); }
+  __device__ __forceinline__ void frags(uint32_t (&b)[4][2]) const {
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      b[s][0] = ((w >> (4 * s)) & 0x00030003u) | 0x43004300u;
+      b[s][1] = ((w >> (4 * s + 2)) & 0x00030003u) | 0x43004300u;
+    }
+  }
+};
+
+// One unit of a routed tile: windows [u*W, u*W + W) of 8-row block `rbl` of
+// the segment.  gu: gate and up against x (bf16, A rows 0..7); otherwise down
+// against the routed intermediate (hi in A rows 0..7, lo in rows 8..15).
+// afrag: this token's (pair's) A fragments; asum: its group sums (gu) or
+// 8-row partial sums (down).  Returns rows 2t and 2t+1 of the block in
+// res[matrix][0/1] (every lane t, t = lane % 4, holds the sums of its rows).
+template <int FMT>
+__device__ __forceinline__ void routed_unit(const uint8_t* sl, const Seg& sg, int rbl, int u, const RoutedGeo& geo,
+                                            bool gu, const uint4* afrag, const float* asum, const uint4* zero4,
+                                            float (&res)[2][2]) {
+  constexpr int CB = LaneCodes<FMT>::kBytes;
+  constexpr int BB = 32 * CB;  // code bytes of one 8x64 block
+  const int lane = threadIdx.x & 31, m = lane >> 2, t = lane & 3;
+  const int na = gu ? 2 : 4;  // 16-byte A pieces per lane and group
+  const int nm = gu ? 2 : 1;
+  float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  const int wa = u * geo.W, wb = min(wa + geo.W, geo.nwin);
+  const int blk0 = rbl * geo.G - sg.gbase;
+#pragma unroll 1
+  for (int w = wa; w < wb; ++w) {
+    const int g0 = 8 * w, nv = min(8, geo.G - g0);
+    float d[2][4][4];
+#pragma unroll
+    for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+      for (int s = 0; s < 4; ++s) d[mm][s][0] = d[mm][s][1] = d[mm][s][2] = d[mm][s][3] = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < nv; ++j) {
+      const uint4* ap = (m == j) ? afrag + ((size_t)(g0 + j) * 4 + t) * na : zero4;
+      uint32_t a[4][4];
+      if (gu) {
+        const uint4 v0 = ap[0], v1 = ap[1];
+        a[0][0] = v0.x, a[0][2] = v0.y, a[1][0] = v0.z, a[1][2] = v0.w;
+        a[2][0] = v1.x, a[2][2] = v1.y, a[3][0] = v1.z, a[3][2] = v1.w;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) a[s][1] = a[s][3] = 0u;
+      } else {
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const uint4 v = ap[s];
+          a[s][0] = v.x, a[s][1] = v.y, a[s][2] = v.z, a[s][3] = v.w;
+        }
+      }
+      const size_t boff = (size_t)(blk0 + g0 + j) * BB + lane * CB;
+#pragma unroll
+      for (int mm = 0; mm < 2; ++mm) {
+        if (mm < nm) {
+          LaneCodes<FMT> c;
+          c.load(sl + sg.off[mm] + boff);
+          uint32_t b[4][2];
+          c.frags(b);
+#pragma unroll
+          for (int s = 0; s < 4; ++s) mma_16816(d[mm][s], a[s][0], a[s][1], a[s][2], a[s][3], b[s][0], b[s][1]);
+        }
+      }
+    }
+    // lane group m owns group g0 + m: rows 2t, 2t+1
+    if (m < nv) {
+      const int g = g0 + m;
+      float X;
+      if (gu) {
+        X = asum[g];
+      } else {
+        const float4 p0 = *reinterpret_cast<const float4*>(asum + 8 * g);
+        const float4 p1 = *reinterpret_cast<const float4*>(asum + 8 * g + 4);
+        X = ((p0.x + p0.y) + (p0.z + p0.w)) + ((p1.x + p1.y) + (p1.z + p1.w));
+      }
+#pragma unroll
+      for (int mm = 0; mm < 2; ++mm) {
+        if (mm < nm) {
+          const uint2 sw = *reinterpret_cast<const uint2*>(sl + sg.off[nm + mm] + (size_t)(blk0 + g) * 32 + t * 8);
+          // rows m (hi) and m + 8 (lo, zero for gate/up) of D
+          const float D0 = ((d[mm][0][0] + d[mm][1][0]) + (d[mm][2][0] + d[mm][3][0])) +
+                           ((d[mm][0][2] + d[mm][1][2]) + (d[mm][2][2] + d[mm][3][2]));
+          const float D1 = ((d[mm][0][1] + d[mm][1][1]) + (d[mm][2][1] + d[mm][3][1])) +
+                           ((d[mm][0][3] + d[mm][1][3]) + (d[mm][2][3] + d[mm][3][3]));
+          const float s0 = __uint_as_float(sw.x << 16), b0 = __uint_as_float(sw.x & 0xffff0000u);
+          const float s1 = __uint_as_float(sw.y << 16), b1 = __uint_as_float(sw.y & 0xffff0000u);
+          acc[mm][0] = fmaf(s0, D0, fmaf(fmaf(-128.f, s0, b0), X, acc[mm][0]));
+          acc[mm][1] = fmaf(s1, D1, fmaf(fmaf(-128.f, s1, b1), X, acc[mm][1]));
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      float v = acc[mm][k];
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      res[mm][k] = v;
+    }
+}
+
+// A routed gate/up unit is done: store its partial sums in accumulator entry
+// e; the warp that completes the row block's last unit sums the units in
+// order, applies SiLU(gate) * up and publishes the 8 intermediate values as
+// hi/lo A fragments of the down projection, with their sum.
+__device__ __noinline__ void gu_unit_done(float r00, float r01, float r10, float r11, int e, int u, int U,
+                                          float* part, int* cnt, int pair, int rb, int I, uint8_t* hf,
+                                          float* hx) {
+  const int lane = threadIdx.x & 31;
+  float* pe = part + (size_t)e * kMaxUnits * 16;
+  if (lane < 4) {
+    *reinterpret_cast<float4*>(pe + u * 16 + 4 * lane) = make_float4(r00, r10, r01, r11);
+    __threadfence_block();
+  }
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) {
+    __threadfence_block();
+    last = atomicAdd(&cnt[e], 1) == U - 1 ? 1 : 0;
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence_block();
+  float g = 0.f, up = 0.f;
+  if (lane < 8) {
+    const volatile float* pp = pe + 2 * lane;
+#pragma unroll 1
+    for (int uu = 0; uu < U; ++uu) {
+      g += pp[uu * 16];
+      up += pp[uu * 16 + 1];
+    }
+  }
+  if (lane == 0) cnt[e] = 0;  // entry free for a later row block
+  const float h = silu_mul(g, up);
+  const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
+  float hsum = lane < 8 ? __bfloat162float(hi) + __bfloat162float(lo) : 0.f;
+  hsum += __shfl_xor_sync(0xffffffffu, hsum, 1);
+  hsum += __shfl_xor_sync(0xffffffffu, hsum, 2);
+  hsum += __shfl_xor_sync(0xffffffffu, hsum, 4);
+  const uint32_t hb = __bfloat16_as_ushort(hi), lb = __bfloat16_as_ushort(lo);
+  const int t = lane & 3;
+  const uint32_t h0 = __shfl_sync(0xffffffffu, hb, 2 * t), h1 = __shfl_sync(0xffffffffu, hb, 2 * t + 1);
+  const uint32_t l0 = __shfl_sync(0xffffffffu, lb, 2 * t), l1 = __shfl_sync(0xffffffffu, lb, 2 * t + 1);
+  // rows 8rb..8rb+7 of I: group rb/8, step (rb%8)/2, first or second 8 columns
+  const int Gi = I / 64;
+  const int gq = rb >> 3, sq = (rb & 7) >> 1, half = rb & 1;
+  if (lane < 4) {
+    const size_t off = ((((size_t)pair * Gi + gq) * 4 + lane) * 4 + sq) * 16 + half * 8;
+    *reinterpret_cast<uint2*>(hf + off) = make_uint2(h0 | (h1 << 16), l0 | (l1 << 16));
+  }
+  if (lane == 0) hx[(size_t)pair * (I / 8) + rb] = hsum;
 }
 
 // ---- producer ----------------------------------------------------------------------
@@ -280,20 +479,36 @@ struct Producer {
   uint64_t* empty;
   TileDesc* descs;
   uint32_t slot_bytes;
-  uint32_t slot, phase;
+  uint32_t slot, phase, nslots;
   uint64_t timeout_ns;
   uint32_t* err;
   uint32_t* abort_flag;
   uint64_t* trace;
+  uint32_t* spins;  // [0] empty-slot waits, [1] routing wait (traced launches only)
   int ncommit;
   bool ok;
+  bool open;
+  int pending_pre;
+  int nrb_tile;
   TileDesc* d;
   uint32_t fill;
   uint64_t policy;  // L2 evict-first: weights are read once per launch
 
+  __device__ __noinline__ void commit() {
+    if (!open) return;
+    if (trace && ncommit < 16) trace[48 + ncommit] = globaltimer_ns();
+    ++ncommit;
+    mbar_arrive(&full[slot]);
+    if (++slot == nslots) {
+      slot = 0;
+      phase ^= 1u;
+    }
+    open = false;
+  }
   __device__ __noinline__ bool begin(int type) {
+    commit();
     if (!ok) return false;
-    if (!mbar_wait(&empty[slot], phase ^ 1u, timeout_ns)) {
+    if (!mbar_wait(&empty[slot], phase ^ 1u, timeout_ns, spins)) {
       ok = false;
       atomicCAS(err, 0u, 1u);
       atomicExch(abort_flag, 1u);
@@ -302,7 +517,12 @@ struct Producer {
     d = &descs[slot];
     d->type = type;
     d->nseg = 0;
+    d->pre = pending_pre;
+    d->post = 0;
+    pending_pre = 0;
     fill = 0;
+    nrb_tile = 0;
+    open = true;
     return true;
   }
   __device__ Seg& seg(int pair, int row0, int nrows) {
@@ -310,6 +530,10 @@ struct Producer {
     s.pair = pair;
     s.row0 = row0;
     s.nrows = nrows;
+    s.u0 = 0;
+    s.u1 = 0;
+    s.gbase = 0;
+    s.acc = 0;
     return s;
   }
   // Copy a byte range into the slot; returns the slot offset of its first
@@ -327,322 +551,384 @@ struct Producer {
     fill += n;
     return off;
   }
-  __device__ __noinline__ void commit() {
-    if (trace && ncommit < 16) trace[48 + ncommit] = globaltimer_ns();
-    ++ncommit;
-    mbar_arrive(&full[slot]);
-    if (++slot == kSlots) {
-      slot = 0;
-      phase ^= 1u;
-    }
+  // Attach arrival flags to the current tile (an empty tile if none is open)
+  // and publish it.
+  __device__ void post(int flag) {
+    if (!open && !begin(TILE_NONE)) return;
+    d->post |= flag;
+    commit();
   }
-  __device__ void marker(int type) {
-    if (begin(type)) commit();
+  // Waits for the consumers to do before the next tile's compute.
+  __device__ void pre(int flag) {
+    commit();
+    pending_pre |= flag;
   }
 };
 
-template <int FMT>
-__device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, uint64_t* xbar, float* tk_w,
-                             int* tk_i, const uint8_t** eptr) {
+// Routed tiles for row blocks [rb_a, rb_b) of nm matrices of one (token,
+// expert) pair (off_codes / off_scales: the matrices' section offsets).  A
+// segment is one row block's run of whole units [u0, u1) that fits the open
+// tile; a tile takes segments until it is full, holds kMaxSeg of them or
+// max_rb row blocks.  Each row block gets the next accumulator entry.
+__device__ __noinline__ void emit_routed(Producer& pr, int type, int bits, const size_t* off_codes,
+                                         const size_t* off_scales, const uint8_t* blob, int pair, int rb_a,
+                                         int rb_b, int nm, RoutedGeo geo, int max_rb, int* rbseq) {
+  const uint32_t bb = 64u * (uint32_t)bits;
+  const uint32_t per_unit = (uint32_t)(8 * geo.W) * (uint32_t)nm * (bb + 32u);
+  const uint32_t slack = 64;
+#pragma unroll 1
+  for (int rb = rb_a; rb < rb_b; ++rb) {
+    const int e = (*rbseq)++ % kAccSlots;
+#pragma unroll 1
+    for (int u = 0; u < geo.U;) {
+      if (pr.open && (pr.d->type != type || pr.d->nseg >= kMaxSeg || pr.nrb_tile >= max_rb ||
+                      pr.fill + per_unit + slack > pr.slot_bytes))
+        pr.commit();
+      if (!pr.open && !pr.begin(type)) return;
+      const int un = min(geo.U - u, max(1, (int)((pr.slot_bytes - pr.fill - slack) / per_unit)));
+      const int ga = 8 * geo.W * u, gb = min(geo.G, 8 * geo.W * (u + un));
+      Seg& s = pr.seg(pair, rb, 1);
+      s.u0 = u;
+      s.u1 = u + un;
+      s.gbase = ga;
+      s.acc = e;
+      const size_t b0 = (size_t)rb * geo.G + ga;
+#pragma unroll 1
+      for (int mm = 0; mm < 2 * nm; ++mm) {
+        const bool sc = mm >= nm;
+        const uint32_t per = sc ? 32u : bb;
+        s.off[mm] = pr.range(blob + (sc ? off_scales[mm - nm] : off_codes[mm]) + b0 * per, (size_t)(gb - ga) * per);
+      }
+      ++pr.nrb_tile;
+      u += un;
+    }
+  }
+}
+
+// bf16 rows [a, b) of one or two row-major matrices (row_bytes each), as many
+// rows per tile as fit.
+__device__ __noinline__ void emit_rows(Producer& pr, int type, const uint8_t* m0, const uint8_t* m1,
+                                       uint32_t row_bytes, int a, int b) {
+  const uint32_t nm = m1 ? 2u : 1u;
+  const int cap = max(1, min(1024, (int)((pr.slot_bytes - 16u * nm) / (nm * row_bytes))));
+#pragma unroll 1
+  for (int r = a; r < b; r += cap) {
+    const int n = min(cap, b - r);
+    if (!pr.begin(type)) return;
+    Seg& s = pr.seg(-1, r, n);
+    s.off[0] = pr.range(m0 + (size_t)r * row_bytes, (size_t)n * row_bytes);
+    if (m1) s.off[1] = pr.range(m1 + (size_t)r * row_bytes, (size_t)n * row_bytes);
+  }
+}
+
+template <bool TRACE>
+__device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, uint16_t* res_s, uint16_t* gam_s,
+                             uint64_t* xbar, uint64_t* topkbar, const int* flags, const uint8_t* const* eptr) {
   const Layout& L = p.L;
   const int T = p.T, K = L.K, H = L.H, I = L.I, E = L.E;
   const int G = gridDim.x, c = blockIdx.x;
-  const int lane = threadIdx.x & 31;
-  const bool leader = lane == 0;
-  const int r0 = (int)((long long)H * c / G), r1 = (int)((long long)H * (c + 1) / G);
+  int r0, r1;
+  block_rows(H, c, G, r0, r1);
+  // the token activations, and this block's rows of the residual and of gamma
+  const uint32_t xb = (uint32_t)(2ull * T * H);
+  const uint32_t rb = (uint32_t)(2 * (r1 - r0));
+  mbar_expect_tx(xbar, xb + (uint32_t)(T + 1) * rb);
+  bulk_g2s(xs, p.x, xb, xbar);
+  if (rb > 0) {
+#pragma unroll 1
+    for (int t = 0; t < T; ++t) bulk_g2s(res_s + (size_t)t * (r1 - r0), p.res + (size_t)t * H + r0, rb, xbar);
+    bulk_g2s(gam_s, p.gamma + r0, rb, xbar);
+  }
+  mbar_arrive(xbar);
+  int a, b;
+  range_of(E, c, G, a, b);
+  emit_rows(pr, TILE_ROUTER, reinterpret_cast<const uint8_t*>(p.wr), nullptr, 2u * H, a, b);
+  pr.post(F_ARRIVE_R);
+  if (L.has_shared) {
+    range_of(I, c, G, a, b);
+    emit_rows(pr, TILE_SHARED_GU, reinterpret_cast<const uint8_t*>(p.sg), reinterpret_cast<const uint8_t*>(p.su),
+              2u * H, a, b);
+  }
+  pr.post(F_ARRIVE_S);
+  // the routing, from the sync warp
+  bool routed = false;
+  if (pr.ok) {
+    if (mbar_wait(topkbar, 0, p.timeout_ns, pr.spins ? pr.spins + 1 : nullptr)) {
+      routed = flags[FLAG_TOPK] != 0;
+    } else {
+      pr.ok = false;
+      atomicCAS(p.err, 0u, 1u);
+      atomicExch(pr.abort_flag, 1u);
+    }
+  }
+  if (pr.trace) pr.trace[9] = globaltimer_ns();
+  const RoutedGeo gh = routed_geo(H), gi = routed_geo(I);
+  const size_t oc[3] = {L.off_codes[0], L.off_codes[1], L.off_codes[2]};
+  const size_t os[3] = {L.off_scales[0], L.off_scales[1], L.off_scales[2]};
+  const int nrb_i = I / 8;
+  int rbseq = 0;
+  if (routed) {
+    // routed gate/up: this block's share of the T*K*(I/8) (pair, row block) items
+    range_of(T * K * nrb_i, c, G, a, b);
+#pragma unroll 1
+    for (int q = a; q < b && pr.ok;) {
+      const int pair = q / nrb_i, rb0 = q - pair * nrb_i;
+      const int n = min(b - q, nrb_i - rb0);
+      emit_routed(pr, TILE_EXPERT_GU, L.bits, oc, os, eptr[pair], pair, rb0, rb0 + n, 2, gh, kMaxRbPerTile, &rbseq);
+      q += n;
+    }
+  }
+  pr.post(F_ARRIVE_E);
+  pr.pre(F_WAIT_S);
+  if (L.has_shared) emit_rows(pr, TILE_SHARED_DOWN, reinterpret_cast<const uint8_t*>(p.sd), nullptr, 2u * I, r0, r1);
+  pr.pre(F_WAIT_E);
+  if (routed && r1 > r0) {
+#pragma unroll 1
+    for (int pair = 0; pair < T * K && pr.ok; ++pair)
+      emit_routed(pr, TILE_EXPERT_DOWN, L.bits, oc + 2, os + 2, eptr[pair], pair, r0 / 8, r1 / 8, 1, gi, 1 << 20,
+                  &rbseq);
+  }
+  pr.post(F_END);
+  if (pr.trace) pr.trace[10] = globaltimer_ns();
+}
 
-  if (leader) {
-    // the token activations, once per block
-    const uint32_t xb = (uint32_t)(2ull * T * H);
-    mbar_expect_tx(xbar, xb);
-    bulk_g2s(xs, p.x, xb, xbar);
-    mbar_arrive(xbar);
-    // router rows
-    int a, b;
-    range_of(E, c, G, a, b);
-    const int rmax = cap_rows(pr.slot_bytes, 16, 2 * H);
+// ---- sync warp ----------------------------------------------------------------------
+// Prepares x as A fragments with its group sums, then does the block's
+// grid-wide arrivals (R, S, E, D) and waits (R, S, E, D).  After the R wait it
+// runs the top-K and hands the expert pointers to the producer; after the S
+// and E waits it stages the shared / routed intermediates into shared memory
+// with bulk copies that complete the consumers' "go" barriers.
+template <bool TRACE>
+__device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar, uint64_t* topkbar, uint64_t* evt,
+                         uint64_t* go, int* flags, const uint16_t* xs, uint4* xf, float* xsum, float* hs_s,
+                         uint8_t* hf_s, float* hx_s, float* tk_w, int* tk_i, const uint8_t** eptr, uint64_t* tkbuf,
+                         uint32_t* spins) {
+  const int lane = threadIdx.x & 31;
+  const Layout& L = p.L;
+  const int T = p.T, H = L.H, K = L.K, E = L.E, G = gridDim.x;
+  uint32_t* ctr = p.ctr;
+  const uint64_t to = p.timeout_ns;
+  uint32_t* sp_evt = spins ? spins + 5 : nullptr;
+  uint32_t* sp_grid = spins ? spins + 6 : nullptr;
+  bool ok = warp_wait(xbar, 0, to, spins ? spins + 7 : nullptr);
+  if (ok) {
+    // piece q: 8 columns (16 bytes) of one token's x; its four words go to
+    // lanes t = 0..3 of the A fragment of their group and step half
+    const int np = T * H / 8;
 #pragma unroll 1
-    for (int e = a; e < b; e += rmax) {
-      const int n = min(rmax, b - e);
-      if (!pr.begin(TILE_ROUTER)) break;
-      Seg& s = pr.seg(-1, e, n);
-      s.off[0] = pr.range(p.wr + (size_t)e * H, (size_t)n * H * 2);
-      pr.commit();
-    }
-    pr.marker(TILE_ARRIVE_R);
-    // shared gate/up rows
-    if (L.has_shared) {
-      range_of(I, c, G, a, b);
-      const int smax = cap_rows(pr.slot_bytes, 32, 4 * H);
-#pragma unroll 1
-      for (int i = a; i < b; i += smax) {
-        const int n = min(smax, b - i);
-        if (!pr.begin(TILE_SHARED_GU)) break;
-        Seg& s = pr.seg(-1, i, n);
-        s.off[0] = pr.range(p.sg + (size_t)i * H, (size_t)n * H * 2);
-        s.off[1] = pr.range(p.su + (size_t)i * H, (size_t)n * H * 2);
-        pr.commit();
+    for (int q0 = 0; q0 < np; q0 += 32) {
+      const int q = q0 + lane;
+      float s = 0.f;
+      if (q < np) {
+        const uint4 v = reinterpret_cast<const uint4*>(xs)[q];
+        const int tg = q >> 3, o8 = q & 7;  // tg = token * Gh + group
+        uint32_t* dst = reinterpret_cast<uint32_t*>(xf) + (size_t)tg * 32 + o8;
+        dst[0] = v.x;
+        dst[8] = v.y;
+        dst[16] = v.z;
+        dst[24] = v.w;
+        float xx[8];
+        unpack_bf16x8(v, xx);
+        s = ((xx[0] + xx[1]) + (xx[2] + xx[3])) + ((xx[4] + xx[5]) + (xx[6] + xx[7]));
       }
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s += __shfl_xor_sync(0xffffffffu, s, 4);
+      if (q < np && (q & 7) == 0) xsum[q >> 3] = s;
     }
-    pr.marker(TILE_ARRIVE_S);
   }
   __syncwarp();
-
-  // top-K, once the router logits of every block are written
-  bool ok = true;
-  if (leader) ok = grid_wait_thread(&p.ctr[0], G, &p.ctr[5], p.err, p.timeout_ns);
-  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-  if (ok) {
+  if (lane == 0) {
+    mbar_arrive(xfbar);
+    trace_mark<TRACE>(p, 64);
+    // R: arrive once every consumer warp has passed the router tiles
+    if (!mbar_wait(&evt[EVT_R], 0, to, sp_evt)) ok = false;
+    red_release_add(&ctr[0], 1u);
+  }
+  // top-K once every block's router logits are written
+  int good = 0;
+  if (lane == 0) good = (ok && grid_wait_thread(&ctr[0], G, &ctr[5], p.err, to, sp_grid)) ? 1 : 0;
+  good = __shfl_sync(0xffffffffu, good, 0);
+  if (lane == 0) trace_mark<TRACE>(p, 65);
+  if (good) {
 #pragma unroll 1
-    for (int t = 0; t < T; ++t) warp_topk(p.logits + (size_t)t * E, E, K, tk_i + t * K, tk_w + t * K);
+    for (int t = 0; t < T; ++t) warp_topk_keys(p.logits + (size_t)t * E, E, K, tkbuf, tk_i + t * K, tk_w + t * K);
     __syncwarp();
+    if (lane == 0) trace_mark<TRACE>(p, 66);
 #pragma unroll 1
     for (int j = lane; j < T * K; j += 32) {
       const int e = tk_i[j];
       const void* bp = (e >= 0 && e < E) ? p.expert_ptr[e] : nullptr;
       if (bp == nullptr || (reinterpret_cast<uintptr_t>(bp) & 255u)) {
         atomicCAS(p.err, 0u, 2u);
-        atomicExch(&p.ctr[5], 1u);
+        atomicExch(&ctr[5], 1u);
         bp = nullptr;
+        good = 0;
       }
       eptr[j] = reinterpret_cast<const uint8_t*>(bp);
-      if (c == 0) {
+      if (blockIdx.x == 0) {
         if (p.idx_out) p.idx_out[j] = e;
         if (p.w_out) p.w_out[j] = tk_w[j];
       }
     }
-    __syncwarp();
-#pragma unroll 1
-    for (int j = 0; j < T * K; ++j) ok = ok && eptr[j] != nullptr;
+    good = __all_sync(0xffffffffu, good != 0) ? 1 : 0;
   }
-  if (leader) {
-    trace_mark(p, 9);
-    const uint32_t cr_h = L.code_row_bytes[0], sr_h = L.scale_row_bytes[0];
-    const uint32_t cr_i = L.code_row_bytes[2], sr_i = L.scale_row_bytes[2];
-    if (ok) {
-      // routed gate/up: this block's share of the T*K*I (pair, row) items
-      int a, b;
-      range_of(T * K * I, c, G, a, b);
-      const int gmax = cap_rows(pr.slot_bytes, 64, 2 * (cr_h + sr_h));
-#pragma unroll 1
-      for (int q = a; q < b;) {
-        const int pair = q / I, i = q - pair * I;
-        const int n = min(gmax, min(b - q, I - i));
-        const uint8_t* blob = eptr[pair];
-        if (!pr.begin(TILE_EXPERT_GU)) break;
-        Seg& s = pr.seg(pair, i, n);
-        s.off[0] = pr.range(blob + L.off_codes[0] + (size_t)i * cr_h, (size_t)n * cr_h);
-        s.off[1] = pr.range(blob + L.off_codes[1] + (size_t)i * cr_h, (size_t)n * cr_h);
-        s.off[2] = pr.range(blob + L.off_scales[0] + (size_t)i * sr_h, (size_t)n * sr_h);
-        s.off[3] = pr.range(blob + L.off_scales[1] + (size_t)i * sr_h, (size_t)n * sr_h);
-        pr.commit();
-        q += n;
-      }
-    }
-    pr.marker(TILE_ARRIVE_E);
-    pr.marker(TILE_WAIT_S);
-    if (L.has_shared) {
-      const int dmax = cap_rows(pr.slot_bytes, 16, 2 * I);
-#pragma unroll 1
-      for (int r = r0; r < r1; r += dmax) {
-        const int n = min(dmax, r1 - r);
-        if (!pr.begin(TILE_SHARED_DOWN)) break;
-        Seg& s = pr.seg(-1, r, n);
-        s.off[0] = pr.range(p.sd + (size_t)r * I, (size_t)n * I * 2);
-        pr.commit();
-      }
-    }
-    pr.marker(TILE_WAIT_E);
-    if (ok) {
-      // routed down rows [r0, r1) of every pair, several pairs per tile
-      const uint32_t per_row = cr_i + sr_i;
-      const int emax = cap_rows(pr.slot_bytes, 32, per_row);
-      bool open = false;
-#pragma unroll 1
-      for (int pair = 0; pair < T * K && pr.ok; ++pair) {
-#pragma unroll 1
-        for (int r = r0; r < r1;) {
-          const int n = min(emax, r1 - r);
-          if (open && (pr.d->nseg == kMaxSeg || pr.fill + (uint32_t)n * per_row + 32 > pr.slot_bytes)) {
-            pr.commit();
-            open = false;
-          }
-          if (!open) {
-            if (!pr.begin(TILE_EXPERT_DOWN)) break;
-            open = true;
-          }
-          const uint8_t* blob = eptr[pair];
-          Seg& s = pr.seg(pair, r, n);
-          s.off[0] = pr.range(blob + L.off_codes[2] + (size_t)r * cr_i, (size_t)n * cr_i);
-          s.off[1] = pr.range(blob + L.off_scales[2] + (size_t)r * sr_i, (size_t)n * sr_i);
-          r += n;
-        }
-      }
-      if (open) pr.commit();
-    }
-    pr.marker(TILE_END);
-    trace_mark(p, 10);
-  }
-}
-
-// ---- sync warp ----------------------------------------------------------------------
-// Prepares the quantised-layout copy of x and its constants, then does the
-// block's grid-wide arrivals (R, S, E, D) and waits (S, E, D).  After the S
-// and E waits it stages the shared / routed intermediates into shared memory
-// with bulk copies that complete the consumers' "go" barriers.
-template <int FMT>
-__device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xcbar, uint64_t* evt, uint64_t* go,
-                         int* flags, const uint16_t* xs, uint4* xq, float2* xc, float* hs_s, float* he_s) {
-  const int lane = threadIdx.x & 31;
-  const Layout& L = p.L;
-  const int T = p.T, H = L.H, G = gridDim.x;
-  const int nch = (H + 1023) / 1024;
-  uint32_t* ctr = p.ctr;
-  const uint64_t to = p.timeout_ns;
-  bool ok = warp_wait(xbar, 0, to);
-  if (ok) {
-#pragma unroll 1
-    for (int u = lane; u < T * nch * 32; u += 32) {
-      const int t = u / (nch * 32), cidx = u - t * nch * 32;  // cidx = 32*ch + l
-      const int ch = cidx >> 5, l = cidx & 31;
-      LaneX lx;
-      if (cidx * 32 < H) {
-        const uint16_t* src = xs + (size_t)t * H + cidx * 32;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 v = *reinterpret_cast<const uint4*>(src + 8 * j);
-          xq[(size_t)((t * nch + ch) * 4 + j) * 32 + l] = v;
-          unpack_bf16x8(v, lx.x + 8 * j);
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) xq[(size_t)((t * nch + ch) * 4 + j) * 32 + l] = make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) lx.x[i] = 0.f;
-      }
-      lane_constants<FMT>(lx);
-      xc[u] = make_float2(lx.xsum, lx.corr);
-    }
-  }
-  __syncwarp();
   if (lane == 0) {
-    mbar_arrive(xcbar);
-    // R, S, E: arrive once every consumer warp has passed the phase's marker
+    flags[FLAG_TOPK] = good;
+    mbar_arrive(topkbar);
+    trace_mark<TRACE>(p, 67);
+    // S and E: arrive once every consumer warp has passed the phase's tiles
 #pragma unroll 1
-    for (int k = EVT_R; k <= EVT_E; ++k) {
-      if (!mbar_wait(&evt[k], 0, to)) ok = false;
+    for (int k = EVT_S; k <= EVT_E; ++k) {
+      if (!mbar_wait(&evt[k], 0, to, sp_evt)) ok = false;
       red_release_add(&ctr[k], 1u);
+      trace_mark<TRACE>(p, 68 + k - EVT_S);
     }
     // wait S, then E; stage the intermediates; release the consumers
 #pragma unroll 1
     for (int k = 0; k < 2; ++k) {
-      bool good = ok;
-      if (good && (k == 1 || L.has_shared)) good = grid_wait_thread(&ctr[1 + k], G, &ctr[5], p.err, to);
-      flags[GO_S + k] = good ? 1 : 0;
+      bool g = ok;
+      const bool need = k == 1 ? good != 0 : L.has_shared != 0;
+      if (g && need) g = grid_wait_thread(&ctr[1 + k], G, &ctr[5], p.err, to, sp_grid);
+      trace_mark<TRACE>(p, 70 + k);
+      flags[GO_S + k] = g ? 1 : 0;
       uint64_t* bar = &go[GO_S + k];
-      if (good && (k == 1 || L.has_shared)) {
+      if (g && need) {
         fence_proxy_async_global();
-        const uint32_t bytes = k == 0 ? (uint32_t)(4ull * T * L.I) : (uint32_t)(4ull * T * L.K * L.I);
-        mbar_expect_tx(bar, bytes);
-        bulk_g2s(k == 0 ? hs_s : he_s, k == 0 ? p.hs : p.he, bytes, bar);
+        if (k == 0) {
+          const uint32_t bytes = (uint32_t)(4ull * T * L.I);
+          mbar_expect_tx(bar, bytes);
+          bulk_g2s(hs_s, p.hs, bytes, bar);
+        } else {
+          const uint32_t hfb = (uint32_t)(4ull * T * K * L.I), hxb = (uint32_t)(4ull * T * K * (L.I / 8));
+          mbar_expect_tx(bar, hfb + hxb);
+          bulk_g2s(hf_s, p.hf, hfb, bar);
+          bulk_g2s(hx_s, p.hx, hxb, bar);
+        }
       }
       mbar_arrive(bar);
     }
     // D: sum of squares written -> arrive, wait, release the consumers
-    if (!mbar_wait(&evt[EVT_D], 0, to)) ok = false;
+    if (!mbar_wait(&evt[EVT_D], 0, to, sp_evt)) ok = false;
     red_release_add(&ctr[3], 1u);
-    const bool good = ok && grid_wait_thread(&ctr[3], G, &ctr[5], p.err, to);
-    flags[GO_D] = good ? 1 : 0;
+    trace_mark<TRACE>(p, 72);
+    const bool g = ok && grid_wait_thread(&ctr[3], G, &ctr[5], p.err, to, sp_grid);
+    trace_mark<TRACE>(p, 73);
+    flags[GO_D] = g ? 1 : 0;
     mbar_arrive(&go[GO_D]);
   }
   __syncwarp();
 }
 
-template <int FMT>
+template <int FMT, bool TRACE>
 __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const Layout& L = p.L;
   const int T = p.T, K = L.K, H = L.H, I = L.I;
   const int G = gridDim.x, c = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int r0 = (int)((long long)H * c / G), r1 = (int)((long long)H * (c + 1) / G);
+  int r0, r1;
+  block_rows(H, c, G, r0, r1);
   const int nrows = r1 - r0;
-  const int nrows_max = (H + G - 1) / G;
-  const int nch_h = (H + 1023) / 1024, nch_i = (I + 1023) / 1024;
-  const DecodeSmem sp = decode_smem_plan(T, K, H, I, nrows_max, p.slot_bytes);
+  const int nslots = p.nslots;
+  const DecodeSmem sp = decode_smem_plan(T, K, L.E, H, I, decode_rows_max(H, G), nslots, p.slot_bytes);
   uint8_t* ring = smem + sp.ring;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + sp.bars);
-  uint64_t* empty = full + kSlots;
+  uint64_t* empty = full + nslots;
   uint64_t* xbar = empty + kSlots;
-  uint64_t* xcbar = xbar + 1;
-  uint64_t* evt = xcbar + 1;
+  uint64_t* xfbar = xbar + 1;
+  uint64_t* topkbar = xfbar + 1;
+  uint64_t* evt = topkbar + 1;
   uint64_t* go = evt + NEVT;
   TileDesc* descs = reinterpret_cast<TileDesc*>(smem + sp.desc);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + sp.xs);
-  uint4* xq = reinterpret_cast<uint4*>(smem + sp.xq);
-  float2* xc = reinterpret_cast<float2*>(smem + sp.xc);
+  uint4* xf = reinterpret_cast<uint4*>(smem + sp.xf);
+  float* xsum = reinterpret_cast<float*>(smem + sp.xsum);
   float* hs_s = reinterpret_cast<float*>(smem + sp.hs);
-  float* he_s = reinterpret_cast<float*>(smem + sp.he);
+  uint8_t* hf_s = smem + sp.hf;
+  float* hx_s = reinterpret_cast<float*>(smem + sp.hx);
+  uint4* zero4 = reinterpret_cast<uint4*>(smem + sp.zero);
+  float* part = reinterpret_cast<float*>(smem + sp.part);
+  int* cnt = reinterpret_cast<int*>(smem + sp.cnt);
   float* tk_w = reinterpret_cast<float*>(smem + sp.tk_w);
   int* tk_i = reinterpret_cast<int*>(smem + sp.tk_i);
   const uint8_t** eptr = reinterpret_cast<const uint8_t**>(smem + sp.eptr);
+  uint64_t* tkbuf = reinterpret_cast<uint64_t*>(smem + sp.tkbuf);
+  uint16_t* res_s = reinterpret_cast<uint16_t*>(smem + sp.res);
+  uint16_t* gam_s = reinterpret_cast<uint16_t*>(smem + sp.gam);
   float* ypart = reinterpret_cast<float*>(smem + sp.ypart);
   float* ys = reinterpret_cast<float*>(smem + sp.ys);
   float* hacc = reinterpret_cast<float*>(smem + sp.hacc);
   float* inv = reinterpret_cast<float*>(smem + sp.inv);
   int* flags = reinterpret_cast<int*>(smem + sp.flags);
+  uint32_t* spin_s = reinterpret_cast<uint32_t*>(smem + sp.spin);
+  uint32_t* spins = TRACE ? spin_s : nullptr;  // poll counts, traced launches only
   uint32_t* ctr = p.ctr;
 
   if (tid == 0) {
-    for (int s = 0; s < kSlots; ++s) {
+    for (int s = 0; s < nslots; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
     }
     mbar_init(xbar, 1);
-    mbar_init(xcbar, 1);
+    mbar_init(xfbar, 1);
+    mbar_init(topkbar, 1);
     for (int k = 0; k < NEVT; ++k) mbar_init(&evt[k], k == EVT_D ? 1 : kConsumerWarps);
     for (int k = 0; k < NGO; ++k) mbar_init(&go[k], 1);
     mbar_fence_init();
-    trace_mark(p, 0);
+    trace_mark<TRACE>(p, 0);
   }
+  if (tid < 16) {
+    zero4[tid >> 2] = make_uint4(0u, 0u, 0u, 0u);
+    spin_s[tid] = 0u;
+  }
+  if (tid < kAccSlots) cnt[tid] = 0;
   __syncthreads();
 
   if (warp == kProducerWarp) {
-    Producer pr;
-    pr.ring = ring;
-    pr.full = full;
-    pr.empty = empty;
-    pr.descs = descs;
-    pr.slot_bytes = p.slot_bytes;
-    pr.slot = 0;
-    pr.phase = 0;
-    pr.timeout_ns = p.timeout_ns;
-    pr.err = p.err;
-    pr.abort_flag = &ctr[5];
-    pr.trace = p.trace ? p.trace + (size_t)c * kTraceEntries : nullptr;
-    pr.ncommit = 0;
-    pr.ok = true;
-    pr.d = descs;
-    pr.fill = 0;
-    pr.policy = l2_policy_evict_first();
-    run_producer<FMT>(p, pr, xs, xbar, tk_w, tk_i, eptr);
+    if (lane == 0) {
+      Producer pr;
+      pr.ring = ring;
+      pr.full = full;
+      pr.empty = empty;
+      pr.descs = descs;
+      pr.slot_bytes = p.slot_bytes;
+      pr.slot = 0;
+      pr.phase = 0;
+      pr.nslots = (uint32_t)nslots;
+      pr.timeout_ns = p.timeout_ns;
+      pr.err = p.err;
+      pr.abort_flag = &ctr[5];
+      pr.trace = TRACE ? p.trace + (size_t)c * kTraceEntries : nullptr;
+      pr.spins = spins ? spins + 3 : nullptr;
+      pr.ncommit = 0;
+      pr.ok = true;
+      pr.open = false;
+      pr.pending_pre = 0;
+      pr.nrb_tile = 0;
+      pr.d = descs;
+      pr.fill = 0;
+      pr.policy = l2_policy_evict_first();
+      run_producer<TRACE>(p, pr, xs, res_s, gam_s, xbar, topkbar, flags, eptr);
+    }
+    __syncwarp();
   } else if (warp == kSyncWarp) {
-    run_sync<FMT>(p, xbar, xcbar, evt, go, flags, xs, xq, xc, hs_s, he_s);
+    run_sync<TRACE>(p, xbar, xfbar, topkbar, evt, go, flags, xs, xf, xsum, hs_s, hf_s, hx_s, tk_w, tk_i, eptr, tkbuf,
+                    spins);
   } else {
     // ---------------- consumer warps ----------------
-    // Every compute tile runs through one loop nest: segment -> this warp's
-    // row items -> token -> matrix -> 1024-column chunk.  The tile kind only
-    // selects the row format, the activation source and the epilogue, so the
-    // dot-product code exists once and stays in the instruction cache.
-    bool ok = true;
-    bool have_x = false, have_xc = false;
-    int item = 0;      // running count of row items over the compute tiles
-    int held = -1;     // key of the activation chunk cached in lx
-    bool probed = false;
-    LaneX lx;
+    // Every warp walks every tile; the tile's work items (bf16 rows, or units
+    // of packed row blocks) are dealt round-robin to the warps, continuing
+    // across tiles, and each warp releases a slot on its own.
+    const RoutedGeo gh = routed_geo(H), gi = routed_geo(I);
+    bool ok = warp_wait(xbar, 0, p.timeout_ns, spins ? spins + 2 : nullptr);
+    bool have_xf = false;
+    int item = 0;  // running count of work items over the compute tiles
+    int probed = 0;  // first routed units traced: bit 0 gate/up, bit 1 down
     uint32_t slot = 0, phase = 0;
+#pragma unroll 1
     for (int ntile = 0;; ++ntile) {
-      if (!warp_wait(&full[slot], phase, p.timeout_ns)) {
+      if (!warp_wait(&full[slot], phase, p.timeout_ns, spins)) {
         if (lane == 0) {
           atomicCAS(p.err, 0u, 1u);
           atomicExch(&ctr[5], 1u);
@@ -650,153 +936,138 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         ok = false;
         break;
       }
-      if (tid == 0 && ntile < 16) trace_mark(p, 16 + 2 * ntile);
+      if (tid == 0 && ntile < 16) trace_mark<TRACE>(p, 16 + 2 * ntile);
       const TileDesc& d = descs[slot];
       const int type = d.type;
       const uint8_t* sl = ring + (size_t)slot * p.slot_bytes;
-      if (type == TILE_END) break;
-      if (type >= TILE_ARRIVE_R) {
-        if (type <= TILE_ARRIVE_E) {
-          __syncwarp();  // the warp's stores of this phase precede its arrival
-          if (lane == 0) mbar_arrive(&evt[type - TILE_ARRIVE_R]);
-          if (tid == 0) trace_mark(p, 1 + type - TILE_ARRIVE_R);
-        } else {
-          const int k = type == TILE_WAIT_S ? GO_S : GO_E;
-          ok = warp_wait(&go[k], 0, p.timeout_ns) && flags[k] != 0 && ok;
-          if (tid == 0) trace_mark(p, type == TILE_WAIT_S ? 4 : 5);
+#pragma unroll 1
+      for (int k = 0; k < 2; ++k) {
+        if (d.pre & (F_WAIT_S << k)) {
+          ok = warp_wait(&go[GO_S + k], 0, p.timeout_ns, spins ? spins + 1 : nullptr) && flags[GO_S + k] != 0 && ok;
+          if (tid == 0) trace_mark<TRACE>(p, 4 + k);
         }
-      } else {
-        // ---- compute tile ----
-        const bool routed = type == TILE_EXPERT_GU || type == TILE_EXPERT_DOWN;
-        const bool down = type >= TILE_SHARED_DOWN;
-        const int nm = (type == TILE_SHARED_GU || type == TILE_EXPERT_GU) ? 2 : 1;
-        const int cols = down ? I : H;
-        const int nch = down ? nch_i : nch_h;
-        const int ntok = routed ? 1 : T;
-        const uint32_t crow = routed ? L.code_row_bytes[down ? 2 : 0] : 2u * (uint32_t)cols;
-        const uint32_t srow = routed ? L.scale_row_bytes[down ? 2 : 0] : 0u;
-        // activation source: 0 x (bf16 rows), 1 x (quantised rows), 2 shared
-        // intermediate (bf16 rows), 3 routed intermediate (quantised rows)
-        const int xk = type == TILE_ROUTER || type == TILE_SHARED_GU ? 0
-                       : type == TILE_EXPERT_GU                       ? 1
-                       : type == TILE_SHARED_DOWN                     ? 2
-                                                                      : 3;
-        if (xk == 0 && !have_x) {
-          ok = warp_wait(xbar, 0, p.timeout_ns) && ok;
-          have_x = true;
-        }
-        if (xk == 1 && !have_xc) {
-          ok = warp_wait(xcbar, 0, p.timeout_ns) && ok;
-          have_xc = true;
-        }
-        const bool work = ok || !routed;  // routed tiles need the routing
+      }
+      const bool routed_tile = type == TILE_EXPERT_GU || type == TILE_EXPERT_DOWN;
+      if (type == TILE_EXPERT_GU && !have_xf) {
+        ok = warp_wait(xfbar, 0, p.timeout_ns, spins ? spins + 2 : nullptr) && ok;
+        have_xf = true;
+      }
+      const bool down = type == TILE_SHARED_DOWN || type == TILE_EXPERT_DOWN;
+      const bool work = type != TILE_NONE && (ok || !down);  // down tiles need the staged intermediate
 #pragma unroll 1
-        for (int si = 0; si < d.nseg; ++si) {
-          const Seg& sg = d.seg[si];
-          if (work && !(down && !ok)) {
+      for (int si = 0; si < d.nseg; ++si) {
+        const Seg& sg = d.seg[si];
+        const int nu = sg.u1 - sg.u0;
+        const int nitems = routed_tile ? sg.nrows * nu : sg.nrows;
+        if (work) {
 #pragma unroll 1
-            for (int j = (warp - item % kConsumerWarps + kConsumerWarps) % kConsumerWarps; j < sg.nrows;
-                 j += kConsumerWarps) {
+          for (int j = (warp - item % kConsumerWarps + kConsumerWarps) % kConsumerWarps; j < nitems;
+               j += kConsumerWarps) {
+            if (routed_tile) {
+              // ---- one unit of a packed row block: gate/up, or down ----
+              const bool gu = type == TILE_EXPERT_GU;
+              const int rbl = j / nu, u = sg.u0 + (j - rbl * nu);
+              const int pb = gu ? 1 : 2;
+              if (tid == 0 && !(probed & pb)) trace_mark<TRACE>(p, gu ? 11 : 13);
+              const uint4* af = gu ? xf + (size_t)(sg.pair / K) * gh.G * 8
+                                   : reinterpret_cast<const uint4*>(hf_s) + (size_t)sg.pair * gi.G * 16;
+              const float* as = gu ? xsum + (size_t)(sg.pair / K) * gh.G : hx_s + (size_t)sg.pair * (I / 8);
+              float r[2][2];
+              routed_unit<FMT>(sl, sg, rbl, u, gu ? gh : gi, gu, af, as, zero4, r);
+              if (gu) {
+                gu_unit_done(r[0][0], r[0][1], r[1][0], r[1][1], (sg.acc + rbl) % kAccSlots, u, gh.U, part, cnt,
+                             sg.pair, sg.row0 + rbl, I, p.hf, p.hx);
+              } else if (lane < 4) {
+                float* yp = ypart + (size_t)(sg.pair * gi.U + u) * nrows + 8 * (sg.row0 + rbl) + 2 * lane - r0;
+                yp[0] = r[0][0];
+                yp[1] = r[0][1];
+              }
+              if (tid == 0 && !(probed & pb)) {
+                trace_mark<TRACE>(p, gu ? 12 : 14);
+                probed |= pb;
+              }
+            } else {
+              // ---- one bf16 row (the gate/up pair for the shared expert) ----
+              const int cols = down ? I : H;
+              const uint8_t* w0 = sl + sg.off[0] + (size_t)j * 2 * cols;
+              const int row = sg.row0 + j;
 #pragma unroll 1
-              for (int tt = 0; tt < ntok; ++tt) {
-                const int t = routed ? sg.pair / K : tt;
-                float a0 = 0.f, a1 = 0.f;
+              for (int t0 = 0; t0 < T; t0 += 4) {
+                const int nt = min(4, T - t0);
+                float acc[2][4];
+                if (down)
+                  bf16_dot4(w0, nullptr, I, reinterpret_cast<const uint8_t*>(hs_s + (size_t)t0 * I), 4u * I, true,
+                            nt, acc);
+                else
+                  bf16_dot4(w0, type == TILE_SHARED_GU ? sl + sg.off[1] + (size_t)j * 2 * cols : nullptr, H,
+                            reinterpret_cast<const uint8_t*>(xs + (size_t)t0 * H), 2u * H, false, nt, acc);
 #pragma unroll 1
-                for (int ch = 0; ch < nch; ++ch) {
-                  const int cidx = ch * 32 + lane;
-                  const bool act = cidx * 32 < cols;
-                  const int key = ((xk * 64 + (xk == 3 ? sg.pair : t)) * 64 + ch);
-                  const bool probe = tid == 0 && type == TILE_EXPERT_GU && !probed && ch == 0;
-                  if (probe) trace_mark(p, 11);
-                  if (key != held) {
-                    if (xk == 0) {
-                      x_strided_bf16(lx.x, xs + (size_t)t * H, ch, H);
-                    } else if (xk == 1) {
-                      xq_chunk(lx, xq, xc, t, nch_h, ch);
-                    } else if (xk == 2) {
-                      x_strided_f32(lx.x, hs_s + (size_t)t * I, ch, I);
-                    } else {
-                      if (act) {
-                        const float4* hv = reinterpret_cast<const float4*>(he_s + (size_t)sg.pair * I + cidx * 32);
+                for (int tt = 0; tt < nt; ++tt) {
+                  const int t = t0 + tt;
+                  float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                          const float4 v = hv[q];
-                          lx.x[4 * q] = v.x;
-                          lx.x[4 * q + 1] = v.y;
-                          lx.x[4 * q + 2] = v.z;
-                          lx.x[4 * q + 3] = v.w;
-                        }
-                      } else {
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) lx.x[q] = 0.f;
-                      }
-                      lane_constants<FMT>(lx);
-                    }
-                    held = key;
-                  }
-                  if (probe) trace_mark(p, 12);
-#pragma unroll 1
-                  for (int m = 0; m < nm; ++m) {
-                    const uint8_t* row = sl + sg.off[m] + (size_t)j * crow;
-                    const float v = routed ? q_chunk<FMT>(row, sl + sg.off[nm + m] + (size_t)j * srow, cidx, act, lx)
-                                           : bf16_chunk(row, ch, cols, lx.x);
-                    if (m == 0)
-                      a0 += v;
+                  for (int q = 0; q < 4; ++q)
+                    if (q == tt) a0 = acc[0][q], a1 = acc[1][q];
+                  a0 = warp_sum(a0);
+                  if (type == TILE_SHARED_GU) a1 = warp_sum(a1);
+                  if (lane == 0) {
+                    if (type == TILE_ROUTER)
+                      p.logits[(size_t)t * L.E + row] = a0 + (p.bias ? p.bias[row] : 0.f);
+                    else if (type == TILE_SHARED_GU)
+                      p.hs[(size_t)t * I + row] = silu_mul(a0, a1);
                     else
-                      a1 += v;
+                      ys[t * nrows + row - r0] = a0;
                   }
-                  if (probe) trace_mark(p, 13);
-                }
-                if (tid == 0 && type == TILE_EXPERT_GU && !probed) trace_mark(p, 14);
-                a0 = warp_sum(a0);
-                if (nm == 2) a1 = warp_sum(a1);
-                if (lane == 0) {
-                  const int row = sg.row0 + j;
-                  if (type == TILE_ROUTER)
-                    p.logits[(size_t)t * L.E + row] = a0 + (p.bias ? p.bias[row] : 0.f);
-                  else if (type == TILE_SHARED_GU)
-                    p.hs[(size_t)t * I + row] = silu_mul(a0, a1);
-                  else if (type == TILE_EXPERT_GU)
-                    p.he[(size_t)sg.pair * I + row] = silu_mul(a0, a1);
-                  else if (type == TILE_SHARED_DOWN)
-                    ys[t * nrows + row - r0] = a0;
-                  else
-                    ypart[sg.pair * nrows + row - r0] = a0;
-                }
-                if (tid == 0 && type == TILE_EXPERT_GU && !probed) {
-                  trace_mark(p, 15);
-                  probed = true;
                 }
               }
             }
           }
-          item += sg.nrows;
         }
+        item += nitems;
       }
       // this warp is done with the slot
       __syncwarp();
+      if (lane == 0) {
+#pragma unroll 1
+        for (int k = 0; k < 3; ++k)
+          if (d.post & (F_ARRIVE_R << k)) mbar_arrive(&evt[EVT_R + k]);
+      }
+      if (tid == 0) {
+#pragma unroll 1
+        for (int k = 0; k < 3; ++k)
+          if (d.post & (F_ARRIVE_R << k)) trace_mark<TRACE>(p, 1 + k);
+      }
+      const bool end = (d.post & F_END) != 0;
+      __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
-      if (tid == 0 && ntile < 16) trace_mark(p, 17 + 2 * ntile);
-      if (++slot == kSlots) {
+      if (tid == 0 && ntile < 16) trace_mark<TRACE>(p, 17 + 2 * ntile);
+      if (++slot == (uint32_t)nslots) {
         slot = 0;
         phase ^= 1u;
       }
+      if (end) break;
     }
-    if (tid == 0) trace_mark(p, 6);
+    if (tid == 0) trace_mark<TRACE>(p, 6);
 
     // ---- combine + residual, sum of squares ----
     consumer_sync();
-    if (ok) {
+    const bool routed = flags[FLAG_TOPK] != 0;
+    if (ok && routed) {
 #pragma unroll 1
       for (int q = tid; q < T * nrows; q += kConsumers) {
         const int t = q / nrows, j = q - t * nrows;
         float acc = 0.f;
 #pragma unroll 1
-        for (int k = 0; k < K; ++k) acc = fmaf(tk_w[t * K + k], ypart[(t * K + k) * nrows + j], acc);
-        const float res = __bfloat162float(__ushort_as_bfloat16(p.res[(size_t)t * H + r0 + j]));
-        float h = res + acc;
-        if (L.has_shared) h += ys[t * nrows + j];
-        hacc[t * nrows + j] = h;
+        for (int k = 0; k < K; ++k) {
+          const int pair = t * K + k;
+          float yk = 0.f;
+#pragma unroll 1
+          for (int u = 0; u < gi.U; ++u) yk += ypart[(size_t)(pair * gi.U + u) * nrows + j];
+          acc = fmaf(tk_w[pair], yk, acc);
+        }
+        float h = __bfloat162float(__ushort_as_bfloat16(res_s[q])) + acc;
+        if (L.has_shared) h += ys[q];
+        hacc[q] = h;
         p.h_out[(size_t)t * H + r0 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
       }
       consumer_sync();
@@ -810,23 +1081,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     }
     consumer_sync();
     if (tid == 0) mbar_arrive(&evt[EVT_D]);
-    ok = warp_wait(&go[GO_D], 0, p.timeout_ns) && flags[GO_D] != 0 && ok;
-    if (tid == 0) trace_mark(p, 7);
+    ok = warp_wait(&go[GO_D], 0, p.timeout_ns, spins ? spins + 1 : nullptr) && flags[GO_D] != 0 && ok && routed;
+    if (tid == 0) trace_mark<TRACE>(p, 7);
     if (ok) {
       if (warp < T) {
         float s = 0.f;
 #pragma unroll 1
         for (int b = lane; b < G; b += 32) s += __ldcg(p.ss + (size_t)b * T + warp);
         s = warp_sum(s);
-        if (lane == 0) inv[warp] = 1.f / sqrtf(s / (float)H + L.eps);
+        if (lane == 0) inv[warp] = rsqrtf(__fdividef(s, (float)H) + L.eps);
       }
       consumer_sync();
 #pragma unroll 1
       for (int q = tid; q < T * nrows; q += kConsumers) {
         const int t = q / nrows, j = q - t * nrows;
-        const float gm = __bfloat162float(__ushort_as_bfloat16(p.gamma[r0 + j]));
-        p.y_norm[(size_t)t * H + r0 + j] =
-            __bfloat16_as_ushort(__float2bfloat16_rn(hacc[t * nrows + j] * inv[t] * gm));
+        const float gm = __bfloat162float(__ushort_as_bfloat16(gam_s[j]));
+        p.y_norm[(size_t)t * H + r0 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(hacc[q] * inv[t] * gm));
       }
     }
   }
@@ -834,7 +1104,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   // ---- exit: the last block out resets the counters for the next launch ----
   __syncthreads();
   if (tid == 0) {
-    trace_mark(p, 8);
+    trace_mark<TRACE>(p, 8);
+    if constexpr (TRACE)
+      for (int k = 0; k < 8; ++k) p.trace[(size_t)c * kTraceEntries + 80 + k] = spin_s[k];
     __threadfence();
     const uint32_t old = atomicAdd(&ctr[4], 1u);
     if (old == (uint32_t)G - 1u) {
@@ -844,14 +1116,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   }
 }
 
-template <int FMT>
+template <int FMT, bool TRACE>
 static cudaError_t launch_one(const DecodeParams& p, int grid, size_t smem, cudaStream_t st) {
   static size_t attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && attr_set[dev] < smem) {
     cudaError_t e =
-        cudaFuncSetAttribute(moe_decode_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(moe_decode_kernel<FMT, TRACE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = smem;
   }
@@ -865,29 +1137,39 @@ static cudaError_t launch_one(const DecodeParams& p, int grid, size_t smem, cuda
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, moe_decode_kernel<FMT>, p);
+  return cudaLaunchKernelEx(&cfg, moe_decode_kernel<FMT, TRACE>, p);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int grid, size_t smem, cudaStream_t st) {
-  return p.L.bits == 4 ? launch_one<FMT_Q4>(p, grid, smem, st) : launch_one<FMT_Q2>(p, grid, smem, st);
+  if (p.trace)
+    return p.L.bits == 4 ? launch_one<FMT_Q4, true>(p, grid, smem, st) : launch_one<FMT_Q2, true>(p, grid, smem, st);
+  return p.L.bits == 4 ? launch_one<FMT_Q4, false>(p, grid, smem, st) : launch_one<FMT_Q2, false>(p, grid, smem, st);
 }
 
-// Largest slot size (bytes, multiple of 1 KB, at most 48 KB) that fits the
-// shared memory of one block together with the rest of the plan; 0 if the
-// smallest tile of some phase would not fit.
-uint32_t decode_slot_bytes(const Layout& L, int T, int nrows_max) {
+// Ring geometry for a shape: the most slots (4, else 3, else 2) whose size
+// (a multiple of 1 KB, at most 48 KB) holds the largest tile of every phase
+// next to the rest of the shared-memory plan.  Returns the slot size and sets
+// *nslots, or returns 0 if no ring fits.
+uint32_t decode_slot_bytes(const Layout& L, int T, int nrows_max, int* nslots) {
   const size_t limit = 227 * 1024;
-  const size_t other = decode_smem_plan(T, L.K, L.H, L.I, nrows_max, 0).total + 1024;
-  if (other >= limit) return 0;
-  size_t slot = (limit - other) / kSlots;
-  slot = slot / 1024 * 1024;
-  if (slot > (size_t)kMaxSlotBytes) slot = kMaxSlotBytes;
-  const size_t need[5] = {2ull * L.H + 16, 4ull * L.H + 32,
-                          2ull * (L.code_row_bytes[0] + L.scale_row_bytes[0]) + 64, 2ull * L.I + 16,
-                          (size_t)L.code_row_bytes[2] + L.scale_row_bytes[2] + 32};
-  for (size_t n : need)
-    if (n > slot) return 0;
-  return (uint32_t)slot;
+  const RoutedGeo gh = routed_geo(L.H), gi = routed_geo(L.I);
+  const size_t per_group = 64ull * L.bits + 32;
+  const size_t need[5] = {2ull * L.H + 16, 4ull * L.H + 32, 2ull * L.I + 16,
+                          2ull * 8 * gh.W * per_group + 64, 8ull * gi.W * per_group + 64};
+  for (int ns = kSlots; ns >= 2; --ns) {
+    const size_t other = decode_smem_plan(T, L.K, L.E, L.H, L.I, nrows_max, ns, 0).total + 1024;
+    if (other >= limit) return 0;
+    size_t slot = (limit - other) / ns;
+    slot = slot / 1024 * 1024;
+    if (slot > (size_t)kMaxSlotBytes) slot = kMaxSlotBytes;
+    bool fits = true;
+    for (size_t n : need) fits = fits && n <= slot;
+    if (fits) {
+      *nslots = ns;
+      return (uint32_t)slot;
+    }
+  }
+  return 0;
 }
 
 // A stand-alone bounded wait on a counter that nothing increments: checks the

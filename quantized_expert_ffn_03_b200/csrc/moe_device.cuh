@@ -1,7 +1,7 @@
 // moe_device.cuh -- device-side building blocks of libmoe (sm_100a).
 //
-// Row dot products over packed 4/2-bit group-affine weights and bf16 weights,
-// warp/team reductions, bounded grid-wide waits and the router's top-K.
+// bf16 unpacking, warp reductions, bounded grid-wide waits, the router's
+// top-K, and the mbarrier / bulk-copy primitives of the streaming ring.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -11,208 +11,7 @@
 
 namespace moe {
 
-
-enum Fmt { FMT_Q4 = 4, FMT_Q2 = 2, FMT_BF16 = 16 };
-
-// ---------------------------------------------------------------------------
-// Per-lane activation slice: 32 consecutive input columns in fp32 registers,
-// plus the two per-lane constants of the factored dequant dot (below).
-// ---------------------------------------------------------------------------
-struct LaneX {
-  float x[32];
-  float xsum;  // sum of the 32 values (multiplies the group bias)
-  float corr;  // sum of magic offsets times x (removed from the code sum)
-};
-
-// Dequant dot, factored per group.  For one group with scale s and bias beta:
-//   sum_i (q_i*s + beta) x_i = s * sum_i q_i x_i + beta * sum_i x_i,
-// the per-weight fma(q, s*x, beta*x) of the FMA kernel summed over the group
-// ("Streaming experts: как запустить триллионную модель на MacBook",
-// section "Оптимизации, которые сработали").  The code q is turned into a
-// float without a conversion instruction: the word is rotated so that the
-// code lands in the top mantissa bits (bits 15..22) and OR-ed with the
-// exponent of 2^e, which gives exactly 2^e + q.  The known 2^e terms are
-// summed once per lane into `corr` and subtracted after the loop.
-//   4-bit: a rotation puts nibble 2p at bits 15..18 (256 + q) and nibble
-//          2p+1 at bits 19..22 (16 + q).
-//   2-bit: a rotation puts codes 4p..4p+3 at bits 15,17,19,21
-//          (256 + q, 64 + q, 16 + q, 4 + q).
-// The rotation for pair/quad p of a word is rotl(word, (15 - 8p) mod 32).
-__device__ __forceinline__ uint32_t rotl(uint32_t v, int r) { return __funnelshift_l(v, v, r); }
-
-__device__ __forceinline__ float magic(uint32_t r, uint32_t mask, uint32_t expo) {
-  return __uint_as_float((r & mask) | expo);
-}
-
-template <int FMT>
-__device__ __forceinline__ void lane_constants(LaneX& lx) {
-  float s = 0.f, c = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    s += lx.x[i];
-    float off;
-    if (FMT == FMT_Q4) {
-      off = (i & 1) ? 16.f : 256.f;
-    } else if (FMT == FMT_Q2) {
-      const int j = i & 3;
-      off = j == 0 ? 256.f : j == 1 ? 64.f : j == 2 ? 16.f : 4.f;
-    } else {
-      off = 0.f;
-    }
-    c = fmaf(off, lx.x[i], c);
-  }
-  lx.xsum = s;
-  lx.corr = c;
-}
-
-// Sum over 32 columns of (2^e + q_i) * x_i for one 4-bit fragment.  The two
-// codes a rotation exposes multiply two adjacent activations, so each pair is
-// one packed fp32 FMA (fma.rn.f32x2): lane x[2i] pairs with the 256+q code of
-// its word position, x[2i+1] with the 16+q code.
-__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
-
-__device__ __forceinline__ float codes_dot_q4(const uint4 q, const LaneX& lx) {
-  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-  float2 acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const uint32_t r = rotl(w[j], (15 - 8 * p) & 31);
-      const float2 c = f2(magic(r, 0x00078000u, 0x43800000u), magic(r, 0x00780000u, 0x41800000u));
-      const float2 xx = f2(lx.x[8 * j + 2 * p], lx.x[8 * j + 2 * p + 1]);
-      if (p & 1)
-        acc1 = __ffma2_rn(c, xx, acc1);
-      else
-        acc0 = __ffma2_rn(c, xx, acc0);
-    }
-  }
-  return (acc0.x + acc1.x) + (acc0.y + acc1.y);
-}
-
-// Same for a 2-bit fragment (two words, 32 codes): codes 4p..4p+3 of a word
-// sit at bits 15, 17, 19, 21 after one rotation (256+q, 64+q, 16+q, 4+q).
-__device__ __forceinline__ float codes_dot_q2(const uint2 q, const LaneX& lx) {
-  const uint32_t w[2] = {q.x, q.y};
-  float2 acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const uint32_t r = rotl(w[j], (15 - 8 * p) & 31);
-      const float* xx = lx.x + 16 * j + 4 * p;
-      acc0 = __ffma2_rn(f2(magic(r, 0x00018000u, 0x43800000u), magic(r, 0x00060000u, 0x42800000u)),
-                        f2(xx[0], xx[1]), acc0);
-      acc1 = __ffma2_rn(f2(magic(r, 0x00180000u, 0x41800000u), magic(r, 0x00600000u, 0x40800000u)),
-                        f2(xx[2], xx[3]), acc1);
-    }
-  }
-  return (acc0.x + acc1.x) + (acc0.y + acc1.y);
-}
-
-__device__ __forceinline__ float bf16_dot(const uint4 (&q)[4], const LaneX& lx) {
-  float2 acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const float2 c = f2(__uint_as_float(w[m] << 16), __uint_as_float(w[m] & 0xffff0000u));
-      const float2 xx = f2(lx.x[8 * j + 2 * m], lx.x[8 * j + 2 * m + 1]);
-      if (m & 1)
-        acc1 = __ffma2_rn(c, xx, acc1);
-      else
-        acc0 = __ffma2_rn(c, xx, acc0);
-    }
-  }
-  return (acc0.x + acc1.x) + (acc0.y + acc1.y);
-}
-
-// ---------------------------------------------------------------------------
-// Per-lane fragment of one weight row: the lane's 32 columns.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 v;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
-  uint2 v;
-  asm("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
-  uint32_t v;
-  asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
-
-template <int FMT>
-struct Frag;
-template <>
-struct Frag<FMT_Q4> {
-  uint4 q;
-  uint32_t s;
-};
-template <>
-struct Frag<FMT_Q2> {
-  uint2 q;
-  uint32_t s;
-};
-template <>
-struct Frag<FMT_BF16> {
-  uint4 q[4];
-};
-
-// Quantised row: codes_row / scales_row point at the row's first byte.
-template <int FMT>
-__device__ __forceinline__ void load_frag(Frag<FMT>& f, const uint8_t* codes_row,
-                                          const uint8_t* scales_row, int chunk) {
-  if constexpr (FMT == FMT_Q4) {
-    f.q = ld_stream_v4(codes_row + chunk * 16);
-    f.s = ld_stream_u32(scales_row + (chunk >> 1) * 4);
-  } else if constexpr (FMT == FMT_Q2) {
-    f.q = ld_stream_v2(codes_row + chunk * 8);
-    f.s = ld_stream_u32(scales_row + (chunk >> 1) * 4);
-  } else {
-    const uint8_t* p = codes_row + chunk * 64;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) f.q[j] = ld_stream_v4(p + 16 * j);
-  }
-}
-
-template <int FMT>
-__device__ __forceinline__ void zero_frag(Frag<FMT>& f) {
-  if constexpr (FMT == FMT_BF16) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) f.q[j] = make_uint4(0, 0, 0, 0);
-  } else if constexpr (FMT == FMT_Q4) {
-    f.q = make_uint4(0, 0, 0, 0);
-    f.s = 0;
-  } else {
-    f.q = make_uint2(0, 0);
-    f.s = 0;
-  }
-}
-
-// Partial dot of the lane's 32 columns with the lane's activations.
-template <int FMT>
-__device__ __forceinline__ float frag_dot(const Frag<FMT>& f, const LaneX& lx) {
-  if constexpr (FMT == FMT_BF16) {
-    return bf16_dot(f.q, lx);
-  } else {
-    float raw;
-    if constexpr (FMT == FMT_Q4)
-      raw = codes_dot_q4(f.q, lx);
-    else
-      raw = codes_dot_q2(f.q, lx);
-    const float s = __uint_as_float(f.s << 16);
-    const float beta = __uint_as_float(f.s & 0xffff0000u);
-    return fmaf(s, raw - lx.corr, beta * lx.xsum);
-  }
-}
+enum Fmt { FMT_Q4 = 4, FMT_Q2 = 2 };
 
 // ---------------------------------------------------------------------------
 // Activation loads.
@@ -224,43 +23,6 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4 v, float* out) {
     out[2 * m] = __uint_as_float(w[m] << 16);
     out[2 * m + 1] = __uint_as_float(w[m] & 0xffff0000u);
   }
-}
-
-// bf16 activations (read-only for the whole kernel).
-template <int FMT>
-__device__ __forceinline__ void load_lane_x_bf16(LaneX& lx, const uint16_t* row, int chunk,
-                                                 bool active) {
-  if (active) {
-    const uint4* p = reinterpret_cast<const uint4*>(row + chunk * 32);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) unpack_bf16x8(__ldg(p + j), lx.x + 8 * j);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) lx.x[i] = 0.f;
-  }
-  lane_constants<FMT>(lx);
-}
-
-// fp32 activations written earlier in the same launch by other blocks: read
-// through L2 only (ld.global.cg), never from a possibly stale L1 line.
-template <int FMT>
-__device__ __forceinline__ void load_lane_x_f32(LaneX& lx, const float* row, int chunk,
-                                                bool active) {
-  if (active) {
-    const float4* p = reinterpret_cast<const float4*>(row + chunk * 32);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 v = __ldcg(p + j);
-      lx.x[4 * j] = v.x;
-      lx.x[4 * j + 1] = v.y;
-      lx.x[4 * j + 2] = v.z;
-      lx.x[4 * j + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) lx.x[i] = 0.f;
-  }
-  lane_constants<FMT>(lx);
 }
 
 // ---------------------------------------------------------------------------
@@ -347,86 +109,102 @@ __device__ __forceinline__ bool grid_wait(const uint32_t* ctr, uint32_t target, 
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float rank_key(float v) { return v != v ? -INFINITY : v; }
 
-__device__ __forceinline__ bool ranks_before(float ka, int ia, float kb, int ib) {
-  return ka > kb || (ka == kb && ia < ib);
+
+// Top-K keys as one ordered 64-bit integer: the logit's bits mapped so that
+// unsigned order is float order (after -0 -> +0 and NaN -> -inf), above the
+// complemented expert index, so a larger key ranks first and equal logits
+// rank by lower index.
+__device__ __forceinline__ uint64_t topk_key(float v, int e) {
+  v = rank_key(v);
+  if (v == 0.f) v = 0.f;
+  const uint32_t u = __float_as_uint(v);
+  const uint32_t o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((uint64_t)o << 32) | (uint32_t)~(uint32_t)e;
+}
+__device__ __forceinline__ float topk_key_value(uint64_t k) {
+  const uint32_t o = (uint32_t)(k >> 32);
+  return __uint_as_float((o & 0x80000000u) ? (o ^ 0x80000000u) : ~o);
+}
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = w > v ? w : v;
+  }
+  return v;
 }
 
-// logits: [E] for this token (read through L2).  Writes idx[K], w[K] from
-// lane 0..K-1 (any memory space).
-static __device__ __noinline__ void warp_topk(const float* logits, int E, int K, int32_t* idx, float* w) {
+// w[0..K) holds the chosen logits in rank order; replace them by the weights
+// exp(l_k - l_max) / sum_j exp(l_j - l_max) over the K chosen logits (fast
+// division: a few ulp).
+__device__ __forceinline__ void topk_weights(int K, float* w) {
   const int lane = threadIdx.x & 31;
-  float prev_k = INFINITY;
-  int prev_i = -1;
-  float sel_k[kMaxK];
-  int sel_i[kMaxK];
-  const bool in_regs = E <= 1024;
-  float vals[32];
-  if (in_regs) {
-#pragma unroll
-    for (int m = 0; m < 32; ++m) {
-      const int e = lane + 32 * m;
-      vals[m] = e < E ? rank_key(__ldcg(logits + e)) : -INFINITY;
-    }
-  }
-#pragma unroll 1
-  for (int k = 0; k < K; ++k) {
-    // best element of this lane that ranks strictly after the previous pick
-    float bk = -INFINITY;
-    int bi = 0x7fffffff;
-    if (in_regs) {
-#pragma unroll
-      for (int m = 0; m < 32; ++m) {
-        const int e = lane + 32 * m;
-        if (e < E && ranks_before(prev_k, prev_i, vals[m], e) &&
-            ranks_before(vals[m], e, bk, bi))
-          bk = vals[m], bi = e;
-      }
-    } else {
-      for (int e = lane; e < E; e += 32) {
-        const float v = rank_key(__ldcg(logits + e));
-        if (ranks_before(prev_k, prev_i, v, e) && ranks_before(v, e, bk, bi)) bk = v, bi = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ranks_before(ok, oi, bk, bi)) bk = ok, bi = oi;
-    }
-    sel_k[k < kMaxK ? k : 0] = bk;
-    sel_i[k < kMaxK ? k : 0] = bi;
-    prev_k = bk;
-    prev_i = bi;
-  }
-  // weights, computed redundantly by every lane; lane k writes entry k
-  const float lmax = sel_k[0];
+  __syncwarp();
+  const float lmax = w[0];
   float den = 0.f;
 #pragma unroll 1
-  for (int k = 0; k < K; ++k) den += expf(sel_k[k] - lmax);
+  for (int k = 0; k < K; ++k) den += expf(w[k] - lmax);
+  __syncwarp();
+#pragma unroll 1
+  for (int k = lane; k < K; k += 32) w[k] = __fdividef(expf(w[k] - lmax), den);
+  __syncwarp();
+}
+
+// vals: [E] logits of one token, read with plain loads (memory written by an
+// earlier launch, or staged by this warp).  Writes idx[K] and w[K] (any
+// memory space; w holds the chosen logits before it receives the weights).
+static __device__ __noinline__ void warp_topk(const float* vals, int E, int K, int32_t* idx, float* w) {
+  const int lane = threadIdx.x & 31;
+  uint64_t prev = ~0ull;
 #pragma unroll 1
   for (int k = 0; k < K; ++k) {
-    if (lane == (k & 31)) {
-      idx[k] = sel_i[k];
-      w[k] = expf(sel_k[k] - lmax) / den;
+    uint64_t best = 0;
+#pragma unroll 4
+    for (int e = lane; e < E; e += 32) {
+      const uint64_t key = topk_key(vals[e], e);
+      if (key < prev && key > best) best = key;
     }
+    best = warp_max_u64(best);
+    if (lane == 0) {
+      idx[k] = (int)~(uint32_t)best;
+      w[k] = topk_key_value(best);
+    }
+    prev = best;
   }
+  topk_weights(K, w);
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.f + expf(-g)) * u; }
-
-// L2 prefetch of a byte range through the bulk-copy engine (no shared
-// memory).  The range is widened to 16-byte boundaries; callers keep it
-// inside the allocation (all sections of a blob are 256-byte aligned).
-__device__ __forceinline__ void l2_prefetch(const void* p, size_t bytes) {
-  if (bytes == 0) return;
-  uintptr_t a = reinterpret_cast<uintptr_t>(p) & ~uintptr_t(15);
-  const uintptr_t end = (reinterpret_cast<uintptr_t>(p) + bytes + 15) & ~uintptr_t(15);
-  while (a < end) {
-    const uint32_t n = (uint32_t)((end - a) < 32768 ? (end - a) : 32768);
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
-    a += n;
+// The same for logits written earlier in this launch by other blocks
+// (global memory, read through L2): their keys are staged once into `keys`
+// (E entries of shared memory) with independent loads, then each of the K
+// rounds scans shared memory.
+static __device__ __noinline__ void warp_topk_keys(const float* logits, int E, int K, uint64_t* keys,
+                                                   int32_t* idx, float* w) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll 4
+  for (int e = lane; e < E; e += 32) keys[e] = topk_key(__ldcg(logits + e), e);
+  __syncwarp();
+  uint64_t prev = ~0ull;
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    uint64_t best = 0;
+#pragma unroll 4
+    for (int e = lane; e < E; e += 32) {
+      const uint64_t key = keys[e];
+      best = (key < prev && key > best) ? key : best;
+    }
+    best = warp_max_u64(best);
+    if (lane == 0) {
+      idx[k] = (int)~(uint32_t)best;
+      w[k] = topk_key_value(best);
+    }
+    prev = best;
   }
+  topk_weights(K, w);
 }
+
+// SiLU(g) * u with a fast division (relative error of a few ulp).
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.f + expf(-g)) * u; }
 
 // ---------------------------------------------------------------------------
 // Shared-memory barriers (mbarrier) and bulk copies global -> shared.
@@ -477,14 +255,24 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Bounded wait for phase `parity` of an mbarrier; false on timeout.
-static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 1023u) == 1023u && globaltimer_ns() - t0 > timeout_ns) return false;
+// Bounded wait for phase `parity` of an mbarrier; false on timeout.  If
+// `spins` is not null, the number of polls is added to it (shared memory).
+static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
+                                              uint32_t* spins = nullptr) {
+  bool ok = true;
+  uint32_t it = 0;
+  if (!mbar_try_wait(bar, parity)) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;; ++it) {
+      if (mbar_try_wait(bar, parity)) break;
+      if ((it & 1023u) == 1023u && globaltimer_ns() - t0 > timeout_ns) {
+        ok = false;
+        break;
+      }
+    }
   }
+  if (spins) atomicAdd(spins, it + 1);
+  return ok;
 }
 
 // Orders this thread's earlier generic-proxy accesses (e.g. an acquire that

@@ -9,13 +9,36 @@
 
 namespace moe {
 
+// Geometry of the packed rows of one matrix with `cols` input columns, as the
+// tensor-core dot walks it: G groups of 64 columns, nwin windows of 8 groups,
+// W windows per work unit, U units per 8-row block (U <= kMaxUnits).
+constexpr int kMaxUnits = 8;
+struct RoutedGeo {
+  int G, nwin, W, U;
+};
+__host__ __device__ inline RoutedGeo routed_geo(int cols) {
+  RoutedGeo g;
+  g.G = cols / 64;
+  g.nwin = (g.G + 7) / 8;
+  g.W = (g.nwin + kMaxUnits - 1) / kMaxUnits;
+  g.U = (g.nwin + g.W - 1) / g.W;
+  return g;
+}
+
+// Output rows [r0, r1) of block c of G: whole 8-row blocks, spread evenly.
+__host__ __device__ inline void block_rows(int H, int c, int G, int& r0, int& r1) {
+  const uint32_t nrb = (uint32_t)H / 8u;  // nrb * G < 2^32
+  r0 = (int)(8u * (nrb * (uint32_t)c / (uint32_t)G));
+  r1 = (int)(8u * (nrb * (uint32_t)(c + 1) / (uint32_t)G));
+}
+__host__ __device__ inline int decode_rows_max(int H, int G) { return 8 * ((H / 8 + G - 1) / G); }
+
 // Workspace of a layer call: counters and error word first, then fp32
 // intermediates.  ctr[0] router, [1] shared gate/up, [2] routed gate/up,
 // [3] down, [4] blocks that exited, [5] abort flag of the running launch.
 struct DecodeParams {
   Layout L;
   int T;
-  int tw_h, tw_i;  // warps per team for H-wide and I-wide rows
   const void* const* expert_ptr;
   const uint16_t* wr;
   const float* bias;
@@ -33,16 +56,18 @@ struct DecodeParams {
   uint32_t* err;
   float* logits;  // [T][E]
   float* hs;      // [T][I]
-  float* he;      // [T][K][I]
+  uint8_t* hf;    // routed intermediate as hi/lo bf16 A fragments, 4*T*K*I bytes
+  float* hx;      // [T*K][I/8] sums of hi + lo over 8-row blocks
   float* ss;      // [grid][T]
   uint64_t timeout_ns;
   uint32_t slot_bytes;  // bytes per shared-memory ring slot
-  uint64_t* trace;      // optional [grid][16] phase timestamps (ns), or null
+  int nslots;           // ring slots (2..4)
+  uint64_t* trace;      // optional [grid][64] phase timestamps (ns), or null
 };
 
 constexpr int kDecodeBlockThreads = 512;  // 14 consumer warps, a producer warp, a sync warp
-size_t decode_smem_bytes(const Layout& L, int T, int nrows, uint32_t slot_bytes);
-uint32_t decode_slot_bytes(const Layout& L, int T, int nrows_max);
+size_t decode_smem_bytes(const Layout& L, int T, int nrows, int nslots, uint32_t slot_bytes);
+uint32_t decode_slot_bytes(const Layout& L, int T, int nrows_max, int* nslots);
 cudaError_t launch_decode(const DecodeParams& p, int grid, size_t smem, cudaStream_t st);
 cudaError_t decode_occupancy(int bits, size_t smem, int* blocks_per_sm);
 cudaError_t launch_barrier_timeout_probe(uint32_t* ctr, uint32_t* err, uint64_t timeout_ns,
@@ -50,7 +75,7 @@ cudaError_t launch_barrier_timeout_probe(uint32_t* ctr, uint32_t* err, uint64_t 
 
 // Stand-alone router: logits into `logits` ([T][E]), then top-K.
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* wr, const float* bias, int T,
-                                 int H, int E, int tw, int grid, float* logits, cudaStream_t st);
+                                 int H, int E, int grid, float* logits, cudaStream_t st);
 cudaError_t launch_topk(const float* logits, int T, int E, int K, int32_t* idx, float* w,
                         cudaStream_t st);
 

@@ -8,16 +8,22 @@
 
 namespace moe {
 
-constexpr int kThreads = 512;                // threads per block of the GEMV kernels
-constexpr int kWarps = kThreads / 32;
 constexpr int kMaxTokensFused = 8;           // tokens per launch of the fused decode kernel
 constexpr int kMaxK = 32;                    // largest top_k
 
 // Where the sections of one packed expert blob live (byte offsets) and how
-// long a row is in each.  Matrix index m: 0 gate [I][H], 1 up [I][H],
+// many bytes a row takes in each.  Matrix index m: 0 gate [I][H], 1 up [I][H],
 // 2 down [H][I].  Sections follow each other in the order gate codes, up
 // codes, down codes, gate scales, up scales, down scales, each starting on a
 // 256-byte boundary.
+//
+// Inside a code section the codes come in blocks of 8 rows x 64 columns,
+// row-block major then column group (64*b bytes per block); inside a block,
+// lane l = 4*(row % 8) + t owns 2*b bytes holding the codes that the
+// tensor-core B fragment of an m16n8k16 step takes for t (see moe_pack.cu).
+// Scale words are stored [row block][group][row % 8].  So any run of whole
+// row blocks is one contiguous byte range in both sections, of
+// rows * code_row_bytes and rows * scale_row_bytes bytes.
 struct Layout {
   int H, I, E, K, bits;
   int has_shared;

@@ -8,6 +8,7 @@
 // single-precision operation in the same order, with no contraction.
 //   s = bf16_rne((max - min) / (2^b - 1)),  beta = bf16_rne(min)
 //   q = clamp(rint((w - beta) / s), 0, 2^b - 1),  q = 0 when s == 0
+// and the codes are stored in the block layout described in moe_layout.h.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -61,9 +62,9 @@ __host__ __device__ inline float div_rn(float a, float b) {
 #endif
 }
 
-// Quantise one 64-weight group: writes 64*bits/32 code words and returns the
-// scale word (scale in bits 0..15, bias in bits 16..31).
-__host__ __device__ inline uint32_t quantize_group64(const float* w, int bits, uint32_t* words) {
+// Quantise one 64-weight group: writes the 64 codes (column order) to q and
+// returns the scale word (scale in bits 0..15, bias in bits 16..31).
+__host__ __device__ inline uint32_t quantize_group64(const float* w, int bits, uint8_t* q) {
   float mn = w[0], mx = w[0];
   for (int i = 1; i < 64; ++i) {
     mn = w[i] < mn ? w[i] : mn;
@@ -73,21 +74,62 @@ __host__ __device__ inline uint32_t quantize_group64(const float* w, int bits, u
   const uint16_t sb = bf16_rne_bits(div_rn(sub_rn(mx, mn), qmax));
   const uint16_t bb = bf16_rne_bits(mn);
   const float s = bf16_bits_to_f32(sb), beta = bf16_bits_to_f32(bb);
-  const int per_word = 32 / bits;
-  for (int j = 0; j < 64 / per_word; ++j) {
-    uint32_t word = 0;
-    for (int n = 0; n < per_word; ++n) {
-      uint32_t q = 0;
-      if (s != 0.f) {
-        float r = rintf(div_rn(sub_rn(w[j * per_word + n], beta), s));
-        r = r < 0.f ? 0.f : (r > qmax ? qmax : r);
-        q = (uint32_t)r;
-      }
-      word |= q << (n * bits);
+  for (int i = 0; i < 64; ++i) {
+    uint8_t c = 0;
+    if (s != 0.f) {
+      float r = rintf(div_rn(sub_rn(w[i], beta), s));
+      r = r < 0.f ? 0.f : (r > qmax ? qmax : r);
+      c = (uint8_t)r;
     }
-    words[j] = word;
+    q[i] = c;
   }
   return (uint32_t)sb | ((uint32_t)bb << 16);
+}
+
+// Block layout of the codes (see moe_layout.h): the words of row `row`
+// (row % 8 = n) for one 64-column group are the lanes 4n + t, t = 0..3;
+// lane words hold, per 16-column step s, the columns 16s + 2t + e ("first")
+// and 16s + 8 + 2t + e ("second"), e = 0, 1.
+// 4-bit: two words per lane; word s/2, nibble 2(s%2) + 4e (first) or
+//        2(s%2) + 1 + 4e (second).  2-bit: one word; code 2s + 8e (first) or
+//        2s + 1 + 8e (second).
+__host__ __device__ inline void group_words(const uint8_t* q, int bits, int t, uint32_t* words) {
+  if (bits == 4) {
+    for (int h = 0; h < 2; ++h) {
+      uint32_t w = 0;
+      for (int j = 0; j < 2; ++j) {
+        const int s = 2 * h + j;
+        for (int e = 0; e < 2; ++e) {
+          w |= (uint32_t)q[16 * s + 2 * t + e] << (4 * (2 * j + 4 * e));
+          w |= (uint32_t)q[16 * s + 8 + 2 * t + e] << (4 * (2 * j + 1 + 4 * e));
+        }
+      }
+      words[h] = w;
+    }
+  } else {
+    uint32_t w = 0;
+    for (int s = 0; s < 4; ++s)
+      for (int e = 0; e < 2; ++e) {
+        w |= (uint32_t)q[16 * s + 2 * t + e] << (2 * (2 * s + 8 * e));
+        w |= (uint32_t)q[16 * s + 8 + 2 * t + e] << (2 * (2 * s + 1 + 8 * e));
+      }
+    words[0] = w;
+  }
+}
+
+// Store the codes and scale word of (row, group g) of a [rows][cols] matrix.
+__host__ __device__ inline void store_group(uint8_t* codes, uint8_t* scales, int bits, int cols, int row,
+                                            int g, const uint8_t* q, uint32_t sw) {
+  const size_t block = (size_t)(row / 8) * (cols / 64) + g;
+  const int n = row % 8;
+  const int wpl = bits == 4 ? 2 : 1;  // words per lane
+  uint32_t* blk = reinterpret_cast<uint32_t*>(codes + block * (size_t)(64 * bits));
+  for (int t = 0; t < 4; ++t) {
+    uint32_t words[2];
+    group_words(q, bits, t, words);
+    for (int h = 0; h < wpl; ++h) blk[(4 * n + t) * wpl + h] = words[h];
+  }
+  reinterpret_cast<uint32_t*>(scales)[block * 8 + n] = sw;
 }
 
 // ---- device packer: one thread per (expert, matrix, row, group) -------------
@@ -125,13 +167,10 @@ __global__ void pack_kernel(Layout L, const float* wg, const float* wu, const fl
     w[4 * i + 2] = v.z;
     w[4 * i + 3] = v.w;
   }
-  uint32_t words[8];
-  const uint32_t sw = quantize_group64(w, L.bits, words);
+  uint8_t q[64];
+  const uint32_t sw = quantize_group64(w, L.bits, q);
   uint8_t* blob = out + e * L.blob_bytes;
-  uint32_t* cdst = reinterpret_cast<uint32_t*>(blob + L.off_codes[m] + row * L.code_row_bytes[m] +
-                                               g * (64 * L.bits / 8));
-  for (int j = 0; j < 2 * L.bits; ++j) cdst[j] = words[j];
-  *reinterpret_cast<uint32_t*>(blob + L.off_scales[m] + row * L.scale_row_bytes[m] + g * 4) = sw;
+  store_group(blob + L.off_codes[m], blob + L.off_scales[m], L.bits, (int)cols, (int)row, (int)g, q, sw);
 }
 
 cudaError_t launch_pack(const Layout& L, const float* wg, const float* wu, const float* wd,
@@ -154,14 +193,12 @@ static void pack_one_host(const Layout& L, const float* wg, const float* wu, con
   const float* src[3] = {wg, wu, wd};
   const int rows[3] = {L.I, L.I, L.H};
   const int cols[3] = {L.H, L.H, L.I};
-  uint32_t words[8];
+  uint8_t q[64];
   for (int m = 0; m < 3; ++m)
     for (int r = 0; r < rows[m]; ++r)
       for (int g = 0; g < cols[m] / 64; ++g) {
-        const uint32_t sw = quantize_group64(src[m] + (size_t)r * cols[m] + (size_t)g * 64, L.bits, words);
-        std::memcpy(blob + L.off_codes[m] + (size_t)r * L.code_row_bytes[m] + (size_t)g * (64 * L.bits / 8),
-                    words, 8 * L.bits);
-        std::memcpy(blob + L.off_scales[m] + (size_t)r * L.scale_row_bytes[m] + (size_t)g * 4, &sw, 4);
+        const uint32_t sw = quantize_group64(src[m] + (size_t)r * cols[m] + (size_t)g * 64, L.bits, q);
+        store_group(blob + L.off_codes[m], blob + L.off_scales[m], L.bits, cols[m], r, g, q, sw);
       }
 }
 

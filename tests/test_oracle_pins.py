@@ -62,12 +62,10 @@ def _hand_cases():
         if not f:
             continue
         if f[0] == "cfg":
-            cur = dict(cfg=tuple(map(int, f[1:4])), bytes=[], scales=[], expect=[])
+            cur = dict(cfg=tuple(map(int, f[1:4])), bytes=[], expect=[])
             cases.append(cur)
         elif f[0] == "byte":
             cur["bytes"].append((int(f[1]), int(f[2]), int(f[3], 16)))
-        elif f[0] == "scale":
-            cur["scales"].append((int(f[1]), int(f[2]), int(f[3]), int(f[4], 16), int(f[5], 16)))
         elif f[0] == "expect":
             cur["expect"].append((int(f[1]), int(f[2]), int(f[3]), float(f[4])))
     return cases
@@ -81,10 +79,6 @@ def test_hand_packed_dequant(case):
     off = O.section_offsets(c)
     for sec, pos, val in case["bytes"]:
         blob[off[sec] + pos] = val
-    for m, row, grp, s, beta in case["scales"]:
-        cols = I if m == 2 else H
-        p = off[3 + m] + (row * (cols // 64) + grp) * 4
-        blob[p:p + 4] = np.frombuffer(np.uint32(s | (beta << 16)).tobytes(), dtype=np.uint8)
     for m, row, col, val in case["expect"]:
         assert O.dequant(c, blob, m, row, col) == val, (m, row, col)
 
@@ -125,18 +119,20 @@ def test_quantizer_picks_nearest_code(bits):
     wu = (g.standard_normal((64, 128)) * 0.5).astype(np.float32)
     wd = (g.standard_normal((128, 64)) * 0.02).astype(np.float32)
     blob = O.quantize_expert(c, wg, wu, wd)
-    off = O.section_offsets(c)
     qmax = 2**bits - 1
     ties = 0
     for m, w in ((0, wg), (1, wu), (2, wd)):
         rows, cols = w.shape
-        words = blob[off[3 + m]:off[3 + m] + rows * cols // 64 * 4].view(np.uint32)
-        words = words.reshape(rows, cols // 64)
         for r in range(rows):
             for grp in range(cols // 64):
                 seg = w[r, grp * 64:(grp + 1) * 64]
-                s = O.bf16_to_f64(words[r, grp] & 0xFFFF)
-                beta = O.bf16_to_f64(words[r, grp] >> 16)
+                # scale and bias from the dequantised values of two codes of the group
+                i0 = int(np.argmin([O.code(c, blob, m, r, grp * 64 + i) for i in range(64)]))
+                i1 = int(np.argmax([O.code(c, blob, m, r, grp * 64 + i) for i in range(64)]))
+                q0, q1 = O.code(c, blob, m, r, grp * 64 + i0), O.code(c, blob, m, r, grp * 64 + i1)
+                d0, d1 = O.dequant(c, blob, m, r, grp * 64 + i0), O.dequant(c, blob, m, r, grp * 64 + i1)
+                s = (d1 - d0) / (q1 - q0) if q1 != q0 else 0.0
+                beta = d0 - q0 * s
                 # scale and bias follow min and max of the group
                 assert s == O.bf16_to_f64(O.f32_to_bf16(np.float32((seg.max() - seg.min()) / np.float32(qmax))))
                 assert beta == O.bf16_to_f64(O.f32_to_bf16(seg.min()))
