@@ -177,14 +177,14 @@ size_t decode_smem_bytes(const Layout& L, int T, int nrows, int nslots, uint32_t
 
 __device__ __forceinline__ void consumer_sync() { named_sync(1, kConsumers); }
 
-// Warp-wide bounded wait on an mbarrier phase: lane 0 polls, the warp
-// synchronises on the result (other lanes see the data through __syncwarp).
+// Warp-wide bounded wait on an mbarrier phase.  Every lane polls, so the
+// warp never diverges around a wait: a warp left split into lane groups after
+// a one-lane wait runs its later warp-wide code (shuffles, mma) several times
+// slower.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
                                           uint32_t* spins = nullptr) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, timeout_ns, spins) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  return ok != 0;
+  const bool ok = mbar_wait(bar, parity, timeout_ns, (threadIdx.x & 31) == 0 ? spins : nullptr);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // Trace stamp k of this block (traced launches only; the untraced kernel
@@ -773,6 +773,8 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
     }
     good = __all_sync(0xffffffffu, good != 0) ? 1 : 0;
   }
+  // every lane's eptr store must precede lane 0's release to the producer
+  __syncwarp();
   if (lane == 0) {
     flags[FLAG_TOPK] = good;
     mbar_arrive(topkbar);
