@@ -741,14 +741,15 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
   if (lane == 0) {
     mbar_arrive(xfbar);
     trace_mark<TRACE>(p, 64);
-    // R: arrive once every consumer warp has passed the router tiles
-    if (!mbar_wait(&evt[EVT_R], 0, to, sp_evt)) ok = false;
-    red_release_add(&ctr[0], 1u);
   }
+  // R: arrive once every consumer warp has passed the router tiles.  The
+  // waits up to the top-K are warp-uniform so the top-K runs unsplit.
+  ok = warp_wait(&evt[EVT_R], 0, to, sp_evt) && ok;
+  if (lane == 0) red_release_add(&ctr[0], 1u);
+  __syncwarp();
   // top-K once every block's router logits are written
-  int good = 0;
-  if (lane == 0) good = (ok && grid_wait_thread(&ctr[0], G, &ctr[5], p.err, to, sp_grid)) ? 1 : 0;
-  good = __shfl_sync(0xffffffffu, good, 0);
+  bool gr = ok && grid_wait_thread(&ctr[0], G, &ctr[5], p.err, to, lane == 0 ? sp_grid : nullptr);
+  int good = __all_sync(0xffffffffu, gr) ? 1 : 0;
   if (lane == 0) trace_mark<TRACE>(p, 65);
   if (good) {
 #pragma unroll 1
