@@ -302,7 +302,7 @@ def print_trace(M, reps, cfg, xs, rs, h_out, y_out, stream, P, R, calls=16):
     probe = [round((b0[k] - b0[0]) / 1e3, 3) for k in range(11, 15)]
     print("trace_block0 first routed units (gate/up start, end, down start, end): %s" % probe,
           file=sys.stderr, flush=True)
-    sync = {k: round(float(np.median(rel[:, :, k])) / 1e3, 3) for k in list(range(64, 74)) + list(range(90, 100))}
+    sync = {k: round(float(np.median(rel[:, :, k])) / 1e3, 3) for k in list(range(64, 74)) + list(range(100, 104))}
     print("trace sync warp (median us): %s" % json.dumps(sync), file=sys.stderr, flush=True)
     polls = {SPIN_NAMES[k]: float(np.median(t[:, :, 80 + k])) for k in range(8)}
     print("trace polls per block (median): %s" % json.dumps(polls), file=sys.stderr, flush=True)

@@ -437,14 +437,14 @@ __device__ __noinline__ void gu_unit_done(float r00, float r01, float r10, float
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return;
   __threadfence_block();
+  // every lane runs the loop (lanes 8..31 repeat rows 0..7 and are dropped),
+  // so the warp does not diverge around it
   float g = 0.f, up = 0.f;
-  if (lane < 8) {
-    const volatile float* pp = pe + 2 * lane;
+  const volatile float* pp = pe + 2 * (lane & 7);
 #pragma unroll 1
-    for (int uu = 0; uu < U; ++uu) {
-      g += pp[uu * 16];
-      up += pp[uu * 16 + 1];
-    }
+  for (int uu = 0; uu < U; ++uu) {
+    g += pp[uu * 16];
+    up += pp[uu * 16 + 1];
   }
   if (lane == 0) cnt[e] = 0;  // entry free for a later row block
   const float h = silu_mul(g, up);
@@ -977,6 +977,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
               const float* as = gu ? xsum + (size_t)(sg.pair / K) * gh.G : hx_s + (size_t)sg.pair * (I / 8);
               float r[2][2];
               routed_unit<FMT>(sl, sg, rbl, u, gu ? gh : gi, gu, af, as, zero4, r);
+              if (TRACE && tid == 0 && !(probed & pb)) p.trace[(size_t)c * kTraceEntries + (gu ? 100 : 102)] = globaltimer_after(r[0][0]);
               if (gu) {
                 gu_unit_done(r[0][0], r[0][1], r[1][0], r[1][1], (sg.acc + rbl) % kAccSlots, u, gh.U, part, cnt,
                              sg.pair, sg.row0 + rbl, I, p.hf, p.hx);
@@ -1030,17 +1031,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       }
       // this warp is done with the slot
       __syncwarp();
-      if (lane == 0) {
-#pragma unroll 1
-        for (int k = 0; k < 3; ++k)
-          if (d.post & (F_ARRIVE_R << k)) mbar_arrive(&evt[EVT_R + k]);
-      }
-      if (tid == 0) {
-#pragma unroll 1
-        for (int k = 0; k < 3; ++k)
-          if (d.post & (F_ARRIVE_R << k)) trace_mark<TRACE>(p, 1 + k);
-      }
-      const bool end = (d.post & F_END) != 0;
+      const int post = d.post;
+      if (lane == 0 && (post & F_ARRIVE_R)) mbar_arrive(&evt[EVT_R]);
+      if (lane == 0 && (post & F_ARRIVE_S)) mbar_arrive(&evt[EVT_S]);
+      if (lane == 0 && (post & F_ARRIVE_E)) mbar_arrive(&evt[EVT_E]);
+      if (TRACE && tid == 0 && (post & F_ARRIVE_R)) trace_mark<TRACE>(p, 1);
+      if (TRACE && tid == 0 && (post & F_ARRIVE_S)) trace_mark<TRACE>(p, 2);
+      if (TRACE && tid == 0 && (post & F_ARRIVE_E)) trace_mark<TRACE>(p, 3);
+      const bool end = (post & F_END) != 0;
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
       if (tid == 0 && ntile < 16) trace_mark<TRACE>(p, 17 + 2 * ntile);

@@ -43,6 +43,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+// The same, read only once `dep` has been computed (orders a trace stamp
+// after the arithmetic that produced dep).
+__device__ __forceinline__ uint64_t globaltimer_after(float dep) {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t) : "f"(dep) : "memory");
+  return t;
+}
 
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;
