@@ -472,7 +472,10 @@ __device__ __noinline__ void gu_unit_done(float r00, float r01, float r10, float
 // One thread (lane 0 of the producer warp) builds each tile's descriptor in
 // place in shared memory once the consumers have freed the slot, announces
 // each copy's bytes on the slot's "full" barrier and issues it, and finally
-// arrives on the barrier, which completes when every copy has landed.
+// arrives on the barrier, which completes when every copy has landed.  All of
+// it is inlined so the producer's state stays in registers: the producer is
+// on the critical path of every phase, and out-of-line calls kept this state
+// in local memory at a round trip per access.
 struct Producer {
   uint8_t* ring;
   uint64_t* full;
@@ -494,7 +497,7 @@ struct Producer {
   uint32_t fill;
   uint64_t policy;  // L2 evict-first: weights are read once per launch
 
-  __device__ __noinline__ void commit() {
+  __device__ __forceinline__ void commit() {
     if (!open) return;
     if (trace && ncommit < 16) trace[48 + ncommit] = globaltimer_ns();
     ++ncommit;
@@ -505,7 +508,7 @@ struct Producer {
     }
     open = false;
   }
-  __device__ __noinline__ bool begin(int type) {
+  __device__ __forceinline__ bool begin(int type) {
     commit();
     if (!ok) return false;
     if (!mbar_wait(&empty[slot], phase ^ 1u, timeout_ns, spins)) {
@@ -539,7 +542,7 @@ struct Producer {
   // Copy a byte range into the slot; returns the slot offset of its first
   // byte.  The copy is widened to 16-byte boundaries (the widened range stays
   // inside the same 256-byte aligned section).
-  __device__ __noinline__ uint32_t range(const void* p, size_t bytes) {
+  __device__ __forceinline__ uint32_t range(const void* p, size_t bytes) {
     const uintptr_t a = reinterpret_cast<uintptr_t>(p);
     const uintptr_t al = a & ~uintptr_t(15);
     const uint32_t pad = (uint32_t)(a - al);
@@ -570,7 +573,7 @@ struct Producer {
 // segment is one row block's run of whole units [u0, u1) that fits the open
 // tile; a tile takes segments until it is full, holds kMaxSeg of them or
 // max_rb row blocks.  Each row block gets the next accumulator entry.
-__device__ __noinline__ void emit_routed(Producer& pr, int type, int bits, const size_t* off_codes,
+__device__ __forceinline__ void emit_routed(Producer& pr, int type, int bits, const size_t* off_codes,
                                          const size_t* off_scales, const uint8_t* blob, int pair, int rb_a,
                                          int rb_b, int nm, RoutedGeo geo, int max_rb, int* rbseq) {
   const uint32_t bb = 64u * (uint32_t)bits;
@@ -593,11 +596,14 @@ __device__ __noinline__ void emit_routed(Producer& pr, int type, int bits, const
       s.gbase = ga;
       s.acc = e;
       const size_t b0 = (size_t)rb * geo.G + ga;
-#pragma unroll 1
-      for (int mm = 0; mm < 2 * nm; ++mm) {
-        const bool sc = mm >= nm;
-        const uint32_t per = sc ? 32u : bb;
-        s.off[mm] = pr.range(blob + (sc ? off_scales[mm - nm] : off_codes[mm]) + b0 * per, (size_t)(gb - ga) * per);
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm) {
+        if (mm < 2 * nm) {
+          const bool sc = mm >= nm;
+          const uint32_t per = sc ? 32u : bb;
+          const size_t base = sc ? (mm - nm == 0 ? off_scales[0] : off_scales[1]) : (mm == 0 ? off_codes[0] : off_codes[1]);
+          s.off[mm] = pr.range(blob + base + b0 * per, (size_t)(gb - ga) * per);
+        }
       }
       ++pr.nrb_tile;
       u += un;
@@ -607,7 +613,7 @@ __device__ __noinline__ void emit_routed(Producer& pr, int type, int bits, const
 
 // bf16 rows [a, b) of one or two row-major matrices (row_bytes each), as many
 // rows per tile as fit.
-__device__ __noinline__ void emit_rows(Producer& pr, int type, const uint8_t* m0, const uint8_t* m1,
+__device__ __forceinline__ void emit_rows(Producer& pr, int type, const uint8_t* m0, const uint8_t* m1,
                                        uint32_t row_bytes, int a, int b) {
   const uint32_t nm = m1 ? 2u : 1u;
   const int cap = max(1, min(1024, (int)((pr.slot_bytes - 16u * nm) / (nm * row_bytes))));
