@@ -319,38 +319,74 @@ struct LaneCodes<FMT_Q2> {
   }
 };
 
-// One unit of a routed tile: windows [u*W, u*W + W) of 8-row block `rbl` of
-// the segment.  gu: gate and up against x (bf16, A rows 0..7); otherwise down
-// against the routed intermediate (hi in A rows 0..7, lo in rows 8..15).
-// afrag: this token's (pair's) A fragments; asum: its group sums (gu) or
-// 8-row partial sums (down).  Returns rows 2t and 2t+1 of the block in
-// res[matrix][0/1] (every lane t, t = lane % 4, holds the sums of its rows).
+// Shared-memory loads at 32-bit shared addresses (no generic address math).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds32f(uint32_t a) { return __uint_as_float(lds32(a)); }
+
 template <int FMT>
-__device__ __forceinline__ void routed_unit(const uint8_t* sl, const Seg& sg, int rbl, int u, const RoutedGeo& geo,
-                                            bool gu, const uint4* afrag, const float* asum, const uint4* zero4,
-                                            float (&res)[2][2]) {
+__device__ __forceinline__ void load_codes(LaneCodes<FMT>& c, uint32_t a);
+template <>
+__device__ __forceinline__ void load_codes<FMT_Q4>(LaneCodes<FMT_Q4>& c, uint32_t a) { c.w = lds64(a); }
+template <>
+__device__ __forceinline__ void load_codes<FMT_Q2>(LaneCodes<FMT_Q2>& c, uint32_t a) { c.w = lds32(a); }
+
+// One unit of a routed tile: windows [u*W, u*W + W) of 8-row block `rbl` of
+// the segment.  GU: gate and up against x (bf16, A rows 0..7); otherwise down
+// against the routed intermediate (hi in A rows 0..7, lo in rows 8..15).
+// afrag: this token's (pair's) A fragments; asum: its group sums (GU) or
+// 8-row partial sums (down); sl, afrag, asum, zero4 are shared-memory
+// addresses.  Returns rows 2t and 2t+1 of the block in res[matrix][0/1]
+// (every lane t, t = lane % 4, holds the sums of its rows).
+template <int FMT, bool GU>
+__device__ __forceinline__ void routed_unit(uint32_t sl, const Seg& sg, int rbl, int u, const RoutedGeo& geo,
+                                            uint32_t afrag, uint32_t asum, uint32_t zero4, float (&res)[2][2]) {
+  constexpr int NM = GU ? 2 : 1;
+  constexpr int NA = GU ? 2 : 4;  // 16-byte A pieces per lane and group
   constexpr int CB = LaneCodes<FMT>::kBytes;
   constexpr int BB = 32 * CB;  // code bytes of one 8x64 block
   const int lane = threadIdx.x & 31, m = lane >> 2, t = lane & 3;
-  const int na = gu ? 2 : 4;  // 16-byte A pieces per lane and group
-  const int nm = gu ? 2 : 1;
-  float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  float acc[NM][2];
+#pragma unroll
+  for (int mm = 0; mm < NM; ++mm) acc[mm][0] = acc[mm][1] = 0.f;
   const int wa = u * geo.W, wb = min(wa + geo.W, geo.nwin);
   const int blk0 = rbl * geo.G - sg.gbase;
+  uint32_t cbase[NM], sbase[NM];
+#pragma unroll
+  for (int mm = 0; mm < NM; ++mm) {
+    cbase[mm] = sl + sg.off[mm] + (uint32_t)(blk0 * BB + lane * CB);
+    sbase[mm] = sl + sg.off[NM + mm] + (uint32_t)(blk0 * 32 + t * 8);
+  }
 #pragma unroll 1
   for (int w = wa; w < wb; ++w) {
     const int g0 = 8 * w, nv = min(8, geo.G - g0);
-    float d[2][4][4];
+    float d[NM][4][4];
 #pragma unroll
-    for (int mm = 0; mm < 2; ++mm)
+    for (int mm = 0; mm < NM; ++mm)
 #pragma unroll
       for (int s = 0; s < 4; ++s) d[mm][s][0] = d[mm][s][1] = d[mm][s][2] = d[mm][s][3] = 0.f;
+    // lane group m presents group g0 + m's activations in step j == m only
+    const uint32_t a_own = afrag + (uint32_t)(((g0 + m) * 4 + t) * NA * 16);
+    const uint32_t cw = (uint32_t)(g0 * BB);
 #pragma unroll 1
     for (int j = 0; j < nv; ++j) {
-      const uint4* ap = (m == j) ? afrag + ((size_t)(g0 + j) * 4 + t) * na : zero4;
+      const uint32_t ap = (m == j) ? a_own : zero4;
       uint32_t a[4][4];
-      if (gu) {
-        const uint4 v0 = ap[0], v1 = ap[1];
+      if constexpr (GU) {
+        const uint4 v0 = lds128(ap), v1 = lds128(ap + 16);
         a[0][0] = v0.x, a[0][2] = v0.y, a[1][0] = v0.z, a[1][2] = v0.w;
         a[2][0] = v1.x, a[2][2] = v1.y, a[3][0] = v1.z, a[3][2] = v1.w;
 #pragma unroll
@@ -358,48 +394,45 @@ __device__ __forceinline__ void routed_unit(const uint8_t* sl, const Seg& sg, in
       } else {
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
-          const uint4 v = ap[s];
+          const uint4 v = lds128(ap + 16 * s);
           a[s][0] = v.x, a[s][1] = v.y, a[s][2] = v.z, a[s][3] = v.w;
         }
       }
-      const size_t boff = (size_t)(blk0 + g0 + j) * BB + lane * CB;
+      LaneCodes<FMT> c[NM];
 #pragma unroll
-      for (int mm = 0; mm < 2; ++mm) {
-        if (mm < nm) {
-          LaneCodes<FMT> c;
-          c.load(sl + sg.off[mm] + boff);
-          uint32_t b[4][2];
-          c.frags(b);
+      for (int mm = 0; mm < NM; ++mm) load_codes<FMT>(c[mm], cbase[mm] + cw + (uint32_t)(j * BB));
 #pragma unroll
-          for (int s = 0; s < 4; ++s) mma_16816(d[mm][s], a[s][0], a[s][1], a[s][2], a[s][3], b[s][0], b[s][1]);
-        }
+      for (int mm = 0; mm < NM; ++mm) {
+        uint32_t b[4][2];
+        c[mm].frags(b);
+#pragma unroll
+        for (int s = 0; s < 4; ++s) mma_16816(d[mm][s], a[s][0], a[s][1], a[s][2], a[s][3], b[s][0], b[s][1]);
       }
     }
     // lane group m owns group g0 + m: rows 2t, 2t+1
     if (m < nv) {
       const int g = g0 + m;
       float X;
-      if (gu) {
-        X = asum[g];
+      if constexpr (GU) {
+        X = lds32f(asum + 4 * g);
       } else {
-        const float4 p0 = *reinterpret_cast<const float4*>(asum + 8 * g);
-        const float4 p1 = *reinterpret_cast<const float4*>(asum + 8 * g + 4);
-        X = ((p0.x + p0.y) + (p0.z + p0.w)) + ((p1.x + p1.y) + (p1.z + p1.w));
+        const uint4 p0 = lds128(asum + 32 * g), p1 = lds128(asum + 32 * g + 16);
+        X = ((__uint_as_float(p0.x) + __uint_as_float(p0.y)) + (__uint_as_float(p0.z) + __uint_as_float(p0.w))) +
+            ((__uint_as_float(p1.x) + __uint_as_float(p1.y)) + (__uint_as_float(p1.z) + __uint_as_float(p1.w)));
       }
 #pragma unroll
-      for (int mm = 0; mm < 2; ++mm) {
-        if (mm < nm) {
-          const uint2 sw = *reinterpret_cast<const uint2*>(sl + sg.off[nm + mm] + (size_t)(blk0 + g) * 32 + t * 8);
-          // rows m (hi) and m + 8 (lo, zero for gate/up) of D
-          const float D0 = ((d[mm][0][0] + d[mm][1][0]) + (d[mm][2][0] + d[mm][3][0])) +
-                           ((d[mm][0][2] + d[mm][1][2]) + (d[mm][2][2] + d[mm][3][2]));
-          const float D1 = ((d[mm][0][1] + d[mm][1][1]) + (d[mm][2][1] + d[mm][3][1])) +
-                           ((d[mm][0][3] + d[mm][1][3]) + (d[mm][2][3] + d[mm][3][3]));
-          const float s0 = __uint_as_float(sw.x << 16), b0 = __uint_as_float(sw.x & 0xffff0000u);
-          const float s1 = __uint_as_float(sw.y << 16), b1 = __uint_as_float(sw.y & 0xffff0000u);
-          acc[mm][0] = fmaf(s0, D0, fmaf(fmaf(-128.f, s0, b0), X, acc[mm][0]));
-          acc[mm][1] = fmaf(s1, D1, fmaf(fmaf(-128.f, s1, b1), X, acc[mm][1]));
+      for (int mm = 0; mm < NM; ++mm) {
+        const uint2 sw = lds64(sbase[mm] + (uint32_t)(g * 32));
+        float D0 = (d[mm][0][0] + d[mm][1][0]) + (d[mm][2][0] + d[mm][3][0]);
+        float D1 = (d[mm][0][1] + d[mm][1][1]) + (d[mm][2][1] + d[mm][3][1]);
+        if constexpr (!GU) {  // rows m + 8 of D: the lo parts of the intermediate
+          D0 += (d[mm][0][2] + d[mm][1][2]) + (d[mm][2][2] + d[mm][3][2]);
+          D1 += (d[mm][0][3] + d[mm][1][3]) + (d[mm][2][3] + d[mm][3][3]);
         }
+        const float s0 = __uint_as_float(sw.x << 16), b0 = __uint_as_float(sw.x & 0xffff0000u);
+        const float s1 = __uint_as_float(sw.y << 16), b1 = __uint_as_float(sw.y & 0xffff0000u);
+        acc[mm][0] = fmaf(s0, D0, fmaf(fmaf(-128.f, s0, b0), X, acc[mm][0]));
+        acc[mm][1] = fmaf(s1, D1, fmaf(fmaf(-128.f, s1, b1), X, acc[mm][1]));
       }
     }
   }
@@ -407,7 +440,7 @@ __device__ __forceinline__ void routed_unit(const uint8_t* sl, const Seg& sg, in
   for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      float v = acc[mm][k];
+      float v = mm < NM ? acc[mm < NM ? mm : 0][k] : 0.f;
       v += __shfl_xor_sync(0xffffffffu, v, 4);
       v += __shfl_xor_sync(0xffffffffu, v, 8);
       v += __shfl_xor_sync(0xffffffffu, v, 16);
@@ -934,6 +967,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     bool have_xf = false;
     int item = 0;  // running count of work items over the compute tiles
     int probed = 0;  // first routed units traced: bit 0 gate/up, bit 1 down
+    int nunit = 0;   // routed units done by this warp (traced launches)
     uint32_t slot = 0, phase = 0;
 #pragma unroll 1
     for (int ntile = 0;; ++ntile) {
@@ -978,12 +1012,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
               const int rbl = j / nu, u = sg.u0 + (j - rbl * nu);
               const int pb = gu ? 1 : 2;
               if (tid == 0 && !(probed & pb)) trace_mark<TRACE>(p, gu ? 11 : 13);
-              const uint4* af = gu ? xf + (size_t)(sg.pair / K) * gh.G * 8
-                                   : reinterpret_cast<const uint4*>(hf_s) + (size_t)sg.pair * gi.G * 16;
-              const float* as = gu ? xsum + (size_t)(sg.pair / K) * gh.G : hx_s + (size_t)sg.pair * (I / 8);
               float r[2][2];
-              routed_unit<FMT>(sl, sg, rbl, u, gu ? gh : gi, gu, af, as, zero4, r);
+              const uint64_t tu0 = TRACE ? globaltimer_ns() : 0;
+              if (gu)
+                routed_unit<FMT, true>(smem_u32(sl), sg, rbl, u, gh, smem_u32(xf + (size_t)(sg.pair / K) * gh.G * 8),
+                                       smem_u32(xsum + (size_t)(sg.pair / K) * gh.G), smem_u32(zero4), r);
+              else
+                routed_unit<FMT, false>(smem_u32(sl), sg, rbl, u, gi, smem_u32(hf_s + (size_t)sg.pair * gi.G * 256),
+                                        smem_u32(hx_s + (size_t)sg.pair * (I / 8)), smem_u32(zero4), r);
               if (TRACE && tid == 0 && !(probed & pb)) p.trace[(size_t)c * kTraceEntries + (gu ? 100 : 102)] = globaltimer_after(r[0][0]);
+              if (TRACE && tid == 0 && nunit < 8) {
+                p.trace[(size_t)c * kTraceEntries + 104 + 2 * nunit] = tu0;
+                p.trace[(size_t)c * kTraceEntries + 105 + 2 * nunit] = globaltimer_after(r[0][0] + r[1][1]);
+              }
+              if (TRACE) ++nunit;
               if (gu) {
                 gu_unit_done(r[0][0], r[0][1], r[1][0], r[1][1], (sg.acc + rbl) % kAccSlots, u, gh.U, part, cnt,
                              sg.pair, sg.row0 + rbl, I, p.hf, p.hx);
