@@ -169,6 +169,28 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts
                              float* w_out, void* workspace, size_t ws_bytes,
                              cudaStream_t stream);
 
+/* Allocation-free variant of moe_layer_forward.  The pages have no
+ * counterpart: their engine owns all of its buffers.  It is for callers that
+ * must not allocate device memory (a fixed memory budget, or a loop where
+ * cudaMalloc -- which can synchronise the device and can fail under memory
+ * pressure -- is not allowed) and that keep no workspace of their own: the
+ * scratch is a MOE_NOALLOC_SCRATCH_BYTES area inside the library (a device
+ * array of the loaded module), so the call allocates nothing.
+ * Arguments and results are those of moe_layer_forward, without the
+ * workspace.  A shape whose moe_layer_workspace_bytes exceeds
+ * MOE_NOALLOC_SCRATCH_BYTES is rejected with MOE_ERR_WORKSPACE.
+ * The first call on a device (with that device current) looks the scratch up
+ * and zeroes its counters with synchronous CUDA calls: make it before any
+ * stream capture.  All calls on a device share the one scratch, so calls that
+ * may overlap in time (other streams, other host threads) race and must be
+ * serialised by the caller.  Device-side wait timeouts of this path are not
+ * readable through moe_device_error (the scratch is internal). */
+#define MOE_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+moe_status moe_layer_forward_noalloc(const moe_config* cfg, const moe_layer_weights* wts,
+                                     const void* x_bf16, const void* residual_bf16, int T,
+                                     void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
+                                     float* w_out, cudaStream_t stream);
+
 /* Per-phase timing of one layer call, in the spirit of the pages' per-layer
  * --timing breakdown ("Flash-MoE: ...", section "パイプライン概要"): the same
  * computation as moe_layer_forward (idx/w outputs omitted), and every block

@@ -22,6 +22,8 @@ if not os.path.exists(LIB_PATH):
 _lib = C.CDLL(LIB_PATH)
 
 MOE_OK = 0
+MOE_ERR_WORKSPACE = 3
+NOALLOC_SCRATCH_BYTES = 4 << 20  # MOE_NOALLOC_SCRATCH_BYTES of moe.h
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_OOM", 6: "MOE_ERR_TIMEOUT", 7: "MOE_ERR_IO",
           8: "MOE_ERR_DEVICE"}
@@ -70,6 +72,8 @@ EXPORTS = {
     "moe_layer_forward_traced": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p,
                                            C.c_size_t, C.c_void_p]),
+    "moe_layer_forward_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "moe_device_error": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
     "moe_selftest_bounded_wait": (C.c_int, [C.c_void_p, C.c_size_t, C.c_uint64, C.c_void_p]),
 }
@@ -200,6 +204,13 @@ def moe_layer_forward(cfg, wts, x, residual, h_out, y_norm, idx_out=None, w_out=
     _check(_lib.moe_layer_forward(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T, _ptr(h_out),
                                   _ptr(y_norm), _ptr(idx_out), _ptr(w_out), _ptr(workspace),
                                   workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_layer_forward_noalloc(cfg, wts, x, residual, h_out, y_norm, idx_out=None, w_out=None, stream=None):
+    """moe_layer_forward on the library's built-in scratch (no workspace)."""
+    T = x.shape[0]
+    _check(_lib.moe_layer_forward_noalloc(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T, _ptr(h_out),
+                                          _ptr(y_norm), _ptr(idx_out), _ptr(w_out), _stream(stream)))
 
 
 def moe_layer_trace_blocks():

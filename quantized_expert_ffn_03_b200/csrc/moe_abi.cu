@@ -306,6 +306,19 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
   return ok();
 }
 
+namespace moe {
+// For the library's other translation units: record an error message, and
+// run the fused layer on a given workspace.
+moe_status abi_fail(moe_status s, const char* msg) { return fail(s, "%s", msg); }
+moe_status layer_forward_on(const moe_config* cfg, const moe_layer_weights* wts, const void* x_bf16,
+                            const void* residual_bf16, int T, void* h_out_bf16, void* y_norm_bf16,
+                            int32_t* idx_out, float* w_out, void* workspace, size_t ws_bytes,
+                            cudaStream_t stream) {
+  return layer_forward_impl(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out,
+                            workspace, ws_bytes, nullptr, 0, stream);
+}
+}  // namespace moe
+
 extern "C" {
 
 moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts,
