@@ -1043,6 +1043,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
               const int cols = down ? I : H;
               const uint8_t* w0 = sl + sg.off[0] + (size_t)j * 2 * cols;
               const int row = sg.row0 + j;
+              // the router bias is a global load: issue it before the dot
+              const float rbias = (type == TILE_ROUTER && p.bias) ? __ldg(p.bias + row) : 0.f;
 #pragma unroll 1
               for (int t0 = 0; t0 < T; t0 += 4) {
                 const int nt = min(4, T - t0);
@@ -1064,7 +1066,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
                   if (type == TILE_SHARED_GU) a1 = warp_sum(a1);
                   if (lane == 0) {
                     if (type == TILE_ROUTER)
-                      p.logits[(size_t)t * L.E + row] = a0 + (p.bias ? p.bias[row] : 0.f);
+                      p.logits[(size_t)t * L.E + row] = a0 + rbias;
                     else if (type == TILE_SHARED_GU)
                       p.hs[(size_t)t * I + row] = silu_mul(a0, a1);
                     else

@@ -188,8 +188,21 @@ static __device__ __noinline__ void warp_topk(const float* vals, int E, int K, i
 static __device__ __noinline__ void warp_topk_keys(const float* logits, int E, int K, uint64_t* keys,
                                                    int32_t* idx, float* w) {
   const int lane = threadIdx.x & 31;
-#pragma unroll 4
-  for (int e = lane; e < E; e += 32) keys[e] = topk_key(__ldcg(logits + e), e);
+  // 16 independent loads per lane in flight: one round trip for E <= 512
+#pragma unroll 1
+  for (int e0 = 0; e0 < E; e0 += 512) {
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = e0 + lane + 32 * i;
+      v[i] = e < E ? __ldcg(logits + e) : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = e0 + lane + 32 * i;
+      if (e < E) keys[e] = topk_key(v[i], e);
+    }
+  }
   __syncwarp();
   uint64_t prev = ~0ull;
 #pragma unroll 1
