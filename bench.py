@@ -221,12 +221,14 @@ def run_reference(args):
     s = workload(args.bits)
     # each step is one token through the oracle; the run is capped so that the
     # whole --steps/--warmup invocation ends within a few minutes
-    rate1, _, t1 = oracle_token_rate(s, 1)
-    n = max(1, min(args.steps, int(150.0 / max(t1, 1e-3))))
+    # warm-up tokens (at most 3, at least 1), which also size the timed run
+    nw = max(1, min(args.warmup, 3))
+    rate1, _, t1 = oracle_token_rate(s, nw)
+    n = max(1, min(args.steps, int(150.0 / max(t1 / nw, 1e-3))))
     rate, done, dt = oracle_token_rate(s, n, seconds_cap=150.0)
     line = {
         "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": done, "warmup": 1, "ms_per_step": 1e3 * dt / done, "higher_is_better": True,
+        "steps": done, "warmup": nw, "ms_per_step": 1e3 * dt / done, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": s.name, "hidden": s.hidden, "inter": s.inter, "n_experts": s.n_experts,
                    "top_k": s.top_k, "bits": s.bits, "tokens_per_step": 1},
@@ -303,6 +305,9 @@ def print_trace(M, reps, cfg, xs, rs, h_out, y_out, stream, P, R, calls=16):
     print("trace_block0 first routed units (gate/up start, end, down start, end): %s" % probe,
           file=sys.stderr, flush=True)
     sync = {k: round(float(np.median(rel[:, :, k])) / 1e3, 3) for k in list(range(64, 74)) + list(range(100, 104))}
+    units = [(round((b0[104 + 2 * n] - b0[0]) / 1e3, 2), round((b0[105 + 2 * n] - b0[104 + 2 * n]) / 1e3, 2))
+             for n in range(8) if b0[104 + 2 * n] > 0]
+    print("trace_block0 warp0 routed units (start, duration): %s" % units, file=sys.stderr, flush=True)
     print("trace sync warp (median us): %s" % json.dumps(sync), file=sys.stderr, flush=True)
     polls = {SPIN_NAMES[k]: float(np.median(t[:, :, 80 + k])) for k in range(8)}
     print("trace polls per block (median): %s" % json.dumps(polls), file=sys.stderr, flush=True)

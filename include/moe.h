@@ -24,8 +24,7 @@
  * Conventions for every call:
  *   - Pointers are owned by the caller.  Device pointers are CUDA global
  *     memory on the current device; host pointers are ordinary host memory
- *     (pinned where stated).  The library allocates device memory only inside
- *     a streaming-cache handle (moe_stream_create).
+ *     (pinned where stated).  The library allocates no device memory.
  *   - Device calls are asynchronous on the given stream and do not
  *     synchronise unless stated.  Inputs are never modified.
  *   - Every call returns a moe_status.  On MOE_OK all outputs are fully
@@ -54,7 +53,7 @@ typedef enum {
   MOE_ERR_CUDA = 4,        /* a CUDA runtime call failed (message has the CUDA error) */
   MOE_ERR_OOM = 5,         /* a device or pinned-host allocation failed */
   MOE_ERR_TIMEOUT = 6,     /* a bounded device-side wait expired (see moe_device_error) */
-  MOE_ERR_IO = 7,          /* a host-store copy of the streaming tier failed */
+  MOE_ERR_IO = 7,          /* reserved for the expert-streaming tier (host-store copies) */
   MOE_ERR_DEVICE = 8       /* a device-side check failed (misaligned expert pointer, bad expert id) */
 } moe_status;
 
@@ -77,8 +76,19 @@ const char* moe_last_error(void);
  * 256-byte boundary:
  *   0 gate codes [I][H*b/8]   1 up codes [I][H*b/8]   2 down codes [H][I*b/8]
  *   3 gate scales [I][H/G]    4 up scales [I][H/G]    5 down scales [H][I/G]
- * Codes: row-major; little-endian 32-bit words; word j of a row holds columns
- * j*(32/b) .. j*(32/b)+32/b-1, column j*(32/b)+n at bits n*b .. n*b+b-1.
+ * Codes come in blocks of 8 rows x 64 columns (one group of 8 rows), ordered
+ * by row block, then column group; a block is 64*b bytes.  Inside a block,
+ * "lane" l = 4*(row % 8) + t (t = 0..3) owns 2*b consecutive bytes
+ * (little-endian 32-bit words) holding, for each 16-column step s = 0..3 of
+ * the group, the columns 16s + 2t + e ("first") and 16s + 8 + 2t + e
+ * ("second"), e = 0, 1 -- the codes a tensor-core B fragment of an m16n8k16
+ * step takes for that lane:
+ *   4-bit: word s/2; code at nibble 2(s%2) + 4e (first) or 2(s%2) + 1 + 4e
+ *          (second);
+ *   2-bit: one word; code at 2-bit slot 2s + 8e (first) or 2s + 1 + 8e
+ *          (second).
+ * Scale words are stored [row block][group][row % 8].  A run of whole row
+ * blocks is therefore one contiguous byte range in both sections.
  * Scale word (uint32): bf16 scale s in bits 0..15, bf16 bias beta in bits
  * 16..31; weight = q*s + beta.  Groups run along the input (reduction) dim.
  * Quantiser (round-to-nearest affine, single precision):
