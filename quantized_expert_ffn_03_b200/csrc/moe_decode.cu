@@ -97,7 +97,7 @@ struct TileDesc {
 // barriers consumers -> sync warp (evt) and sync warp -> consumers (go)
 enum { EVT_R = 0, EVT_S, EVT_E, EVT_D, NEVT };
 enum { GO_S = 0, GO_E, GO_D, NGO };
-enum { FLAG_TOPK = NGO };  // flags[] slot: routing valid
+enum { FLAG_TOPK = NGO, FLAG_SCNT };  // flags[] slots: routing valid; consumer warps past the S tiles
 
 // ---- shared-memory plan ------------------------------------------------------
 // xf: x as mma A fragments, [token][group][t][8 words]; word 2s is the bf16
@@ -336,6 +336,63 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   return v;
 }
 __device__ __forceinline__ float lds32f(uint32_t a) { return __uint_as_float(lds32(a)); }
+
+// One token's dot products with NM bf16 rows (NM = 1 or 2) over `cols`
+// columns (a multiple of 8): w0, w1 (bf16 rows), x (bf16, or fp32 when XF32)
+// and zero (64 zero bytes) are shared-memory addresses.  Each lane keeps four
+// 256-column chunks in flight, each with its own accumulator pair; chunks
+// past the end read the zero bytes.  Returns this lane's sums (the caller
+// reduces over the warp).
+template <int NM, bool XF32>
+__device__ __forceinline__ void row_dot_t1(uint32_t w0, uint32_t w1, uint32_t x, int cols, uint32_t zero,
+                                           float (&out)[NM]) {
+  const int lane = threadIdx.x & 31;
+  float2 a[NM][4];
+#pragma unroll
+  for (int m = 0; m < NM; ++m)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) a[m][k] = make_float2(0.f, 0.f);
+#pragma unroll 1
+  for (int c = 8 * lane; c < cols; c += 1024) {
+    uint4 q[NM][4], xv[4][XF32 ? 2 : 1];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int ck = c + 256 * k;
+      const bool in = ck < cols;
+      q[0][k] = lds128(in ? w0 + 2u * ck : zero);
+      if constexpr (NM == 2) q[1][k] = lds128(in ? w1 + 2u * ck : zero);
+      if constexpr (XF32) {
+        xv[k][0] = lds128(in ? x + 4u * ck : zero);
+        xv[k][XF32 ? 1 : 0] = lds128(in ? x + 4u * ck + 16u : zero + 16u);
+      } else {
+        xv[k][0] = lds128(in ? x + 2u * ck : zero);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float xx[8];
+      if constexpr (XF32) {
+        const uint4 u = xv[k][0], v = xv[k][XF32 ? 1 : 0];
+        xx[0] = __uint_as_float(u.x), xx[1] = __uint_as_float(u.y), xx[2] = __uint_as_float(u.z);
+        xx[3] = __uint_as_float(u.w), xx[4] = __uint_as_float(v.x), xx[5] = __uint_as_float(v.y);
+        xx[6] = __uint_as_float(v.z), xx[7] = __uint_as_float(v.w);
+      } else {
+        unpack_bf16x8(xv[k][0], xx);
+      }
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        const uint32_t wq[4] = {q[m][k].x, q[m][k].y, q[m][k].z, q[m][k].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          a[m][k] = __ffma2_rn(make_float2(__uint_as_float(wq[i] << 16), __uint_as_float(wq[i] & 0xffff0000u)),
+                               make_float2(xx[2 * i], xx[2 * i + 1]), a[m][k]);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < NM; ++m)
+    out[m] = ((a[m][0].x + a[m][0].y) + (a[m][1].x + a[m][1].y)) + ((a[m][2].x + a[m][2].y) + (a[m][3].x + a[m][3].y));
+}
 
 template <int FMT>
 __device__ __forceinline__ void load_codes(LaneCodes<FMT>& c, uint32_t a);
@@ -689,6 +746,12 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
               2u * H, a, b);
   }
   pr.post(F_ARRIVE_S);
+  // the shared expert's down rows of this block: they wait for every block's
+  // shared intermediate (S), which is staged while the routing is found
+  if (L.has_shared) {
+    pr.pre(F_WAIT_S);
+    emit_rows(pr, TILE_SHARED_DOWN, reinterpret_cast<const uint8_t*>(p.sd), nullptr, 2u * I, r0, r1);
+  }
   // the routing, from the sync warp
   bool routed = false;
   if (pr.ok) {
@@ -718,8 +781,6 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
     }
   }
   pr.post(F_ARRIVE_E);
-  pr.pre(F_WAIT_S);
-  if (L.has_shared) emit_rows(pr, TILE_SHARED_DOWN, reinterpret_cast<const uint8_t*>(p.sd), nullptr, 2u * I, r0, r1);
   pr.pre(F_WAIT_E);
   if (routed && r1 > r0) {
 #pragma unroll 1
@@ -819,37 +880,24 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
     flags[FLAG_TOPK] = good;
     mbar_arrive(topkbar);
     trace_mark<TRACE>(p, 67);
-    // S and E: arrive once every consumer warp has passed the phase's tiles
-#pragma unroll 1
-    for (int k = EVT_S; k <= EVT_E; ++k) {
-      if (!mbar_wait(&evt[k], 0, to, sp_evt)) ok = false;
-      red_release_add(&ctr[k], 1u);
-      trace_mark<TRACE>(p, 68 + k - EVT_S);
+    // E: arrive once every consumer warp has passed the routed gate/up
+    // tiles, wait for every block, stage the routed intermediate, release
+    // the consumers (S is handled by the consumer warps themselves)
+    if (!mbar_wait(&evt[EVT_E], 0, to, sp_evt)) ok = false;
+    red_release_add(&ctr[2], 1u);
+    trace_mark<TRACE>(p, 69);
+    bool ge = ok && good != 0;
+    if (ge) ge = grid_wait_thread(&ctr[2], G, &ctr[5], p.err, to, sp_grid);
+    trace_mark<TRACE>(p, 71);
+    flags[GO_E] = ge ? 1 : 0;
+    if (ge) {
+      fence_proxy_async_global();
+      const uint32_t hfb = (uint32_t)(4ull * T * K * L.I), hxb = (uint32_t)(4ull * T * K * (L.I / 8));
+      mbar_expect_tx(&go[GO_E], hfb + hxb);
+      bulk_g2s(hf_s, p.hf, hfb, &go[GO_E]);
+      bulk_g2s(hx_s, p.hx, hxb, &go[GO_E]);
     }
-    // wait S, then E; stage the intermediates; release the consumers
-#pragma unroll 1
-    for (int k = 0; k < 2; ++k) {
-      bool g = ok;
-      const bool need = k == 1 ? good != 0 : L.has_shared != 0;
-      if (g && need) g = grid_wait_thread(&ctr[1 + k], G, &ctr[5], p.err, to, sp_grid);
-      trace_mark<TRACE>(p, 70 + k);
-      flags[GO_S + k] = g ? 1 : 0;
-      uint64_t* bar = &go[GO_S + k];
-      if (g && need) {
-        fence_proxy_async_global();
-        if (k == 0) {
-          const uint32_t bytes = (uint32_t)(4ull * T * L.I);
-          mbar_expect_tx(bar, bytes);
-          bulk_g2s(hs_s, p.hs, bytes, bar);
-        } else {
-          const uint32_t hfb = (uint32_t)(4ull * T * K * L.I), hxb = (uint32_t)(4ull * T * K * (L.I / 8));
-          mbar_expect_tx(bar, hfb + hxb);
-          bulk_g2s(hf_s, p.hf, hfb, bar);
-          bulk_g2s(hx_s, p.hx, hxb, bar);
-        }
-      }
-      mbar_arrive(bar);
-    }
+    mbar_arrive(&go[GO_E]);
     // D: sum of squares written -> arrive, wait, release the consumers
     if (!mbar_wait(&evt[EVT_D], 0, to, sp_evt)) ok = false;
     red_release_add(&ctr[3], 1u);
@@ -923,6 +971,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   if (tid < 16) {
     zero4[tid >> 2] = make_uint4(0u, 0u, 0u, 0u);
     spin_s[tid] = 0u;
+    flags[tid] = 0;
   }
   if (tid < kAccSlots) cnt[tid] = 0;
   __syncthreads();
@@ -1045,6 +1094,36 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
               const int row = sg.row0 + j;
               // the router bias is a global load: issue it before the dot
               const float rbias = (type == TILE_ROUTER && p.bias) ? __ldg(p.bias + row) : 0.f;
+              if (T == 1) {
+                // one token: the chunked dot, no per-token branches
+                const uint32_t zs = smem_u32(zero4);
+                float v0, v1 = 0.f;
+                if (down) {
+                  float o[1];
+                  row_dot_t1<1, true>(smem_u32(w0), 0u, smem_u32(hs_s), I, zs, o);
+                  v0 = o[0];
+                } else if (type == TILE_SHARED_GU) {
+                  float o[2];
+                  row_dot_t1<2, false>(smem_u32(w0), smem_u32(sl + sg.off[1] + (size_t)j * 2 * cols), smem_u32(xs),
+                                       H, zs, o);
+                  v0 = o[0];
+                  v1 = warp_sum(o[1]);
+                } else {
+                  float o[1];
+                  row_dot_t1<1, false>(smem_u32(w0), 0u, smem_u32(xs), H, zs, o);
+                  v0 = o[0];
+                }
+                v0 = warp_sum(v0);
+                if (lane == 0) {
+                  if (type == TILE_ROUTER)
+                    p.logits[row] = v0 + rbias;
+                  else if (type == TILE_SHARED_GU)
+                    p.hs[row] = silu_mul(v0, v1);
+                  else
+                    ys[row - r0] = v0;
+                }
+                continue;
+              }
 #pragma unroll 1
               for (int t0 = 0; t0 < T; t0 += 4) {
                 const int nt = min(4, T - t0);
@@ -1083,7 +1162,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       __syncwarp();
       const int post = d.post;
       if (lane == 0 && (post & F_ARRIVE_R)) mbar_arrive(&evt[EVT_R]);
-      if (lane == 0 && (post & F_ARRIVE_S)) mbar_arrive(&evt[EVT_S]);
       if (lane == 0 && (post & F_ARRIVE_E)) mbar_arrive(&evt[EVT_E]);
       if (TRACE && tid == 0 && (post & F_ARRIVE_R)) trace_mark<TRACE>(p, 1);
       if (TRACE && tid == 0 && (post & F_ARRIVE_S)) trace_mark<TRACE>(p, 2);
@@ -1092,6 +1170,39 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
       if (tid == 0 && ntile < 16) trace_mark<TRACE>(p, 17 + 2 * ntile);
+      if (post & F_ARRIVE_S) {
+        // S (after the slot is released): the last consumer warp past the
+        // shared gate/up tiles arrives for the block, waits for every block
+        // and stages the shared intermediate (warp-uniform, while the routing
+        // is still being found)
+        int last = 0;
+        if (lane == 0) {
+          __threadfence();
+          last = atomicAdd(&flags[FLAG_SCNT], 1) == kConsumerWarps - 1 ? 1 : 0;
+        }
+        if (__shfl_sync(0xffffffffu, last, 0)) {
+          if (lane == 0) {
+            __threadfence();
+            red_release_add(&ctr[1], 1u);
+            trace_mark<TRACE>(p, 68);
+          }
+          __syncwarp();
+          const bool need = L.has_shared != 0;
+          const bool gw = ok && (!need || grid_wait_thread(&ctr[1], G, &ctr[5], p.err, p.timeout_ns));
+          const bool gs = __all_sync(0xffffffffu, gw);
+          if (lane == 0) {
+            trace_mark<TRACE>(p, 70);
+            flags[GO_S] = gs ? 1 : 0;
+            if (gs && need) {
+              fence_proxy_async_global();
+              const uint32_t bytes = (uint32_t)(4ull * T * I);
+              mbar_expect_tx(&go[GO_S], bytes);
+              bulk_g2s(hs_s, p.hs, bytes, &go[GO_S]);
+            }
+            mbar_arrive(&go[GO_S]);
+          }
+        }
+      }
       if (++slot == (uint32_t)nslots) {
         slot = 0;
         phase ^= 1u;

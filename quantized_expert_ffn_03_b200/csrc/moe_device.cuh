@@ -182,43 +182,82 @@ static __device__ __noinline__ void warp_topk(const float* vals, int E, int K, i
 }
 
 // The same for logits written earlier in this launch by other blocks
-// (global memory, read through L2): their keys are staged once into `keys`
-// (E entries of shared memory) with independent loads, then each of the K
-// rounds scans shared memory.
+// (global memory, read through L2), read once with independent loads: for
+// E <= 512 the keys stay in registers, otherwise they are staged into `keys`
+// (E entries of shared memory) and each of the K rounds scans them.
 static __device__ __noinline__ void warp_topk_keys(const float* logits, int E, int K, uint64_t* keys,
                                                    int32_t* idx, float* w) {
   const int lane = threadIdx.x & 31;
-  // 16 independent loads per lane in flight: one round trip for E <= 512
-#pragma unroll 1
-  for (int e0 = 0; e0 < E; e0 += 512) {
+  if (E <= 512) {
+    // Up to 16 keys per lane stay in registers.  Every real key is nonzero
+    // (its high word is at least the order bits of -inf), so 0 means "none".
+    // Each lane holds the best of its keys not yet taken; a round takes the
+    // warp maximum (high words first, then the low words among the lanes
+    // that hold that high word) and only the lane that held it rescans.
+    // all 16 loads are issued before the first use (clamped, unconditional)
     float v[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int e = e0 + lane + 32 * i;
-      v[i] = e < E ? __ldcg(logits + e) : 0.f;
-    }
+    for (int i = 0; i < 16; ++i) v[i] = __ldcg(logits + min(lane + 32 * i, E - 1));
+    uint64_t kr[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int e = e0 + lane + 32 * i;
-      if (e < E) keys[e] = topk_key(v[i], e);
+      const int e = lane + 32 * i;
+      kr[i] = e < E ? topk_key(v[i], e) : 0ull;
     }
-  }
-  __syncwarp();
-  uint64_t prev = ~0ull;
+    uint64_t mine = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mine = kr[i] > mine ? kr[i] : mine;
 #pragma unroll 1
-  for (int k = 0; k < K; ++k) {
-    uint64_t best = 0;
+    for (int k = 0; k < K; ++k) {
+      const uint32_t hi = (uint32_t)(mine >> 32);
+      const uint32_t hmax = __reduce_max_sync(0xffffffffu, hi);
+      const uint32_t lmax = __reduce_max_sync(0xffffffffu, hi == hmax ? (uint32_t)mine : 0u);
+      const uint64_t best = ((uint64_t)hmax << 32) | lmax;
+      if (lane == 0) {
+        idx[k] = (int)~lmax;
+        w[k] = topk_key_value(best);
+      }
+      if (mine == best) {
+        uint64_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = (kr[i] < best && kr[i] > m) ? kr[i] : m;
+        mine = m;
+      }
+    }
+  } else {
+    // 16 independent loads per lane in flight per 512 logits, staged in
+    // shared memory; each of the K rounds scans them
+#pragma unroll 1
+    for (int e0 = 0; e0 < E; e0 += 512) {
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int e = e0 + lane + 32 * i;
+        v[i] = e < E ? __ldcg(logits + e) : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int e = e0 + lane + 32 * i;
+        if (e < E) keys[e] = topk_key(v[i], e);
+      }
+    }
+    __syncwarp();
+    uint64_t prev = ~0ull;
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+      uint64_t best = 0;
 #pragma unroll 4
-    for (int e = lane; e < E; e += 32) {
-      const uint64_t key = keys[e];
-      best = (key < prev && key > best) ? key : best;
+      for (int e = lane; e < E; e += 32) {
+        const uint64_t key = keys[e];
+        best = (key < prev && key > best) ? key : best;
+      }
+      best = warp_max_u64(best);
+      if (lane == 0) {
+        idx[k] = (int)~(uint32_t)best;
+        w[k] = topk_key_value(best);
+      }
+      prev = best;
     }
-    best = warp_max_u64(best);
-    if (lane == 0) {
-      idx[k] = (int)~(uint32_t)best;
-      w[k] = topk_key_value(best);
-    }
-    prev = best;
   }
   topk_weights(K, w);
 }
