@@ -267,7 +267,7 @@ def build_replica(M, s, replica, T, chunk=32):
 
 
 TRACE_NAMES = ["start", "router_done", "shared_gu_done", "expert_gu_done", "wait_S_done", "wait_E_done",
-               "tiles_done", "wait_D_done", "exit", "producer_topk", "producer_last_copy"]
+               "tiles_done", "arrived_D", "exit", "producer_topk", "producer_last_copy"]
 
 
 SPIN_NAMES = ["consumer_slot", "consumer_phase", "consumer_x", "producer_slot", "producer_routing",

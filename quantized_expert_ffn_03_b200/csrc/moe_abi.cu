@@ -96,7 +96,7 @@ moe_status device_info(DeviceInfo* out) {
 }
 
 struct WsPlan {
-  size_t logits, hs, hf, hx, ss, total;
+  size_t logits, hs, hf, hx, ss, hres, total;
 };
 
 WsPlan ws_plan(const Layout& L, int T) {
@@ -112,6 +112,8 @@ WsPlan ws_plan(const Layout& L, int T) {
   pos = round_up_256(pos + sizeof(float) * (size_t)T * L.K * (L.I / 8));
   w.ss = pos;
   pos = round_up_256(pos + sizeof(float) * (size_t)T * kMaxGrid);
+  w.hres = pos;
+  pos = round_up_256(pos + sizeof(float) * (size_t)T * L.H);
   w.total = pos;
   return w;
 }
@@ -296,6 +298,7 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
   p.hf = ws + wp.hf;
   p.hx = reinterpret_cast<float*>(ws + wp.hx);
   p.ss = reinterpret_cast<float*>(ws + wp.ss);
+  p.hres = reinterpret_cast<float*>(ws + wp.hres);
   if (trace && trace_entries < (size_t)grid * 128)
     return fail(MOE_ERR_INVALID_ARG, "trace needs %d entries", grid * 128);
   p.timeout_ns = kTimeoutNs;

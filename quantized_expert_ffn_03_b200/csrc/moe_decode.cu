@@ -97,7 +97,9 @@ struct TileDesc {
 // barriers consumers -> sync warp (evt) and sync warp -> consumers (go)
 enum { EVT_R = 0, EVT_S, EVT_E, EVT_D, NEVT };
 enum { GO_S = 0, GO_E, GO_D, NGO };
-enum { FLAG_TOPK = NGO, FLAG_SCNT };  // flags[] slots: routing valid; consumer warps past the S tiles
+// flags[] slots: routing valid; consumer warps past the S tiles; this block
+// finished last
+enum { FLAG_TOPK = NGO, FLAG_SCNT, FLAG_LAST };
 
 // ---- shared-memory plan ------------------------------------------------------
 // xf: x as mma A fragments, [token][group][t][8 words]; word 2s is the bf16
@@ -746,12 +748,6 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
               2u * H, a, b);
   }
   pr.post(F_ARRIVE_S);
-  // the shared expert's down rows of this block: they wait for every block's
-  // shared intermediate (S), which is staged while the routing is found
-  if (L.has_shared) {
-    pr.pre(F_WAIT_S);
-    emit_rows(pr, TILE_SHARED_DOWN, reinterpret_cast<const uint8_t*>(p.sd), nullptr, 2u * I, r0, r1);
-  }
   // the routing, from the sync warp
   bool routed = false;
   if (pr.ok) {
@@ -781,6 +777,13 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
     }
   }
   pr.post(F_ARRIVE_E);
+  // the shared expert's down rows of this block: every block's shared
+  // intermediate (S) was staged while the routing was found, so they run
+  // while the routed intermediate (E) is being completed
+  if (L.has_shared) {
+    pr.pre(F_WAIT_S);
+    emit_rows(pr, TILE_SHARED_DOWN, reinterpret_cast<const uint8_t*>(p.sd), nullptr, 2u * I, r0, r1);
+  }
   pr.pre(F_WAIT_E);
   if (routed && r1 > r0) {
 #pragma unroll 1
@@ -898,14 +901,6 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
       bulk_g2s(hx_s, p.hx, hxb, &go[GO_E]);
     }
     mbar_arrive(&go[GO_E]);
-    // D: sum of squares written -> arrive, wait, release the consumers
-    if (!mbar_wait(&evt[EVT_D], 0, to, sp_evt)) ok = false;
-    red_release_add(&ctr[3], 1u);
-    trace_mark<TRACE>(p, 72);
-    const bool g = ok && grid_wait_thread(&ctr[3], G, &ctr[5], p.err, to, sp_grid);
-    trace_mark<TRACE>(p, 73);
-    flags[GO_D] = g ? 1 : 0;
-    mbar_arrive(&go[GO_D]);
   }
   __syncwarp();
 }
@@ -1231,6 +1226,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         if (L.has_shared) h += ys[q];
         hacc[q] = h;
         p.h_out[(size_t)t * H + r0 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+        p.hres[(size_t)t * H + r0 + j] = h;
       }
       consumer_sync();
       if (warp < T) {
@@ -1241,41 +1237,65 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         if (lane == 0) p.ss[(size_t)c * T + warp] = s;
       }
     }
-    consumer_sync();
-    if (tid == 0) mbar_arrive(&evt[EVT_D]);
-    ok = warp_wait(&go[GO_D], 0, p.timeout_ns, spins ? spins + 1 : nullptr) && flags[GO_D] != 0 && ok && routed;
-    if (tid == 0) trace_mark<TRACE>(p, 7);
-    if (ok) {
-      if (warp < T) {
-        float s = 0.f;
-#pragma unroll 1
-        for (int b = lane; b < G; b += 32) s += __ldcg(p.ss + (size_t)b * T + warp);
-        s = warp_sum(s);
-        if (lane == 0) inv[warp] = rsqrtf(__fdividef(s, (float)H) + L.eps);
-      }
-      consumer_sync();
-#pragma unroll 1
-      for (int q = tid; q < T * nrows; q += kConsumers) {
-        const int t = q / nrows, j = q - t * nrows;
-        const float gm = __bfloat162float(__ushort_as_bfloat16(gam_s[j]));
-        p.y_norm[(size_t)t * H + r0 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(hacc[q] * inv[t] * gm));
-      }
-    }
   }
 
-  // ---- exit: the last block out resets the counters for the next launch ----
+  // ---- exit: RMSNorm needs every block's sum of squares, so the last block
+  // to finish its rows of h normalises all of them; it also resets the
+  // counters for the next launch (every other block is past its last wait) ----
   __syncthreads();
   if (tid == 0) {
-    trace_mark<TRACE>(p, 8);
     if constexpr (TRACE)
       for (int k = 0; k < 8; ++k) p.trace[(size_t)c * kTraceEntries + 80 + k] = spin_s[k];
-    __threadfence();
-    const uint32_t old = atomicAdd(&ctr[4], 1u);
-    if (old == (uint32_t)G - 1u) {
-      for (int i = 0; i < 6; ++i) atomicExch(&ctr[i], 0u);
-      __threadfence();
-    }
+    flags[FLAG_LAST] = atom_add_acq_rel_gpu(&ctr[3], 1u) == (uint32_t)G - 1u ? 1 : 0;
+    trace_mark<TRACE>(p, 7);
   }
+  __syncthreads();
+  if (flags[FLAG_LAST]) {
+    // eight columns of one token per thread and pass; the first pass's loads,
+    // the sums of squares and the error word are all in flight together
+    const float4* hr = reinterpret_cast<const float4*>(p.hres);
+    const int n8 = T * H / 8;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    uint4 gw = make_uint4(0u, 0u, 0u, 0u);
+    if (tid < n8) {
+      a = __ldcg(hr + 2 * tid);
+      b = __ldcg(hr + 2 * tid + 1);
+      gw = __ldg(reinterpret_cast<const uint4*>(p.gamma + (8 * tid) % H));
+    }
+    const bool good = flags[FLAG_TOPK] != 0 && ld_relaxed_gpu(p.err) == 0u;
+    if (warp < T) {
+      float s = 0.f;
+#pragma unroll 1
+      for (int bk = lane; bk < G; bk += 32) s += __ldcg(p.ss + (size_t)bk * T + warp);
+      s = warp_sum(s);
+      if (lane == 0) inv[warp] = rsqrtf(__fdividef(s, (float)H) + L.eps);
+    }
+    __syncthreads();
+    if (good) {
+#pragma unroll 1
+      for (int q = tid; q < n8; q += kDecodeThreads) {
+        const int t = (8 * q) / H, col = 8 * q - t * H;
+        if (q != tid) {
+          a = __ldcg(hr + 2 * q);
+          b = __ldcg(hr + 2 * q + 1);
+          gw = __ldg(reinterpret_cast<const uint4*>(p.gamma + col));
+        }
+        float gm[8];
+        unpack_bf16x8(gw, gm);
+        const float hv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        const float iv = inv[t];
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          o[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[2 * i] * iv * gm[2 * i])) |
+                 ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[2 * i + 1] * iv * gm[2 * i + 1])) << 16);
+        reinterpret_cast<uint4*>(p.y_norm)[q] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    // plain stores: the next launch reads the counters after this one ends
+    if (tid < 6) reinterpret_cast<volatile uint32_t*>(ctr)[tid] = 0u;
+  }
+  if (tid == 0) trace_mark<TRACE>(p, 8);
 }
 
 template <int FMT, bool TRACE>

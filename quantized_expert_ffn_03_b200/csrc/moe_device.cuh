@@ -67,6 +67,15 @@ __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Fetch-and-add with acquire-release semantics at GPU scope: what this
+// thread has observed is visible to whoever later observes the increment,
+// and what the earlier increments released is visible to this thread.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // Block-wide "arrive" on a grid counter: all writes of this block made before
 // the call become visible to any block that later observes the increment.
 __device__ __forceinline__ void grid_arrive(uint32_t* ctr) {

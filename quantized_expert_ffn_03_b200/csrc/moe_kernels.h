@@ -35,7 +35,8 @@ __host__ __device__ inline int decode_rows_max(int H, int G) { return 8 * ((H / 
 
 // Workspace of a layer call: counters and error word first, then fp32
 // intermediates.  ctr[0] router, [1] shared gate/up, [2] routed gate/up,
-// [3] down, [4] blocks that exited, [5] abort flag of the running launch.
+// [3] blocks that finished their rows of h, [4] unused, [5] abort flag of
+// the running launch.
 struct DecodeParams {
   Layout L;
   int T;
@@ -58,7 +59,8 @@ struct DecodeParams {
   float* hs;      // [T][I]
   uint8_t* hf;    // routed intermediate as hi/lo bf16 A fragments, 4*T*K*I bytes
   float* hx;      // [T*K][I/8] sums of hi + lo over 8-row blocks
-  float* ss;      // [grid][T]
+  float* ss;      // [grid][T] sums of squares of each block's rows of h
+  float* hres;    // [T][H] h in fp32, normalised by the last block to finish
   uint64_t timeout_ns;
   uint32_t slot_bytes;  // bytes per shared-memory ring slot
   int nslots;           // ring slots (2..4)
