@@ -52,6 +52,12 @@ def parse_args(argv=None):
     p.add_argument("--no-graph", action="store_true")
     p.add_argument("--trace", action="store_true",
                    help="also print per-phase timestamps of a few traced layer calls")
+    p.add_argument("--streaming", action="store_true",
+                   help="measure the expert-streaming tier instead (its own JSON line)")
+    p.add_argument("--stream-layers", type=int, default=4)
+    p.add_argument("--stream-slots", type=int, default=512)
+    p.add_argument("--stream-steps", type=int, default=64)
+    p.add_argument("--stream-warmup", type=int, default=32)
     return p.parse_args(argv)
 
 
@@ -475,10 +481,136 @@ def run_ours(args):
     return 0
 
 
+def run_streaming(args):
+    """The expert-streaming tier on one GPU: L layers of the workload shape,
+    every expert in one pinned host store ([layer][expert] blobs), n_slots
+    device slots.  A step is one token through the L layers; per layer: the
+    layer's router and the next layer's router on the same input (the
+    prediction), one device-to-host read of both top-K results,
+    moe_stream_resolve, moe_layer_forward_routed, and moe_stream_prefetch of
+    the predicted experts on a side stream.  The layer output (y_norm, h_out)
+    is the next layer's (x, residual)."""
+    import torch
+    import quantized_expert_ffn_03_b200 as M
+
+    torch.cuda.set_device(0)
+    s = workload(args.bits)
+    L, NS, E, K = args.stream_layers, args.stream_slots, s.n_experts, s.top_k
+    cfg = M.config(s.hidden, s.inter, E, K, bits=s.bits, eps=s.eps, has_shared=s.has_shared)
+    nb = M.moe_packed_expert_bytes(cfg)
+    store = torch.empty((L * E, nb), dtype=torch.uint8).pin_memory()
+    chunk = 32
+    buf = torch.empty((chunk, nb), dtype=torch.uint8, device="cuda")
+    for l in range(L):
+        for e0 in range(0, E, chunk):
+            wg, wu, wd = S.torch_expert_weights(s, e0, chunk, 100 + l, "cuda")
+            M.moe_pack_experts_device(cfg, wg, wu, wd, buf)
+            del wg, wu, wd
+            store[l * E + e0:l * E + e0 + chunk].copy_(buf)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+    dense = []
+    for l in range(L):
+        d = S.dense_weights(s, 100 + l)
+        dense.append(dict(wr=dev(d["wr"]), bias=torch.from_numpy(d["bias"]).cuda(), sg=dev(d["shared_gate"]),
+                          su=dev(d["shared_up"]), sd=dev(d["shared_down"]), gamma=dev(d["gamma"])))
+    table = torch.zeros(E, dtype=torch.int64, device="cuda")
+    wts = [M.layer_weights(table, None, None, d["sg"], d["su"], d["sd"], d["gamma"]) for d in dense]
+    ws = torch.zeros(M.moe_layer_workspace_bytes(cfg, 1), dtype=torch.uint8, device="cuda")
+    M.moe_workspace_init(ws)
+    idx_d = torch.empty((2, 1, K), dtype=torch.int32, device="cuda")
+    w_d = torch.empty((2, 1, K), dtype=torch.float32, device="cuda")
+    lg = torch.empty((2, 1, E), dtype=torch.float32, device="cuda")
+    idx_h = torch.empty((2, K), dtype=torch.int32).pin_memory()
+    comp = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+
+    # pinned host -> device copy peak (1 GiB, one cudaMemcpyAsync)
+    big = torch.empty(1 << 30, dtype=torch.uint8).pin_memory()
+    bigd = torch.empty(1 << 30, dtype=torch.uint8, device="cuda")
+    bigd.copy_(big, non_blocking=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        bigd.copy_(big, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    h2d_peak = 3 * (1 << 30) / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    del big, bigd
+
+    cache = M.moe_stream_create(cfg, L, store, NS)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(4321)
+    h = torch.empty((1, s.hidden), dtype=torch.int16, device="cuda")
+    y = torch.empty_like(h)
+
+    def token(i):
+        x = torch.randn((1, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
+        res = torch.randn((1, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
+        for l in range(L):
+            d = dense[l]
+            M.moe_router_topk(cfg, x, d["wr"], d["bias"], idx_d[0], w_d[0], logits_out=lg[0])
+            if l + 1 < L:
+                dn = dense[l + 1]
+                M.moe_router_topk(cfg, x, dn["wr"], dn["bias"], idx_d[1], w_d[1], logits_out=lg[1])
+            idx_h.copy_(idx_d.view(2, K), non_blocking=True)
+            comp.synchronize()
+            M.moe_stream_resolve(cache, l, idx_h[0].numpy(), table)
+            M.moe_layer_forward_routed(cfg, wts[l], x, res, idx_d[0], w_d[0], h, y, ws)
+            if l + 1 < L:
+                M.moe_stream_prefetch(cache, l + 1, idx_h[1].numpy(), copy_stream=side)
+            x, res = y.clone(), h.clone()
+
+    try:
+        for i in range(args.stream_warmup):
+            token(i)
+        torch.cuda.synchronize()
+        st0 = M.moe_stream_stats(cache)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        wall0 = time.perf_counter()
+        t0.record()
+        for i in range(args.stream_steps):
+            token(args.stream_warmup + i)
+        t1.record()
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+        ms = t0.elapsed_time(t1)
+        st1 = M.moe_stream_stats(cache)
+        err = M.moe_device_error(ws)[0]
+    finally:
+        torch.cuda.synchronize()
+        M.moe_stream_destroy(cache)
+    dst = {k: st1[k] - st0[k] for k in st1}
+    looked = dst["hits"] + dst["misses"]
+    secs = ms * 1e-3
+    line = {
+        "metric": "streaming tier: tokens/s through %d layers, experts in pinned host memory" % L,
+        "value": args.stream_steps / secs, "unit": "tokens/s", "impl": "ours", "mode": "streaming",
+        "n_gpus": 1, "steps": args.stream_steps, "warmup": args.stream_warmup,
+        "ms_per_step": ms / args.stream_steps, "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "%s_x%d_layers" % (s.name, L), "layers": L, "slots": NS,
+                   "slot_bytes": nb, "host_store_gb": L * E * nb / 1e9, "device_cache_gb": NS * nb / 1e9,
+                   "tokens_per_step": 1, "router_bias": "zipf1.1, a different permutation per layer"},
+        "hit_rate": dst["hits"] / looked if looked else None,
+        "misses_per_token": dst["misses"] / args.stream_steps,
+        "prefetches_per_token": dst["prefetches"] / args.stream_steps,
+        "prefetch_hits_per_token": dst["prefetch_hits"] / args.stream_steps,
+        "h2d_gb_per_token": dst["bytes_h2d"] / args.stream_steps / 1e9,
+        "h2d_gbs_average": dst["bytes_h2d"] / secs / 1e9,
+        "h2d_peak_gbs": h2d_peak,
+        "wall_ms_per_step": wall * 1e3 / args.stream_steps,
+        "device_error": err,
+    }
+    print(json.dumps(line), flush=True)
+    return 0 if err == 0 else 1
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.streaming:
+        return run_streaming(args)
     return run_ours(args)
 
 

@@ -24,7 +24,8 @@
  * Conventions for every call:
  *   - Pointers are owned by the caller.  Device pointers are CUDA global
  *     memory on the current device; host pointers are ordinary host memory
- *     (pinned where stated).  The library allocates no device memory.
+ *     (pinned where stated).  The library allocates no device memory,
+ *     except the slots of an expert-streaming cache (moe_stream_create).
  *   - Device calls are asynchronous on the given stream and do not
  *     synchronise unless stated.  Inputs are never modified.
  *   - Every call returns a moe_status.  On MOE_OK all outputs are fully
@@ -53,7 +54,7 @@ typedef enum {
   MOE_ERR_CUDA = 4,        /* a CUDA runtime call failed (message has the CUDA error) */
   MOE_ERR_OOM = 5,         /* a device or pinned-host allocation failed */
   MOE_ERR_TIMEOUT = 6,     /* a bounded device-side wait expired (see moe_device_error) */
-  MOE_ERR_IO = 7,          /* reserved for the expert-streaming tier (host-store copies) */
+  MOE_ERR_IO = 7,          /* the expert-streaming tier could not copy from its host store */
   MOE_ERR_DEVICE = 8       /* a device-side check failed (misaligned expert pointer, bad expert id) */
 } moe_status;
 
@@ -179,6 +180,24 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts
                              float* w_out, void* workspace, size_t ws_bytes,
                              cudaStream_t stream);
 
+/* The same layer with the routing given instead of computed: idx int32
+ * [T][K] (expert ids) and w fp32 [T][K] (their weights) in device memory,
+ * typically the outputs of moe_router_topk.  The router weights
+ * (wts->router_w, wts->router_bias) are not read and may be NULL; only
+ * wts->expert_ptr[idx[t][k]] is read from the pointer table.  This is the
+ * call of the expert-streaming tier, where the host must know the routing
+ * first to bring the chosen experts into device memory (the pages' CPU reads
+ * the GPU router's output, then reads the experts from SSD: "Flash-MoE:
+ * ラップトップでの397Bパラメータモデルの実行", section "パイプライン概要").
+ * An id outside [0, E) or a NULL / misaligned pointer for a chosen expert is
+ * reported as MOE_ERR_DEVICE by moe_device_error.  Workspace: as
+ * moe_layer_forward. */
+moe_status moe_layer_forward_routed(const moe_config* cfg, const moe_layer_weights* wts,
+                                    const void* x_bf16, const void* residual_bf16, int T,
+                                    const int32_t* idx, const float* w, void* h_out_bf16,
+                                    void* y_norm_bf16, void* workspace, size_t ws_bytes,
+                                    cudaStream_t stream);
+
 /* Allocation-free variant of moe_layer_forward.  The pages have no
  * counterpart: their engine owns all of its buffers.  It is for callers that
  * must not allocate device memory (a fixed memory budget, or a loop where
@@ -236,6 +255,75 @@ moe_status moe_layer_forward_host(const moe_config* cfg, const moe_layer_weights
                                   const void* x_bf16_host, const void* residual_bf16_host,
                                   int T, void* h_out_bf16_host, void* y_norm_bf16_host,
                                   void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Expert-streaming tier.  The pages keep all experts on SSD and read the 4
+ * chosen ones per layer and token (toolarium, section "Mixture of Experts и
+ * почему SSD достаточно"; hakusoku, section "パイプライン概要": parallel
+ * pread of the K experts, about 2.4 ms of a 4.3 ms layer), leaning on the OS
+ * page cache as the expert cache (toolarium, section "Flash-MoE: чистый C,
+ * Metal и никакого Python"; hakusoku, section "試行錯誤と最適化": their own
+ * cache measured slower than the page cache).  Here the store is pinned host
+ * memory holding every expert of n_layers layers ([layer][expert] blobs of
+ * moe_packed_expert_bytes each, contiguous), and the cache is n_slots
+ * device slots of one blob each, keyed by (layer, expert) and replaced least
+ * recently used.  Copies are cudaMemcpyAsync host -> device.
+ *
+ * Protocol per layer: moe_router_topk, read idx to the host,
+ * moe_stream_resolve (brings in the misses, waits for pending prefetches,
+ * fills the pointer table), then moe_layer_forward_routed on the same compute
+ * stream with that table.  moe_stream_prefetch, on another stream, may bring
+ * in the experts predicted for a later layer meanwhile (the streaming
+ * implementations that the blog.cecily.jp article on BigMoeOnEdge describes
+ * rely on knowing the next layer's experts before the current layer ends;
+ * the pages' Mac engine measured its prefetch and speculative variants as
+ * losses there: hakusoku, section "試行錯誤と最適化").  The slots that a
+ * resolve call hands out stay resident until
+ * the next resolve call on the cache, which records on its compute stream
+ * that they may be reused: enqueue the layer that reads them on that stream
+ * before the next resolve.  A cache is used by one host thread at a time
+ * (calls lock it). */
+typedef struct moe_stream_cache moe_stream_cache;
+
+/* Creates a cache: allocates n_slots * moe_packed_expert_bytes of device
+ * memory (the one call of the library that allocates device memory) and two
+ * CUDA events per slot.  host_pinned_experts must be page-locked
+ * (cudaHostAlloc / cudaHostRegister) and stay valid until destroy.
+ * MOE_ERR_OOM if the slots do not fit; MOE_ERR_INVALID_ARG for a pageable
+ * store, n_layers < 1 or n_slots < 1. */
+moe_status moe_stream_create(const moe_config* cfg, int n_layers, const void* host_pinned_experts,
+                             int n_slots, moe_stream_cache** out);
+
+/* Enqueues on copy_stream the copies of those of expert_ids_host[0..n)
+ * (experts of `layer`) that are not resident, each into the least recently
+ * used slot that no resolve call holds; the copy waits for the last kernel
+ * that read the slot.  A hint: ids that find no free slot are skipped
+ * (counted in prefetch_dropped).  Does not synchronise.  MOE_ERR_IO if a
+ * copy cannot be enqueued. */
+moe_status moe_stream_prefetch(moe_stream_cache* cache, int layer, const int32_t* expert_ids_host,
+                               int n, cudaStream_t copy_stream);
+
+/* Makes the distinct experts of idx_host[0..n) (experts of `layer`)
+ * resident: misses are copied on compute_stream, and compute_stream waits
+ * for prefetch copies still in flight.  Then writes expert_ptr_dev (device
+ * array [E] of device pointers) on compute_stream: the slot of every
+ * resolved expert; other entries are unspecified.  MOE_ERR_OOM if the
+ * distinct ids outnumber the slots.  Does not synchronise. */
+moe_status moe_stream_resolve(moe_stream_cache* cache, int layer, const int32_t* idx_host, int n,
+                              const void** expert_ptr_dev, cudaStream_t compute_stream);
+
+/* Counters since create: resolved experts found resident (hits) or copied
+ * on demand (misses), prefetch copies issued, resolved experts that a
+ * prefetch had brought in and no resolve had used yet (prefetch_hits),
+ * prefetch ids skipped for want of a free slot, and bytes copied. */
+typedef struct {
+  uint64_t hits, misses, prefetches, prefetch_hits, prefetch_dropped, bytes_h2d;
+} moe_stream_counters;
+moe_status moe_stream_stats(const moe_stream_cache* cache, moe_stream_counters* out);
+
+/* Waits for the cache's copies and kernels that may still use its slots
+ * (synchronises the device), then frees the slots and events. */
+void moe_stream_destroy(moe_stream_cache* cache);
 
 /* Read (synchronising the stream) and clear the device-side error word of a
  * layer workspace.  Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE;

@@ -27,6 +27,7 @@ NOALLOC_SCRATCH_BYTES = 4 << 20  # MOE_NOALLOC_SCRATCH_BYTES of moe.h
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_OOM", 6: "MOE_ERR_TIMEOUT", 7: "MOE_ERR_IO",
           8: "MOE_ERR_DEVICE"}
+STATUS_BY_NAME = {v: k for k, v in STATUS.items()}
 
 
 class MoeError(RuntimeError):
@@ -74,6 +75,14 @@ EXPORTS = {
                                            C.c_size_t, C.c_void_p]),
     "moe_layer_forward_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                             C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "moe_layer_forward_routed": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                           C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                           C.c_size_t, C.c_void_p]),
+    "moe_stream_create": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p]),
+    "moe_stream_prefetch": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p]),
+    "moe_stream_resolve": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
+    "moe_stream_stats": (C.c_int, [C.c_void_p, C.c_void_p]),
+    "moe_stream_destroy": (None, [C.c_void_p]),
     "moe_device_error": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
     "moe_selftest_bounded_wait": (C.c_int, [C.c_void_p, C.c_size_t, C.c_uint64, C.c_void_p]),
 }
@@ -206,6 +215,14 @@ def moe_layer_forward(cfg, wts, x, residual, h_out, y_norm, idx_out=None, w_out=
                                   workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def moe_layer_forward_routed(cfg, wts, x, residual, idx, w, h_out, y_norm, workspace, stream=None):
+    """The layer with the routing given: idx int32 [T][K], w float32 [T][K] (CUDA)."""
+    T = x.shape[0]
+    _check(_lib.moe_layer_forward_routed(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T, _ptr(idx),
+                                         _ptr(w), _ptr(h_out), _ptr(y_norm), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def moe_layer_forward_noalloc(cfg, wts, x, residual, h_out, y_norm, idx_out=None, w_out=None, stream=None):
     """moe_layer_forward on the library's built-in scratch (no workspace)."""
     T = x.shape[0]
@@ -232,6 +249,47 @@ def moe_layer_forward_host(cfg, wts, x, residual, h_out, y_norm, workspace, stre
     _check(_lib.moe_layer_forward_host(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T,
                                        _ptr(h_out), _ptr(y_norm), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+# ---- expert-streaming tier -------------------------------------------------------
+
+class MoeStreamCounters(C.Structure):
+    _fields_ = [("hits", C.c_uint64), ("misses", C.c_uint64), ("prefetches", C.c_uint64),
+                ("prefetch_hits", C.c_uint64), ("prefetch_dropped", C.c_uint64), ("bytes_h2d", C.c_uint64)]
+
+
+def moe_stream_create(cfg, n_layers, host_store, n_slots):
+    """host_store: pinned host tensor (or address) of n_layers*E packed blobs.
+    Returns the cache handle (an int)."""
+    h = C.c_void_p(0)
+    _check(_lib.moe_stream_create(C.byref(cfg), int(n_layers), _ptr(host_store), int(n_slots), C.byref(h)))
+    return h.value
+
+
+def _ids(ids):
+    a = np.ascontiguousarray(np.asarray(ids, dtype=np.int32).reshape(-1))
+    return a, a.size
+
+
+def moe_stream_prefetch(cache, layer, expert_ids, copy_stream=None):
+    a, n = _ids(expert_ids)
+    _check(_lib.moe_stream_prefetch(cache, int(layer), a.ctypes.data, n, _stream(copy_stream)))
+
+
+def moe_stream_resolve(cache, layer, idx, expert_ptr, stream=None):
+    """idx: host ids (numpy / list); expert_ptr: int64 CUDA tensor [E] (written)."""
+    a, n = _ids(idx)
+    _check(_lib.moe_stream_resolve(cache, int(layer), a.ctypes.data, n, _ptr(expert_ptr), _stream(stream)))
+
+
+def moe_stream_stats(cache):
+    out = MoeStreamCounters()
+    _check(_lib.moe_stream_stats(cache, C.byref(out)))
+    return {f: int(getattr(out, f)) for f, _ in MoeStreamCounters._fields_}
+
+
+def moe_stream_destroy(cache):
+    _lib.moe_stream_destroy(cache)
 
 
 def moe_device_error(workspace, stream=None):

@@ -14,8 +14,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe.so")
-SOURCES = ["moe_abi.cu", "moe_decode.cu", "moe_router.cu", "moe_pack.cu", "moe_noalloc.cu"]
-HEADERS = ["moe_device.cuh", "moe_kernels.h", "moe_layout.h"]
+SOURCES = ["moe_abi.cu", "moe_decode.cu", "moe_router.cu", "moe_pack.cu", "moe_noalloc.cu", "moe_stream.cu"]
+HEADERS = ["moe_device.cuh", "moe_kernels.h", "moe_layout.h", "moe_stream_policy.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

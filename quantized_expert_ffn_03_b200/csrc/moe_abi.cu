@@ -239,7 +239,8 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
                                      const void* x_bf16, const void* residual_bf16, int T,
                                      void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
                                      float* w_out, void* workspace, size_t ws_bytes,
-                                     void* trace, size_t trace_entries, cudaStream_t stream) {
+                                     void* trace, size_t trace_entries, cudaStream_t stream,
+                                     const int32_t* idx_in = nullptr, const float* w_in = nullptr) {
   Layout L;
   moe_status s = check_cfg(cfg, &L);
   if (s != MOE_OK) return s;
@@ -249,12 +250,15 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
     return fail(MOE_ERR_UNSUPPORTED, "T=%d: the fused decode path takes at most %d tokens", T,
                 kMaxTokensFused);
   if (T * L.K > 64) return fail(MOE_ERR_UNSUPPORTED, "T*top_k must be <= 64");
-  if (!wts || !wts->expert_ptr || !wts->router_w || !wts->gamma || !x_bf16 || !residual_bf16 ||
+  const bool given = idx_in != nullptr;  // routing given: the router weights are not read
+  if (given && !w_in) return fail(MOE_ERR_INVALID_ARG, "NULL routing weights");
+  if (!wts || !wts->expert_ptr || (!given && !wts->router_w) || !wts->gamma || !x_bf16 || !residual_bf16 ||
       !h_out_bf16 || !y_norm_bf16)
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
   if (L.has_shared && (!wts->shared_gate || !wts->shared_up || !wts->shared_down))
     return fail(MOE_ERR_INVALID_ARG, "has_shared=1 but a shared-expert pointer is NULL");
-  const void* a16[] = {x_bf16, residual_bf16, h_out_bf16, y_norm_bf16, wts->router_w, wts->gamma};
+  const void* a16[] = {x_bf16, residual_bf16, h_out_bf16, y_norm_bf16, given ? nullptr : wts->router_w,
+                       wts->gamma};
   for (const void* p : a16)
     if (!aligned(p, 16)) return fail(MOE_ERR_INVALID_ARG, "bf16 arrays must be 16-byte aligned");
   if (L.has_shared && (!aligned(wts->shared_gate, 16) || !aligned(wts->shared_up, 16) ||
@@ -291,6 +295,8 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
   p.y_norm = static_cast<uint16_t*>(y_norm_bf16);
   p.idx_out = idx_out;
   p.w_out = w_out;
+  p.idx_in = idx_in;
+  p.w_in = w_in;
   p.ctr = reinterpret_cast<uint32_t*>(ws);
   p.err = reinterpret_cast<uint32_t*>(ws + 64);
   p.logits = reinterpret_cast<float*>(ws + wp.logits);
@@ -323,6 +329,16 @@ moe_status layer_forward_on(const moe_config* cfg, const moe_layer_weights* wts,
 }  // namespace moe
 
 extern "C" {
+
+moe_status moe_layer_forward_routed(const moe_config* cfg, const moe_layer_weights* wts,
+                                    const void* x_bf16, const void* residual_bf16, int T,
+                                    const int32_t* idx, const float* w, void* h_out_bf16,
+                                    void* y_norm_bf16, void* workspace, size_t ws_bytes,
+                                    cudaStream_t stream) {
+  if (T > 0 && (!idx || !w)) return fail(MOE_ERR_INVALID_ARG, "NULL routing");
+  return layer_forward_impl(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, nullptr, nullptr,
+                            workspace, ws_bytes, nullptr, 0, stream, idx, w);
+}
 
 moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts,
                              const void* x_bf16, const void* residual_bf16, int T,

@@ -739,8 +739,10 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
   }
   mbar_arrive(xbar);
   int a, b;
-  range_of(E, c, G, a, b);
-  emit_rows(pr, TILE_ROUTER, reinterpret_cast<const uint8_t*>(p.wr), nullptr, 2u * H, a, b);
+  if (!p.idx_in) {  // with the routing given there are no router rows
+    range_of(E, c, G, a, b);
+    emit_rows(pr, TILE_ROUTER, reinterpret_cast<const uint8_t*>(p.wr), nullptr, 2u * H, a, b);
+  }
   pr.post(F_ARRIVE_R);
   if (L.has_shared) {
     range_of(I, c, G, a, b);
@@ -845,20 +847,34 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
     mbar_arrive(xfbar);
     trace_mark<TRACE>(p, 64);
   }
-  // R: arrive once every consumer warp has passed the router tiles.  The
-  // waits up to the top-K are warp-uniform so the top-K runs unsplit.
-  ok = warp_wait(&evt[EVT_R], 0, to, sp_evt) && ok;
-  if (lane == 0) red_release_add(&ctr[0], 1u);
-  __syncwarp();
-  // top-K once every block's router logits are written
-  bool gr = ok && grid_wait_thread(&ctr[0], G, &ctr[5], p.err, to, lane == 0 ? sp_grid : nullptr);
-  int good = __all_sync(0xffffffffu, gr) ? 1 : 0;
-  if (lane == 0) trace_mark<TRACE>(p, 65);
-  if (good) {
+  int good;
+  if (p.idx_in) {
+    // the routing is given: no router barrier, no top-K
 #pragma unroll 1
-    for (int t = 0; t < T; ++t) warp_topk_keys(p.logits + (size_t)t * E, E, K, tkbuf, tk_i + t * K, tk_w + t * K);
+    for (int j = lane; j < T * K; j += 32) {
+      tk_i[j] = __ldg(p.idx_in + j);
+      tk_w[j] = __ldg(p.w_in + j);
+    }
     __syncwarp();
-    if (lane == 0) trace_mark<TRACE>(p, 66);
+    good = __all_sync(0xffffffffu, ok) ? 1 : 0;
+  } else {
+    // R: arrive once every consumer warp has passed the router tiles.  The
+    // waits up to the top-K are warp-uniform so the top-K runs unsplit.
+    ok = warp_wait(&evt[EVT_R], 0, to, sp_evt) && ok;
+    if (lane == 0) red_release_add(&ctr[0], 1u);
+    __syncwarp();
+    // top-K once every block's router logits are written
+    bool gr = ok && grid_wait_thread(&ctr[0], G, &ctr[5], p.err, to, lane == 0 ? sp_grid : nullptr);
+    good = __all_sync(0xffffffffu, gr) ? 1 : 0;
+    if (lane == 0) trace_mark<TRACE>(p, 65);
+    if (good) {
+#pragma unroll 1
+      for (int t = 0; t < T; ++t) warp_topk_keys(p.logits + (size_t)t * E, E, K, tkbuf, tk_i + t * K, tk_w + t * K);
+      __syncwarp();
+      if (lane == 0) trace_mark<TRACE>(p, 66);
+    }
+  }
+  if (good) {
 #pragma unroll 1
     for (int j = lane; j < T * K; j += 32) {
       const int e = tk_i[j];

@@ -53,6 +53,8 @@ struct DecodeParams {
   uint16_t* y_norm;
   int32_t* idx_out;
   float* w_out;
+  const int32_t* idx_in;  // routing given ([T][K] expert ids and weights), or null: the kernel routes
+  const float* w_in;
   uint32_t* ctr;
   uint32_t* err;
   float* logits;  // [T][E]
