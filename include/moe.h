@@ -226,14 +226,16 @@ moe_status moe_layer_forward_noalloc(const moe_config* cfg, const moe_layer_weig
  * of the fused kernel writes global-timer stamps in ns to trace[block*128 + k]
  * (device memory, moe_layer_trace_blocks()*128 entries):
  * k = 0 start, 1 router rows done, 2 shared gate/up done, 3 routed gate/up
- * done, 4 shared wait done, 5 routed wait done, 6 last tile done, 7 norm wait
- * done, 8 exit, 9 producer has the routing, 10 producer issued its last copy,
+ * done, 4 shared wait done, 5 routed wait done, 6 last tile done, 7 arrived
+ * on the final counter, 8 exit (for the last block to arrive: after it
+ * normalised every row), 9 producer has the routing, 10 producer issued its last copy,
  * 11/12 first routed gate/up unit start/end, 13/14 first routed down unit
  * start/end; 16+2n / 17+2n: shared-memory tile n (n < 16) ready / released
  * by the consumers; 48+n: producer publishes tile n; sync warp: 64 x
- * prepared, 65 router barrier passed, 66 logits staged, 67 routing handed
- * over, 68/69 shared / routed gate/up arrivals, 70/71 shared / routed barrier
- * passed, 72 sum-of-squares arrival, 73 norm barrier passed.  Entries 80+k
+ * prepared, 65 router barrier passed, 66 top-K done, 67 routing handed
+ * over, 69 routed gate/up arrival, 71 routed barrier passed; 68 / 70 shared
+ * gate/up arrival / barrier passed (written by the consumer warp that
+ * handles that barrier).  Entries 80+k
  * (k < 8) hold poll counts (not times) of the block's waits: 0 consumers on
  * ring slots, 1 consumers on phase barriers, 2 consumers on x, 3 producer on
  * free slots, 4 producer on the routing, 5 sync warp on consumer arrivals,
