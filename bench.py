@@ -58,6 +58,8 @@ def parse_args(argv=None):
     p.add_argument("--stream-slots", type=int, default=512)
     p.add_argument("--stream-steps", type=int, default=64)
     p.add_argument("--stream-warmup", type=int, default=32)
+    p.add_argument("--batched", default="",
+                   help="comma-separated token counts: measure batches of T tokens per step instead")
     return p.parse_args(argv)
 
 
@@ -605,12 +607,59 @@ def run_streaming(args):
     return 0 if err == 0 else 1
 
 
+def run_batched(args):
+    """Batches of T tokens per step (one JSON line per T): moe_layer_forward
+    runs the fused kernel on successive chunks of up to 8 tokens, so each
+    chunk reads the experts its tokens chose.  8 replicas round-robin as in
+    the decode measurement; Zipf router bias."""
+    import torch
+    import quantized_expert_ffn_03_b200 as M
+
+    torch.cuda.set_device(0)
+    s = workload(args.bits)
+    R = max(1, args.replicas)
+    reps = [build_replica(M, s, rr, 1) for rr in range(R)]
+    cfg = reps[0]["cfg"]
+    ws = torch.zeros(M.moe_layer_workspace_bytes(cfg, 2048), dtype=torch.uint8, device="cuda")
+    M.moe_workspace_init(ws)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(99)
+    rc = 0
+    for T in [int(v) for v in args.batched.split(",") if v]:
+        x = torch.randn((T, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
+        r = torch.randn((T, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
+        h, y = torch.empty_like(x), torch.empty_like(x)
+        steps = max(3, min(50, 4096 // T))
+        for i in range(3):
+            M.moe_layer_forward(cfg, reps[i % R]["wts"], x, r, h, y, workspace=ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            M.moe_layer_forward(cfg, reps[i % R]["wts"], x, r, h, y, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        err = M.moe_device_error(ws)[0]
+        rc = rc or (1 if err else 0)
+        line = {"metric": "batched MoE-layer tokens/s (T tokens per step, fused kernel on chunks of 8)",
+                "value": T / (ms * 1e-3), "unit": "tokens/s", "impl": "ours", "mode": "batched", "n_gpus": 1,
+                "steps": steps, "warmup": 3, "ms_per_step": ms, "higher_is_better": True, "dtype": "f32",
+                "data": "synthetic", "config": {"workload": "%s_T%d" % (s.name, T), "tokens_per_step": T,
+                                                "replicas": R, "router_bias": "zipf1.1"},
+                "launches_per_step": -(-T // 8), "device_error": err}
+        print(json.dumps(line), flush=True)
+    return rc
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
     if args.streaming:
         return run_streaming(args)
+    if args.batched:
+        return run_batched(args)
     return run_ours(args)
 
 

@@ -172,13 +172,25 @@ moe_status moe_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t str
  * x_bf16, residual_bf16 [T][H]; h_out_bf16, y_norm_bf16 [T][H] (y_norm is
  * computed from the fp32 sum, before h_out is rounded to bf16); idx_out
  * int32 [T][K] and w_out fp32 [T][K] may be NULL.  T == 0 is a no-op.
- * T <= 8 runs the fused single-launch decode kernel.  A bounded device wait
- * that expires leaves MOE_ERR_TIMEOUT in the workspace (moe_device_error). */
+ * One launch of the fused kernel takes C = moe_layer_tokens_per_launch(cfg)
+ * tokens; a larger T runs as successive launches of C tokens on the stream
+ * (each token's result depends on that token only, so this is exact; each
+ * launch reads the experts its tokens chose).  The workspace of any T is
+ * that of min(T, 8) tokens.
+ * A bounded device wait that expires leaves MOE_ERR_TIMEOUT in the
+ * workspace (moe_device_error). */
 moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts,
                              const void* x_bf16, const void* residual_bf16, int T,
                              void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
                              float* w_out, void* workspace, size_t ws_bytes,
                              cudaStream_t stream);
+
+/* Tokens one launch of the fused kernel takes for this shape on the current
+ * device: the largest T <= min(8, 64 / K) whose shared-memory plan fits
+ * (4 at hidden 4096, inter 1024, K = 4).  moe_layer_forward runs longer
+ * batches in chunks of this size.  0 for an unsupported shape or when no
+ * device is usable. */
+int moe_layer_tokens_per_launch(const moe_config* cfg);
 
 /* The same layer with the routing given instead of computed: idx int32
  * [T][K] (expert ids) and w fp32 [T][K] (their weights) in device memory,

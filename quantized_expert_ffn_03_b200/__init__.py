@@ -75,6 +75,7 @@ EXPORTS = {
                                            C.c_size_t, C.c_void_p]),
     "moe_layer_forward_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                             C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "moe_layer_tokens_per_launch": (C.c_int, [C.c_void_p]),
     "moe_layer_forward_routed": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                            C.c_size_t, C.c_void_p]),
@@ -213,6 +214,10 @@ def moe_layer_forward(cfg, wts, x, residual, h_out, y_norm, idx_out=None, w_out=
     _check(_lib.moe_layer_forward(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T, _ptr(h_out),
                                   _ptr(y_norm), _ptr(idx_out), _ptr(w_out), _ptr(workspace),
                                   workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_layer_tokens_per_launch(cfg):
+    return _lib.moe_layer_tokens_per_launch(C.byref(cfg))
 
 
 def moe_layer_forward_routed(cfg, wts, x, residual, idx, w, h_out, y_norm, workspace, stream=None):

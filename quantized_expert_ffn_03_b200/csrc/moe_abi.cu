@@ -99,6 +99,23 @@ struct WsPlan {
   size_t logits, hs, hf, hx, ss, hres, total;
 };
 
+// Tokens per launch of the fused kernel: at most kMaxTokensFused, and at
+// most 64 (token, expert) pairs.  Larger T runs in chunks of this size.
+int chunk_tokens(const Layout& L) {
+  const int c = 64 / L.K;
+  return c < kMaxTokensFused ? (c > 0 ? c : 1) : kMaxTokensFused;
+}
+
+// Tokens one launch takes on a grid of `grid` blocks: the largest
+// T <= max_tokens whose shared-memory plan fits (0 if not even one token).
+int tokens_per_launch(const Layout& L, int grid, int max_tokens) {
+  for (int t = max_tokens; t >= 1; --t) {
+    int ns = 0;
+    if (decode_slot_bytes(L, t, decode_rows_max(L.H, grid), &ns) > 0) return t;
+  }
+  return 0;
+}
+
 WsPlan ws_plan(const Layout& L, int T) {
   WsPlan w;
   size_t pos = 256;
@@ -224,7 +241,7 @@ size_t moe_layer_workspace_bytes(const moe_config* cfg, int T) {
   if (!make_layout(cfg->hidden, cfg->inter, cfg->n_experts, cfg->top_k, cfg->bits, cfg->group,
                    cfg->has_shared, cfg->eps, &L))
     return 0;
-  return ws_plan(L, T).total;
+  return ws_plan(L, T < chunk_tokens(L) ? T : chunk_tokens(L)).total;
 }
 
 moe_status moe_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t stream) {
@@ -235,21 +252,16 @@ moe_status moe_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t str
 
 }  // extern "C"
 
-static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weights* wts,
-                                     const void* x_bf16, const void* residual_bf16, int T,
-                                     void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
-                                     float* w_out, void* workspace, size_t ws_bytes,
-                                     void* trace, size_t trace_entries, cudaStream_t stream,
-                                     const int32_t* idx_in = nullptr, const float* w_in = nullptr) {
+static moe_status layer_forward_chunk(const moe_config* cfg, const moe_layer_weights* wts,
+                                      const void* x_bf16, const void* residual_bf16, int T,
+                                      void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
+                                      float* w_out, void* workspace, size_t ws_bytes,
+                                      void* trace, size_t trace_entries, cudaStream_t stream,
+                                      const int32_t* idx_in, const float* w_in) {
   Layout L;
   moe_status s = check_cfg(cfg, &L);
   if (s != MOE_OK) return s;
-  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
-  if (T == 0) return ok();
-  if (T > kMaxTokensFused)
-    return fail(MOE_ERR_UNSUPPORTED, "T=%d: the fused decode path takes at most %d tokens", T,
-                kMaxTokensFused);
-  if (T * L.K > 64) return fail(MOE_ERR_UNSUPPORTED, "T*top_k must be <= 64");
+  if (T > chunk_tokens(L)) return fail(MOE_ERR_UNSUPPORTED, "T=%d: at most %d tokens per launch", T, chunk_tokens(L));
   const bool given = idx_in != nullptr;  // routing given: the router weights are not read
   if (given && !w_in) return fail(MOE_ERR_INVALID_ARG, "NULL routing weights");
   if (!wts || !wts->expert_ptr || (!given && !wts->router_w) || !wts->gamma || !x_bf16 || !residual_bf16 ||
@@ -315,6 +327,52 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
   return ok();
 }
 
+// Any T: the fused kernel on successive chunks of as many tokens as one
+// launch takes on this device (tokens_per_launch), one after another
+// on the stream (each token's result depends on that
+// token only; each chunk reads the experts its tokens chose).
+static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weights* wts,
+                                     const void* x_bf16, const void* residual_bf16, int T,
+                                     void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
+                                     float* w_out, void* workspace, size_t ws_bytes,
+                                     void* trace, size_t trace_entries, cudaStream_t stream,
+                                     const int32_t* idx_in = nullptr, const float* w_in = nullptr) {
+  Layout L;
+  moe_status s = check_cfg(cfg, &L);
+  if (s != MOE_OK) return s;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+  if (T == 0) return ok();
+  // argument checks before any device query
+  if (trace && T > chunk_tokens(L))
+    return fail(MOE_ERR_UNSUPPORTED, "a traced call takes at most %d tokens", chunk_tokens(L));
+  const bool given = idx_in != nullptr;
+  if (given && !w_in) return fail(MOE_ERR_INVALID_ARG, "NULL routing weights");
+  if (!wts || !wts->expert_ptr || (!given && !wts->router_w) || !wts->gamma || !x_bf16 || !residual_bf16 ||
+      !h_out_bf16 || !y_norm_bf16)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  DeviceInfo di;
+  if ((s = device_info(&di)) != MOE_OK) return s;
+  const int C = tokens_per_launch(L, di.sms < kMaxGrid ? di.sms : kMaxGrid, chunk_tokens(L));
+  if (C == 0)
+    return fail(MOE_ERR_UNSUPPORTED, "shape does not fit the fused kernel's shared memory (H=%d, I=%d)", L.H, L.I);
+  if (T <= C)
+    return layer_forward_chunk(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out,
+                               workspace, ws_bytes, trace, trace_entries, stream, idx_in, w_in);
+  if (trace) return fail(MOE_ERR_UNSUPPORTED, "a traced call takes at most %d tokens", C);
+  const size_t row = 2ull * (size_t)L.H;
+  for (int t0 = 0; t0 < T; t0 += C) {
+    const int n = T - t0 < C ? T - t0 : C;
+    const size_t o = (size_t)t0 * row, ok_ = (size_t)t0 * L.K;
+    s = layer_forward_chunk(cfg, wts, static_cast<const uint8_t*>(x_bf16) + o,
+                            static_cast<const uint8_t*>(residual_bf16) + o, n, static_cast<uint8_t*>(h_out_bf16) + o,
+                            static_cast<uint8_t*>(y_norm_bf16) + o, idx_out ? idx_out + ok_ : nullptr,
+                            w_out ? w_out + ok_ : nullptr, workspace, ws_bytes, nullptr, 0, stream,
+                            idx_in ? idx_in + ok_ : nullptr, w_in ? w_in + ok_ : nullptr);
+    if (s != MOE_OK) return s;
+  }
+  return ok();
+}
+
 namespace moe {
 // For the library's other translation units: record an error message, and
 // run the fused layer on a given workspace.
@@ -329,6 +387,17 @@ moe_status layer_forward_on(const moe_config* cfg, const moe_layer_weights* wts,
 }  // namespace moe
 
 extern "C" {
+
+int moe_layer_tokens_per_launch(const moe_config* cfg) {
+  Layout L;
+  if (!cfg || cfg->n_experts <= 0 || cfg->top_k <= 0 || cfg->top_k > cfg->n_experts ||
+      !make_layout(cfg->hidden, cfg->inter, cfg->n_experts, cfg->top_k, cfg->bits, cfg->group, cfg->has_shared,
+                   cfg->eps, &L))
+    return 0;
+  DeviceInfo di;
+  if (device_info(&di) != MOE_OK) return 0;
+  return tokens_per_launch(L, di.sms < kMaxGrid ? di.sms : kMaxGrid, chunk_tokens(L));
+}
 
 moe_status moe_layer_forward_routed(const moe_config* cfg, const moe_layer_weights* wts,
                                     const void* x_bf16, const void* residual_bf16, int T,

@@ -100,10 +100,17 @@ def test_argument_checks_without_gpu():
     assert st == 2 and "bits" in M.last_error()
     st = lib.moe_pack_experts(C.byref(good), None, None, None, 0, 1, None, 0)
     assert st == 1
-    # more tokens than the fused decode path takes
+    # more tokens than one launch takes run in chunks; the argument checks
+    # still come first (a NULL expert table is refused before any device work)
     wts = M.MoeLayerWeights()
     st = lib.moe_layer_forward(C.byref(good), C.byref(wts), 16, 16, 9, 16, 16, None, None, 256, 1 << 20, None)
-    assert st == 2 and "T=9" in M.last_error()
+    assert st == 1 and "NULL" in M.last_error()
+    # a traced call is one launch: at most one chunk of tokens
+    st = lib.moe_layer_forward_traced(C.byref(good), C.byref(wts), 16, 16, 9, 16, 16, 256, 1 << 20, 16, 1 << 20,
+                                      None)
+    assert st == 2 and "at most" in M.last_error()
+    # the workspace of a long batch is one chunk's
+    assert lib.moe_layer_workspace_bytes(C.byref(good), 2048) == lib.moe_layer_workspace_bytes(C.byref(good), 8)
     # T == 0 is a no-op that touches nothing
     st = lib.moe_layer_forward(C.byref(good), None, None, None, 0, None, None, None, None, None, 0, None)
     assert st == 0
