@@ -312,7 +312,12 @@ def print_trace(M, reps, cfg, xs, rs, h_out, y_out, stream, P, R, calls=16):
     probe = [round((b0[k] - b0[0]) / 1e3, 3) for k in range(11, 15)]
     print("trace_block0 first routed units (gate/up start, end, down start, end): %s" % probe,
           file=sys.stderr, flush=True)
-    sync = {k: round(float(np.median(rel[:, :, k])) / 1e3, 3) for k in list(range(64, 74)) + list(range(100, 104))}
+    # marks a launch did not write hold stale values (negative or absurd times): skipped
+    sync = {}
+    for k in list(range(64, 74)) + list(range(100, 104)):
+        v = float(np.median(rel[:, :, k])) / 1e3
+        if 0.0 <= v < 1e5:
+            sync[k] = round(v, 3)
     units = [(round((b0[104 + 2 * n] - b0[0]) / 1e3, 2), round((b0[105 + 2 * n] - b0[104 + 2 * n]) / 1e3, 2))
              for n in range(8) if b0[104 + 2 * n] > 0]
     print("trace_block0 warp0 routed units (start, duration): %s" % units, file=sys.stderr, flush=True)
