@@ -614,8 +614,8 @@ def run_streaming(args):
 
 def run_batched(args):
     """Batches of T tokens per step (one JSON line per T): moe_layer_forward
-    runs the fused kernel on successive chunks of up to 8 tokens, so each
-    chunk reads the experts its tokens chose.  8 replicas round-robin as in
+    runs the fused kernel on successive chunks of moe_layer_tokens_per_launch
+    tokens, so each chunk reads the experts its tokens chose.  8 replicas round-robin as in
     the decode measurement; Zipf router bias."""
     import torch
     import quantized_expert_ffn_03_b200 as M
@@ -647,12 +647,12 @@ def run_batched(args):
         ms = e0.elapsed_time(e1) / steps
         err = M.moe_device_error(ws)[0]
         rc = rc or (1 if err else 0)
-        line = {"metric": "batched MoE-layer tokens/s (T tokens per step, fused kernel on chunks of 8)",
+        line = {"metric": "batched MoE-layer tokens/s (T tokens per step, fused kernel on chunks)",
                 "value": T / (ms * 1e-3), "unit": "tokens/s", "impl": "ours", "mode": "batched", "n_gpus": 1,
                 "steps": steps, "warmup": 3, "ms_per_step": ms, "higher_is_better": True, "dtype": "f32",
                 "data": "synthetic", "config": {"workload": "%s_T%d" % (s.name, T), "tokens_per_step": T,
                                                 "replicas": R, "router_bias": "zipf1.1"},
-                "launches_per_step": -(-T // 8), "device_error": err}
+                "launches_per_step": -(-T // max(1, M.moe_layer_tokens_per_launch(cfg))), "device_error": err}
         print(json.dumps(line), flush=True)
     return rc
 
