@@ -314,8 +314,9 @@ static void router_logits(const orc_cfg* c, const uint16_t* x, const uint16_t* w
     for (int e = 0; e < E; ++e) {
       double acc = 0.0;
       for (int h = 0; h < H; ++h)
-        acc += orc_bf16_to_f64(x[(size_t)t * H + h]) * orc_bf16_to_f64(wr[(size_t)e * H + h]);
-      if (bias) acc += (double)bias[e];
+        acc += orc_bf16_to_f64(x[(size_t)t * H + h]) *
+               orc_bf16_to_f64(wr[ORC_MUTANT == 10 ? (size_t)h * E + e : (size_t)e * H + h]);
+      if (bias && ORC_MUTANT != 11) acc += (double)bias[e];
       logits[(size_t)t * E + e] = (float)acc;
     }
 }
@@ -333,7 +334,10 @@ void orc_router(const orc_cfg* c, const uint16_t* x_bf16, const uint16_t* wr_bf1
 
 /* silu(z) = z / (1 + exp(-z)), the SwiGLU gate ([hakusoku] "主要技術": SwiGLU
  * activation among the hand-written kernels). */
-static double silu(double z) { return z / (1.0 + exp(ORC_MUTANT == 3 ? z : -z)); }
+static double silu(double z) {
+  if (ORC_MUTANT == 12) return 1.0 / (1.0 + exp(-z));
+  return z / (1.0 + exp(ORC_MUTANT == 3 ? z : -z));
+}
 
 /* a[i] = silu(sum_h Wg[i][h] x[h]) * (sum_h Wu[i][h] x[h]) */
 void orc_expert_act(const orc_cfg* c, const uint8_t* blob, const double* x, double* a) {

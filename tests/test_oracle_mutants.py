@@ -15,13 +15,16 @@ import test_oracle_pins as P
 MUTANTS = {
     1: ("dequant drops the bias", [P.test_hand_packed_dequant]),
     2: ("codes read in reversed order", [P.test_hand_packed_dequant]),
-    3: ("silu sign flipped", [P.test_expert_ffn_matches_numpy]),
+    3: ("silu sign flipped", [P.test_expert_ffn_matches_numpy, P.test_expert_ffn_hand_worked]),
     4: ("ties go to the higher index", [P.test_topk_bruteforce_with_ties]),
     5: ("residual dropped", [P.test_one_hot_routing_is_single_expert]),
     6: ("eps added outside the square root", [P.test_rmsnorm_closed_form]),
     7: ("scale divides by 2^b instead of 2^b - 1", [P.test_quantizer_picks_nearest_code]),
-    8: ("shared down projection transposed", [P.test_shared_ffn_matches_numpy]),
-    9: ("gate and up swapped in SwiGLU", [P.test_expert_ffn_matches_numpy]),
+    8: ("shared down projection transposed", [P.test_shared_ffn_matches_numpy, P.test_shared_ffn_hand_worked]),
+    9: ("gate and up swapped in SwiGLU", [P.test_expert_ffn_matches_numpy, P.test_expert_ffn_hand_worked]),
+    10: ("router reads Wr transposed", [P.test_router_hand_worked]),
+    11: ("router drops the bias", [P.test_router_hand_worked]),
+    12: ("silu replaced by the plain sigmoid", [P.test_expert_ffn_hand_worked, P.test_shared_ffn_hand_worked]),
 }
 
 
@@ -50,7 +53,7 @@ def test_pins_catch_planted_mistake(n, tmp_path):
                 _run_pin(fn)
             except AssertionError:
                 caught += 1
-        assert caught, "planted mistake not caught: " + what
+        assert caught == len(pins), "planted mistake not caught by every listed pin: " + what
     finally:
         O.oracle.restore_library(prev)
 

@@ -336,3 +336,102 @@ def test_given_routing_overrides():
     ys = O.shared_ffn(c, d["shared_gate"], d["shared_up"], d["shared_down"], xt)
     ref = O.bf16_to_f64(res[t]) + 0.25 * O.expert_ffn(c, blobs[5], xt) + 0.75 * O.expert_ffn(c, blobs[6], xt) + ys
     np.testing.assert_allclose(h[t], ref, rtol=1e-12, atol=1e-13)
+
+
+# ---- hand-worked values (router projection, routed FFN, shared FFN) -------------
+
+def _lines(name):
+    for line in open(os.path.join(GOLDEN, name)):
+        f = line.split("#")[0].split()
+        if f:
+            yield f
+
+
+def test_router_hand_worked():
+    """Logits, top-K order and weights of tests/golden/router_hand.txt, every
+    value worked out by hand (transposing Wr or dropping the bias changes the
+    chosen experts there)."""
+    rows = list(_lines("router_hand.txt"))
+    H, E, K = map(int, next(f for f in rows if f[0] == "shape")[1:4])
+    fill = float(next(f for f in rows if f[0] == "wr_fill")[1])
+    T = 1 + max(int(f[1]) for f in rows if f[0] == "x")
+    x = np.zeros((T, H), np.float32)
+    wr = np.full((E, H), fill, np.float32)
+    bias = np.zeros(E, np.float32)
+    logit, top = {}, {}
+    for f in rows:
+        if f[0] == "x":
+            x[int(f[1]), int(f[2])] = float(f[3])
+        elif f[0] == "wr":
+            wr[int(f[1]), int(f[2])] = float(f[3])
+        elif f[0] == "bias":
+            bias[int(f[1])] = float(f[2])
+        elif f[0] == "logit":
+            logit[int(f[1]), int(f[2])] = float(f[3])
+        elif f[0] == "top":
+            top[int(f[1]), int(f[2])] = (int(f[3]), float(f[4]))
+    c = O.cfg(H, 64, E, K)
+    logits, idx, w = O.router(c, S.f32_to_bf16_bits(x), S.f32_to_bf16_bits(wr), bias)
+    for (t, e), v in logit.items():
+        assert logits[t, e] == np.float32(v), (t, e, logits[t, e], v)
+    _, _, w64 = O.topk(c, logits)
+    for (t, k), (e, d) in top.items():
+        assert idx[t, k] == e, (t, k)
+        assert abs(w64[t, k] - 1.0 / (1.0 + np.exp(-d))) < 1e-15, (t, k)
+        assert w[t, k] == np.float32(1.0 / (1.0 + np.exp(-d)))
+
+
+def _ffn_expect(rows):
+    L = np.log(3.0)
+    act = {int(f[1]): float(f[2]) * L * L for f in rows if f[0] == "act"}
+    y = {int(f[1]): float(f[2]) * L * L for f in rows if f[0] == "y"}
+    xs = {int(f[1]): float(f[2]) * L for f in rows if f[0] == "x"}
+    return xs, act, y
+
+
+def _check_vec(got, expect, n):
+    ref = np.zeros(n)
+    for i, v in expect.items():
+        ref[i] = v
+    np.testing.assert_allclose(got, ref, rtol=1e-14, atol=1e-14)
+
+
+def test_expert_ffn_hand_worked():
+    """silu(Wg x) * (Wu x) and Wd of it on the hand-packed expert of
+    tests/golden/expert_ffn_hand.txt (values are multiples of (ln 3)^2); the
+    FMA form of the same product must give the same numbers."""
+    rows = list(_lines("expert_ffn_hand.txt"))
+    H, I, b = map(int, next(f for f in rows if f[0] == "cfg")[1:4])
+    c = O.cfg(H, I, 4, 2, bits=b)
+    blob = np.zeros(O.expert_bytes(c), dtype=np.uint8)
+    off = O.section_offsets(c)
+    for f in rows:
+        if f[0] == "byte":
+            blob[off[int(f[1])] + int(f[2])] = int(f[3], 16)
+    xs, act, y = _ffn_expect(rows)
+    x = np.zeros(H)
+    for i, v in xs.items():
+        x[i] = v
+    _check_vec(O.expert_act(c, blob, x), act, I)
+    _check_vec(O.expert_ffn(c, blob, x), y, H)
+    _check_vec(O.expert_ffn_fma_form(c, blob, x), y, H)
+
+
+def test_shared_ffn_hand_worked():
+    """The bf16 shared expert on the hand-set weights of
+    tests/golden/shared_ffn_hand.txt (values are multiples of (ln 3)^2)."""
+    rows = list(_lines("shared_ffn_hand.txt"))
+    H, I = map(int, next(f for f in rows if f[0] == "shape")[1:3])
+    m = {"wg": np.zeros((I, H), np.float32), "wu": np.zeros((I, H), np.float32),
+         "wd": np.zeros((H, I), np.float32)}
+    for f in rows:
+        if f[0] in m:
+            m[f[0]][int(f[1]), int(f[2])] = float(f[3])
+    xs, act, y = _ffn_expect(rows)
+    x = np.zeros(H)
+    for i, v in xs.items():
+        x[i] = v
+    c = O.cfg(H, I, 4, 2)
+    got = O.shared_ffn(c, S.f32_to_bf16_bits(m["wg"]), S.f32_to_bf16_bits(m["wu"]),
+                       S.f32_to_bf16_bits(m["wd"]), x)
+    _check_vec(got, y, H)
