@@ -224,13 +224,21 @@ moe_status moe_layer_forward_routed(const moe_config* cfg, const moe_layer_weigh
  * and zeroes its counters with synchronous CUDA calls: make it before any
  * stream capture.  All calls on a device share the one scratch, so calls that
  * may overlap in time (other streams, other host threads) race and must be
- * serialised by the caller.  Device-side wait timeouts of this path are not
- * readable through moe_device_error (the scratch is internal). */
+ * serialised by the caller.  Each call first clears the scratch's error word
+ * on its stream (one 4-byte memset), so a device-side failure of one call (an
+ * expired wait, a bad expert pointer) leaves only that call's outputs
+ * unspecified; read it with moe_noalloc_device_error before the next call. */
 #define MOE_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
 moe_status moe_layer_forward_noalloc(const moe_config* cfg, const moe_layer_weights* wts,
                                      const void* x_bf16, const void* residual_bf16, int T,
                                      void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
                                      float* w_out, cudaStream_t stream);
+
+/* The device-side error of the last moe_layer_forward_noalloc call on the
+ * current device: as moe_device_error (synchronises the stream, clears the
+ * word), for the library's built-in scratch.  MOE_OK, MOE_ERR_TIMEOUT or
+ * MOE_ERR_DEVICE; *detail (may be NULL) gets the raw code. */
+moe_status moe_noalloc_device_error(uint32_t* detail, cudaStream_t stream);
 
 /* Per-phase timing of one layer call, in the spirit of the pages' per-layer
  * --timing breakdown ("Flash-MoE: ...", section "パイプライン概要"): the same

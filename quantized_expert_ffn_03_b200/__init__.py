@@ -23,6 +23,7 @@ _lib = C.CDLL(LIB_PATH)
 
 MOE_OK = 0
 MOE_ERR_WORKSPACE = 3
+MOE_ERR_DEVICE = 8
 NOALLOC_SCRATCH_BYTES = 4 << 20  # MOE_NOALLOC_SCRATCH_BYTES of moe.h
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_OOM", 6: "MOE_ERR_TIMEOUT", 7: "MOE_ERR_IO",
@@ -85,6 +86,7 @@ EXPORTS = {
     "moe_stream_stats": (C.c_int, [C.c_void_p, C.c_void_p]),
     "moe_stream_destroy": (None, [C.c_void_p]),
     "moe_device_error": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
+    "moe_noalloc_device_error": (C.c_int, [C.c_void_p, C.c_void_p]),
     "moe_selftest_bounded_wait": (C.c_int, [C.c_void_p, C.c_size_t, C.c_uint64, C.c_void_p]),
 }
 
@@ -301,6 +303,14 @@ def moe_device_error(workspace, stream=None):
     """Returns (status, detail) and clears the workspace's error word."""
     detail = C.c_uint32(0)
     st = _lib.moe_device_error(_ptr(workspace), C.byref(detail), _stream(stream))
+    return st, detail.value
+
+
+def moe_noalloc_device_error(stream=None):
+    """Returns (status, detail) of the last moe_layer_forward_noalloc call on
+    the current device and clears it."""
+    detail = C.c_uint32(0)
+    st = _lib.moe_noalloc_device_error(C.byref(detail), _stream(stream))
     return st, detail.value
 
 

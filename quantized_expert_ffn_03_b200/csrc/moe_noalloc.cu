@@ -11,10 +11,15 @@
 //
 // Set-up: the first call on a device (with that device current) looks up the
 // array's address with cudaGetSymbolAddress and zeroes its first 256 bytes
-// (the kernel's grid counters and error word, which must start at zero; the
-// kernel returns them to zero when it exits).  Those two calls are
-// synchronous, so make the first call on each device before any stream
-// capture.  Every call on a device shares the one scratch: calls that may
+// (the kernel's grid counters and error word, which must start at zero).
+// Those two calls are synchronous, so make the first call on each device
+// before any stream capture.  The kernel returns its grid counters to zero
+// when it exits, but not the error word (a failing launch leaves its code
+// there), so every call first clears the error word on its stream: one
+// call's device-side failure (a wait that expired, a bad expert pointer)
+// leaves that call's outputs unspecified and can be read with
+// moe_noalloc_device_error before the next call, and the next call starts
+// clean.  Every call on a device shares the one scratch: calls that may
 // overlap in time (on different streams or host threads) race on it and must
 // be serialised by the caller.
 #include <cuda_runtime.h>
@@ -39,8 +44,26 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
+constexpr size_t kErrOffset = 64;  // the kernel's error word inside the first 256 bytes
+
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices];  // per device, set on first use
+
+// The device address of g_scratch on device `dev` (current), looked up and
+// its first 256 bytes zeroed on first use.
+moe_status scratch_of(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+    if (e != cudaSuccess) return moe::abi_fail(MOE_ERR_CUDA, cudaGetErrorString(e));
+    e = cudaMemset(p, 0, 256);
+    if (e != cudaSuccess) return moe::abi_fail(MOE_ERR_CUDA, cudaGetErrorString(e));
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return MOE_OK;
+}
 
 }  // namespace
 
@@ -67,18 +90,24 @@ extern "C" moe_status moe_layer_forward_noalloc(const moe_config* cfg, const moe
   if (e != cudaSuccess) return moe::abi_fail(MOE_ERR_CUDA, cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return moe::abi_fail(MOE_ERR_UNSUPPORTED, "device index out of range");
   void* scratch = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
-      void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_scratch);
-      if (e != cudaSuccess) return moe::abi_fail(MOE_ERR_CUDA, cudaGetErrorString(e));
-      e = cudaMemset(p, 0, 256);
-      if (e != cudaSuccess) return moe::abi_fail(MOE_ERR_CUDA, cudaGetErrorString(e));
-      g_scratch_ptr[dev] = p;
-    }
-    scratch = g_scratch_ptr[dev];
+  const moe_status st = scratch_of(dev, &scratch);
+  if (st != MOE_OK) return st;
+  if (T > 0) {
+    // the previous call's error code must not outlive it (see the top of the file)
+    e = cudaMemsetAsync(static_cast<unsigned char*>(scratch) + kErrOffset, 0, 4, stream);
+    if (e != cudaSuccess) return moe::abi_fail(MOE_ERR_CUDA, cudaGetErrorString(e));
   }
   return moe::layer_forward_on(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out,
                                scratch, kScratchBytes, stream);
+}
+
+extern "C" moe_status moe_noalloc_device_error(uint32_t* detail, cudaStream_t stream) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return moe::abi_fail(MOE_ERR_CUDA, cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return moe::abi_fail(MOE_ERR_UNSUPPORTED, "device index out of range");
+  void* scratch = nullptr;
+  const moe_status st = scratch_of(dev, &scratch);
+  if (st != MOE_OK) return st;
+  return moe_device_error(scratch, detail, stream);
 }

@@ -21,7 +21,7 @@ def test_long_batch_matches_oracle_tiny():
 
 
 @pytest.mark.gpu
-def test_long_batch_equals_its_chunks_h4096():
+def test_long_batch_matches_oracle_and_its_chunks_h4096():
     import quantized_expert_ffn_03_b200 as M
     s = replace(S.QWEN_4BIT, tokens=16)
     dense = S.dense_weights(s)
@@ -30,6 +30,8 @@ def test_long_batch_equals_its_chunks_h4096():
     dl = DeviceLayer(s, expert_ids=idx_o.ravel().tolist(), dense=dense)
     C = M.moe_layer_tokens_per_launch(dl.cfg)
     assert 1 <= C <= 8
+    # token by token against the oracle (routing and outputs)
+    check_layer(dl, x, res)
     h, y, idx, w = dl.forward(x, res)  # ceil(16 / C) launches
     parts = [dl.forward(x[a:a + C], res[a:a + C]) for a in range(0, 16, C)]
     assert np.array_equal(h, np.concatenate([p[0] for p in parts]))

@@ -345,3 +345,58 @@ def test_streaming_matches_resident_h4096(M):
     lay = _Layers(M, s, n_layers=2, device_pack=True)
     st = _run_streaming(M, lay, n_slots=10, steps=4)
     assert st["misses"] > 0
+
+
+@pytest.mark.gpu
+def test_streaming_overlapped_matches_resident(M):
+    """Layers, resolves and prefetches enqueued back to back with one
+    synchronisation at the very end, so the side-stream prefetch of layer
+    l+1 may evict a slot that layer l-1's kernel is still reading: its copy
+    must wait for that kernel (the slot's "used" event).  Fewer slots than the
+    distinct experts of two layers force such evictions.  Every layer's
+    outputs must equal, bit for bit, the resident routed call's."""
+    import torch
+    s = replace(S.TINY, tokens=2)
+    L, steps, n_slots = 4, 6, 5
+    lay = _Layers(M, s, n_layers=L)
+    E = s.n_experts
+    # routing, inputs and resident reference outputs first (these synchronise)
+    plan = []
+    for step in range(steps):
+        for l in range(L):
+            dl = lay.layers[l]
+            x, res = S.activations(s, step=step, replica=l)
+            _, idx, w = dl.router(x)
+            pred = lay.layers[l + 1].router(x)[1] if l + 1 < L else None
+            xd, rd, idd, wd = to_dev_bits(x), to_dev_bits(res), _dev(idx), _dev(w)
+            h1, y1 = torch.empty_like(xd), torch.empty_like(xd)
+            M.moe_layer_forward_routed(lay.cfg, dl.wts, xd, rd, idd, wd, h1, y1, dl.ws)
+            plan.append((l, idx, pred, xd, rd, idd, wd, h1, y1))
+    torch.cuda.synchronize()
+    cache = M.moe_stream_create(lay.cfg, L, lay.store, n_slots)
+    side = torch.cuda.Stream()
+    table = torch.zeros(E, dtype=torch.int64, device="cuda")
+    ws = torch.zeros(M.moe_layer_workspace_bytes(lay.cfg, 8), dtype=torch.uint8, device="cuda")
+    M.moe_workspace_init(ws)
+    outs = []
+    try:
+        torch.cuda.synchronize()
+        for l, idx, pred, xd, rd, idd, wd, _, _ in plan:
+            dl = lay.layers[l]
+            M.moe_stream_resolve(cache, l, idx.ravel(), table)
+            wts = M.layer_weights(table, None, None, dl.sg, dl.su, dl.sd, dl.gamma)
+            h2, y2 = torch.empty_like(xd), torch.empty_like(xd)
+            M.moe_layer_forward_routed(lay.cfg, wts, xd, rd, idd, wd, h2, y2, ws)
+            outs.append((h2, y2))
+            if pred is not None:
+                M.moe_stream_prefetch(cache, l + 1, pred.ravel(), copy_stream=side)
+        torch.cuda.synchronize()
+        assert M.moe_device_error(ws)[0] == 0
+        st = M.moe_stream_stats(cache)
+        assert st["misses"] > 0 and st["prefetches"] > 0
+        for i, ((h2, y2), p) in enumerate(zip(outs, plan)):
+            assert np.array_equal(from_dev_bits(h2), from_dev_bits(p[7])), i
+            assert np.array_equal(from_dev_bits(y2), from_dev_bits(p[8])), i
+    finally:
+        torch.cuda.synchronize()
+        M.moe_stream_destroy(cache)

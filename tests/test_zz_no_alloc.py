@@ -69,3 +69,32 @@ def test_noalloc_matches_workspace_path_twice(M, shape):
         np.testing.assert_allclose(w.cpu().numpy(), w_ref.cpu().numpy(), rtol=2e-6, atol=1e-7)
         _close(from_dev_bits(h), from_dev_bits(h_ref), "h_out call %d" % call)
         _close(from_dev_bits(y), from_dev_bits(y_ref), "y_norm call %d" % call)
+
+
+@pytest.mark.gpu
+def test_noalloc_failed_call_does_not_poison_the_next(M):
+    """A call whose expert table holds misaligned pointers fails on the device
+    (the kernel checks every chosen pointer before any access); the next good
+    call must write its outputs and match moe_layer_forward, whether or not
+    the failure was read in between."""
+    import torch
+    s = S.TINY
+    dl = DeviceLayer(s)
+    bad_ptr = dl.expert_ptr.clone()
+    bad_ptr += 16
+    bad = M.layer_weights(bad_ptr, dl.wr, dl.bias, dl.sg, dl.su, dl.sd, dl.gamma)
+    x, res = S.activations(s, step=5)
+    xd, rd = to_dev_bits(x), to_dev_bits(res)
+    h_ref, y_ref = torch.empty_like(xd), torch.empty_like(xd)
+    M.moe_layer_forward(dl.cfg, dl.wts, xd, rd, h_ref, y_ref, workspace=dl.ws)
+    torch.cuda.synchronize()
+    for read_error in (False, True):
+        h, y = torch.empty_like(xd), torch.empty_like(xd)
+        M.moe_layer_forward_noalloc(dl.cfg, bad, xd, rd, h, y)
+        if read_error:
+            assert M.moe_noalloc_device_error() == (M.MOE_ERR_DEVICE, 2)
+        h, y = torch.full_like(xd, 0x7fc0), torch.full_like(xd, 0x7fc0)
+        M.moe_layer_forward_noalloc(dl.cfg, dl.wts, xd, rd, h, y)
+        assert M.moe_noalloc_device_error() == (M.MOE_OK, 0)
+        _close(from_dev_bits(h), from_dev_bits(h_ref), "h_out after a failed call (read=%s)" % read_error)
+        _close(from_dev_bits(y), from_dev_bits(y_ref), "y_norm after a failed call (read=%s)" % read_error)
