@@ -309,19 +309,21 @@ typedef struct moe_stream_cache moe_stream_cache;
 
 /* Creates a cache: allocates n_slots * moe_packed_expert_bytes of device
  * memory (the one call of the library that allocates device memory) and two
- * CUDA events per slot.  host_pinned_experts must be page-locked
- * (cudaHostAlloc / cudaHostRegister) and stay valid until destroy.
- * MOE_ERR_OOM if the slots do not fit; MOE_ERR_INVALID_ARG for a pageable
- * store, n_layers < 1 or n_slots < 1. */
+ * CUDA events per slot.  host_pinned_experts (store_bytes long) must hold
+ * n_layers * n_experts blobs in page-locked memory (cudaHostAlloc /
+ * cudaHostRegister) and stay valid until destroy.  MOE_ERR_OOM if the slots
+ * do not fit; MOE_ERR_INVALID_ARG for a store shorter than the blobs need or
+ * not page-locked (both ends are checked), n_layers < 1 or n_slots < 1. */
 moe_status moe_stream_create(const moe_config* cfg, int n_layers, const void* host_pinned_experts,
-                             int n_slots, moe_stream_cache** out);
+                             size_t store_bytes, int n_slots, moe_stream_cache** out);
 
 /* Enqueues on copy_stream the copies of those of expert_ids_host[0..n)
  * (experts of `layer`) that are not resident, each into the least recently
  * used slot that no resolve call holds; the copy waits for the last kernel
  * that read the slot.  A hint: ids that find no free slot are skipped
  * (counted in prefetch_dropped).  Does not synchronise.  MOE_ERR_IO if a
- * copy cannot be enqueued. */
+ * copy cannot be enqueued (its slot is left empty; the ids after it are not
+ * looked at). */
 moe_status moe_stream_prefetch(moe_stream_cache* cache, int layer, const int32_t* expert_ids_host,
                                int n, cudaStream_t copy_stream);
 
@@ -330,7 +332,11 @@ moe_status moe_stream_prefetch(moe_stream_cache* cache, int layer, const int32_t
  * for prefetch copies still in flight.  Then writes expert_ptr_dev (device
  * array [E] of device pointers) on compute_stream: the slot of every
  * resolved expert; other entries are unspecified.  MOE_ERR_OOM if the
- * distinct ids outnumber the slots.  Does not synchronise. */
+ * distinct ids outnumber the slots; MOE_ERR_IO if a miss cannot be copied
+ * (the table is not written, the slots of this call are released, the cache
+ * stays usable).  Does not synchronise the device, but blocks the calling
+ * thread when 8 resolves are still in flight (its pinned staging ring), so it
+ * must not be called while compute_stream is being captured. */
 moe_status moe_stream_resolve(moe_stream_cache* cache, int layer, const int32_t* idx_host, int n,
                               const void** expert_ptr_dev, cudaStream_t compute_stream);
 
@@ -346,6 +352,17 @@ moe_status moe_stream_stats(const moe_stream_cache* cache, moe_stream_counters* 
 /* Waits for the cache's copies and kernels that may still use its slots
  * (synchronises the device), then frees the slots and events. */
 void moe_stream_destroy(moe_stream_cache* cache);
+
+/* Host-side fault injection for tests of the streaming tier's error paths
+ * (no counterpart on the pages; nothing is done to the GPU):
+ *   MOE_FAULT_COPY:  the copy issued after `countdown` more copies on this
+ *                    cache reports failure instead of being enqueued (the
+ *                    calling prefetch or resolve returns MOE_ERR_IO);
+ *   MOE_FAULT_ALLOC: the next moe_stream_create's slot allocation reports
+ *                    failure (MOE_ERR_OOM); cache may be NULL;
+ *   MOE_FAULT_NONE:  clears both. */
+enum { MOE_FAULT_NONE = 0, MOE_FAULT_COPY = 1, MOE_FAULT_ALLOC = 2 };
+moe_status moe_stream_inject_fault(moe_stream_cache* cache, int what, int countdown);
 
 /* Read (synchronising the stream) and clear the device-side error word of a
  * layer workspace.  Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE;

@@ -80,7 +80,8 @@ EXPORTS = {
     "moe_layer_forward_routed": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                            C.c_size_t, C.c_void_p]),
-    "moe_stream_create": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p]),
+    "moe_stream_create": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_size_t, C.c_int, C.c_void_p]),
+    "moe_stream_inject_fault": (C.c_int, [C.c_void_p, C.c_int, C.c_int]),
     "moe_stream_prefetch": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p]),
     "moe_stream_resolve": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
     "moe_stream_stats": (C.c_int, [C.c_void_p, C.c_void_p]),
@@ -122,6 +123,17 @@ def _ptr(t):
     if isinstance(t, np.ndarray):
         return t.ctypes.data
     return t.data_ptr()
+
+
+def _nbytes(t):
+    """Byte size of a torch tensor / numpy array (0 for None)."""
+    if t is None:
+        return 0
+    if isinstance(t, np.ndarray):
+        return t.nbytes
+    if isinstance(t, int):
+        raise TypeError("a raw address needs an explicit byte count")
+    return t.numel() * t.element_size()
 
 
 def _stream(stream):
@@ -265,12 +277,23 @@ class MoeStreamCounters(C.Structure):
                 ("prefetch_hits", C.c_uint64), ("prefetch_dropped", C.c_uint64), ("bytes_h2d", C.c_uint64)]
 
 
-def moe_stream_create(cfg, n_layers, host_store, n_slots):
-    """host_store: pinned host tensor (or address) of n_layers*E packed blobs.
-    Returns the cache handle (an int)."""
+def moe_stream_create(cfg, n_layers, host_store, n_slots, store_bytes=None):
+    """host_store: pinned host tensor (or address) of n_layers*E packed blobs;
+    store_bytes defaults to the tensor's size.  Returns the cache handle (an
+    int)."""
+    if store_bytes is None:
+        store_bytes = _nbytes(host_store)
     h = C.c_void_p(0)
-    _check(_lib.moe_stream_create(C.byref(cfg), int(n_layers), _ptr(host_store), int(n_slots), C.byref(h)))
+    _check(_lib.moe_stream_create(C.byref(cfg), int(n_layers), _ptr(host_store), int(store_bytes), int(n_slots),
+                                  C.byref(h)))
     return h.value
+
+
+MOE_FAULT_NONE, MOE_FAULT_COPY, MOE_FAULT_ALLOC = 0, 1, 2
+
+
+def moe_stream_inject_fault(cache, what, countdown=0):
+    _check(_lib.moe_stream_inject_fault(cache, int(what), int(countdown)))
 
 
 def _ids(ids):

@@ -11,15 +11,26 @@
 // event per slot marking its copy done ("ready") and one marking the last
 // kernel that read it done ("used").
 //
-// Ordering rules (all on the GPU, no host waits):
+// Ordering rules (all on the GPU; the one host wait is noted below):
 //   - a copy into a slot waits for the slot's "used" event and for any copy
 //     into it still in flight ("ready"), then records "ready";
 //   - a resolve makes the compute stream wait for "ready" of every slot it
 //     hands out; those slots are held (never chosen as victims) until the
 //     next resolve, which records their "used" event on its compute stream,
 //     i.e. after the layer kernel the caller enqueued in between;
-//   - the pointer table is copied from a pinned staging buffer of a small
-//     ring; a buffer is reused only after the event of its last copy.
+//   - the pointer table is copied from a pinned staging buffer of a ring of
+//     kStage; a buffer is reused only after the event of its last copy, which
+//     the host waits for (cudaEventSynchronize) when kStage resolves are still
+//     in flight on the GPU.  A resolve can therefore block the host thread,
+//     and must not be called while its stream is being captured into a
+//     CUDA graph.
+//
+// Failures: a copy that cannot be enqueued (MOE_ERR_IO) leaves its slot
+// empty, and a resolve that fails releases the slots it took, so the next
+// call starts from a consistent cache.  Tests drive these paths with
+// moe_stream_inject_fault (a host-side countdown that makes a chosen copy,
+// or the next create's slot allocation, report failure without touching
+// the GPU).
 #include <cuda_runtime.h>
 
 #include <cstdarg>
@@ -64,8 +75,14 @@ struct moe_stream_cache {
   bool stage_used[kStage] = {};
   int stage_next = 0;
   uint64_t bytes_h2d = 0;
+  int fault_copy = -1;  // injected: copies left before one fails (-1: none)
   std::mutex mu;
 };
+
+namespace {
+int g_fault_alloc = 0;  // injected: the next create's slot allocation fails
+std::mutex g_fault_mu;
+}  // namespace
 
 namespace {
 
@@ -88,10 +105,16 @@ moe_status fill_slot(moe_stream_cache* c, int s, int layer, int e, cudaStream_t 
   if (err == cudaSuccess) err = cudaStreamWaitEvent(st, c->ready[s], 0);
   if (err != cudaSuccess) return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
   const uint8_t* src = c->host + ((size_t)layer * c->E + e) * c->blob;
+  if (c->fault_copy >= 0 && c->fault_copy-- == 0) {
+    c->pol.evict(s);
+    return failf(MOE_ERR_IO, "copy of expert %d of layer %d from the host store failed: injected fault", e, layer);
+  }
   err = cudaMemcpyAsync(c->slots + (size_t)s * c->blob, src, c->blob, cudaMemcpyHostToDevice, st);
-  if (err != cudaSuccess)
+  if (err != cudaSuccess) {
+    c->pol.evict(s);
     return failf(MOE_ERR_IO, "copy of expert %d of layer %d from the host store failed: %s", e, layer,
                  cudaGetErrorString(err));
+  }
   err = cudaEventRecord(c->ready[s], st);
   if (err != cudaSuccess) return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
   c->bytes_h2d += c->blob;
@@ -122,7 +145,7 @@ struct DeviceGuard {
 extern "C" {
 
 moe_status moe_stream_create(const moe_config* cfg, int n_layers, const void* host_pinned_experts,
-                             int n_slots, moe_stream_cache** out) {
+                             size_t store_bytes, int n_slots, moe_stream_cache** out) {
   if (!out) return failf(MOE_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if (!cfg) return failf(MOE_ERR_INVALID_ARG, "cfg is NULL");
@@ -130,8 +153,15 @@ moe_status moe_stream_create(const moe_config* cfg, int n_layers, const void* ho
   if (blob == 0 || cfg->n_experts <= 0) return failf(MOE_ERR_UNSUPPORTED, "unsupported shape");
   if (n_layers < 1 || n_slots < 1) return failf(MOE_ERR_INVALID_ARG, "n_layers and n_slots must be >= 1");
   if (!host_pinned_experts) return failf(MOE_ERR_INVALID_ARG, "host store is NULL");
-  cudaPointerAttributes attr;
-  if (cudaPointerGetAttributes(&attr, host_pinned_experts) != cudaSuccess || attr.type != cudaMemoryTypeHost) {
+  const size_t need = blob * (size_t)cfg->n_experts * (size_t)n_layers;
+  if (store_bytes < need)
+    return failf(MOE_ERR_INVALID_ARG, "the host store holds %zu bytes; %d layers of %d experts need %zu", store_bytes,
+                 n_layers, cfg->n_experts, need);
+  // both ends of the store must be page-locked memory
+  cudaPointerAttributes attr, attr_end;
+  const uint8_t* last_byte = static_cast<const uint8_t*>(host_pinned_experts) + need - 1;
+  if (cudaPointerGetAttributes(&attr, host_pinned_experts) != cudaSuccess || attr.type != cudaMemoryTypeHost ||
+      cudaPointerGetAttributes(&attr_end, last_byte) != cudaSuccess || attr_end.type != cudaMemoryTypeHost) {
     cudaGetLastError();
     return failf(MOE_ERR_INVALID_ARG, "the host store must be page-locked (cudaHostAlloc or cudaHostRegister)");
   }
@@ -143,7 +173,13 @@ moe_status moe_stream_create(const moe_config* cfg, int n_layers, const void* ho
   c->host = static_cast<const uint8_t*>(host_pinned_experts);
   cudaGetDevice(&c->device);
   c->pol.init(n_layers, cfg->n_experts, n_slots);
-  if (cudaMalloc(&c->slots, blob * (size_t)n_slots) != cudaSuccess) {
+  bool alloc_fault = false;
+  {
+    std::lock_guard<std::mutex> lk(g_fault_mu);
+    alloc_fault = g_fault_alloc != 0;
+    g_fault_alloc = 0;
+  }
+  if (alloc_fault || cudaMalloc(&c->slots, blob * (size_t)n_slots) != cudaSuccess) {
     cudaGetLastError();
     c->slots = nullptr;
     destroy_parts(c);
@@ -178,7 +214,10 @@ moe_status moe_stream_prefetch(moe_stream_cache* c, int layer, const int32_t* id
   DeviceGuard dg(c->device);
   for (int i = 0; i < n; ++i) {
     const int v = c->pol.prefetch(layer, ids[i]);
-    if (v >= 0 && (s = fill_slot(c, v, layer, ids[i], copy_stream)) != MOE_OK) return s;
+    if (v >= 0 && (s = fill_slot(c, v, layer, ids[i], copy_stream)) != MOE_OK) {
+      --c->pol.prefetches;  // not issued
+      return s;
+    }
   }
   return MOE_OK;
 }
@@ -212,8 +251,13 @@ moe_status moe_stream_resolve(moe_stream_cache* c, int layer, const int32_t* idx
     if (slot < 0)
       return failf(MOE_ERR_OOM, "the cache's %d slots cannot hold the distinct experts of one call", c->S);
     if (fill) {
-      if ((s = fill_slot(c, slot, layer, e, st)) != MOE_OK) return s;
+      if ((s = fill_slot(c, slot, layer, e, st)) != MOE_OK) {
+        --c->pol.misses;  // not issued
+        c->pol.release();  // no layer will read this call's slots
+        return s;
+      }
     } else if ((err = cudaStreamWaitEvent(st, c->ready[slot], 0)) != cudaSuccess) {
+      c->pol.release();
       return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
     }
     tab[e] = c->slots + (size_t)slot * c->blob;
@@ -224,6 +268,30 @@ moe_status moe_stream_resolve(moe_stream_cache* c, int layer, const int32_t* idx
     return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
   c->stage_used[sb] = true;
   return MOE_OK;
+}
+
+moe_status moe_stream_inject_fault(moe_stream_cache* c, int what, int countdown) {
+  if (what == MOE_FAULT_NONE) {
+    if (c) {
+      std::lock_guard<std::mutex> lk(c->mu);
+      c->fault_copy = -1;
+    }
+    std::lock_guard<std::mutex> lk(g_fault_mu);
+    g_fault_alloc = 0;
+    return MOE_OK;
+  }
+  if (what == MOE_FAULT_COPY) {
+    if (!c || countdown < 0) return failf(MOE_ERR_INVALID_ARG, "a copy fault needs a cache and a countdown >= 0");
+    std::lock_guard<std::mutex> lk(c->mu);
+    c->fault_copy = countdown;
+    return MOE_OK;
+  }
+  if (what == MOE_FAULT_ALLOC) {
+    std::lock_guard<std::mutex> lk(g_fault_mu);
+    g_fault_alloc = 1;
+    return MOE_OK;
+  }
+  return failf(MOE_ERR_INVALID_ARG, "unknown fault %d", what);
 }
 
 moe_status moe_stream_stats(const moe_stream_cache* c, moe_stream_counters* out) {

@@ -56,6 +56,12 @@ struct StreamPolicy {
     table[(size_t)layer * E + e] = s;
     fresh[s] = 0;
   }
+  // Slot s holds nothing valid any more (its fill could not be issued).
+  void evict(int s) {
+    if (key[s] >= 0) table[key[s]] = -1;
+    key[s] = -1;
+    fresh[s] = 0;
+  }
   // Prefetch of (layer, e): the slot to fill, or -1 (already resident, which
   // counts as a use, or no slot free of the step in flight: dropped).
   int prefetch(int layer, int e) {

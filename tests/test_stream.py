@@ -400,3 +400,79 @@ def test_streaming_overlapped_matches_resident(M):
     finally:
         torch.cuda.synchronize()
         M.moe_stream_destroy(cache)
+
+
+# ---- failures injected on the host (no GPU fault) ------------------------------------
+
+@pytest.mark.gpu
+def test_stream_create_rejects_a_short_store_and_an_injected_alloc_failure(M):
+    import torch
+    s = replace(S.TINY, tokens=2)
+    cfg = mcfg(s)
+    nb = M.moe_packed_expert_bytes(cfg)
+    store = torch.zeros((2 * s.n_experts, nb), dtype=torch.uint8).pin_memory()
+    with pytest.raises(M.MoeError) as ei:  # 2 layers' blobs, 3 layers claimed
+        M.moe_stream_create(cfg, 3, store, 4)
+    assert ei.value.status == M.STATUS_BY_NAME["MOE_ERR_INVALID_ARG"] and "holds" in str(ei.value)
+    with pytest.raises(M.MoeError) as ei:  # a byte count below the blobs' size
+        M.moe_stream_create(cfg, 2, store, 4, store_bytes=2 * s.n_experts * nb - 1)
+    assert ei.value.status == M.STATUS_BY_NAME["MOE_ERR_INVALID_ARG"]
+    M.moe_stream_inject_fault(None, M.MOE_FAULT_ALLOC)
+    with pytest.raises(M.MoeError) as ei:
+        M.moe_stream_create(cfg, 2, store, 4)
+    assert ei.value.status == M.STATUS_BY_NAME["MOE_ERR_OOM"]
+    cache = M.moe_stream_create(cfg, 2, store, 4)  # one-shot: the next create works
+    M.moe_stream_destroy(cache)
+
+
+@pytest.mark.gpu
+def test_stream_copy_failure_is_reported_and_the_cache_recovers(M):
+    """A failing host-to-device copy (injected on the host) makes resolve and
+    prefetch return MOE_ERR_IO with a message; the cache keeps no slot for the
+    expert whose copy failed, and the next calls produce the resident routed
+    call's outputs bit for bit."""
+    import torch
+    s = replace(S.TINY, tokens=2)
+    lay = _Layers(M, s, n_layers=2)
+    E = s.n_experts
+    cache = M.moe_stream_create(lay.cfg, 2, lay.store, 6)
+    table = torch.zeros(E, dtype=torch.int64, device="cuda")
+    ws = torch.zeros(M.moe_layer_workspace_bytes(lay.cfg, 8), dtype=torch.uint8, device="cuda")
+    M.moe_workspace_init(ws)
+    try:
+        dl = lay.layers[0]
+        x, res = S.activations(s, step=7)
+        _, idx, w = dl.router(x)
+        distinct = len(set(idx.ravel().tolist()))
+        assert distinct >= 2
+        # the second miss of this resolve fails
+        M.moe_stream_inject_fault(cache, M.MOE_FAULT_COPY, 1)
+        with pytest.raises(M.MoeError) as ei:
+            M.moe_stream_resolve(cache, 0, idx.ravel(), table)
+        assert ei.value.status == M.STATUS_BY_NAME["MOE_ERR_IO"] and "injected" in str(ei.value)
+        st = M.moe_stream_stats(cache)
+        assert st["misses"] == 1 and st["hits"] == 0
+        # a prefetch whose first copy fails
+        M.moe_stream_inject_fault(cache, M.MOE_FAULT_COPY, 0)
+        with pytest.raises(M.MoeError) as ei:
+            M.moe_stream_prefetch(cache, 1, [0, 1])
+        assert ei.value.status == M.STATUS_BY_NAME["MOE_ERR_IO"]
+        assert M.moe_stream_stats(cache)["prefetches"] == 0
+        # recovery: resolve again and run the layer
+        M.moe_stream_resolve(cache, 0, idx.ravel(), table)
+        st = M.moe_stream_stats(cache)
+        assert st["misses"] + st["hits"] == 1 + distinct
+        xd, rd, idd, wd = to_dev_bits(x), to_dev_bits(res), _dev(idx), _dev(w)
+        wts = M.layer_weights(table, None, None, dl.sg, dl.su, dl.sd, dl.gamma)
+        h2, y2 = torch.empty_like(xd), torch.empty_like(xd)
+        M.moe_layer_forward_routed(lay.cfg, wts, xd, rd, idd, wd, h2, y2, ws)
+        h1, y1 = torch.empty_like(xd), torch.empty_like(xd)
+        M.moe_layer_forward_routed(lay.cfg, dl.wts, xd, rd, idd, wd, h1, y1, dl.ws)
+        torch.cuda.synchronize()
+        assert M.moe_device_error(ws)[0] == 0
+        assert np.array_equal(from_dev_bits(h1), from_dev_bits(h2))
+        assert np.array_equal(from_dev_bits(y1), from_dev_bits(y2))
+    finally:
+        M.moe_stream_inject_fault(cache, M.MOE_FAULT_NONE)
+        torch.cuda.synchronize()
+        M.moe_stream_destroy(cache)
