@@ -63,6 +63,12 @@ constexpr int kTraceEntries = 128;
 // accumulator entries large enough for every row block of kSlots tiles.
 constexpr int kMaxRbPerTile = 2;
 constexpr int kAccSlots = kSlots * kMaxRbPerTile;
+// One-token router and shared gate/up tiles with few rows: each row is dotted
+// in up to kMaxParts column parts by different warps (a tile of at most
+// kSplitRows rows), and the warp that finishes a row's last part sums the
+// parts in order.
+constexpr int kSplitRows = 7;
+constexpr int kMaxParts = 14;
 
 enum TileType : int { TILE_NONE = 0, TILE_ROUTER, TILE_SHARED_GU, TILE_EXPERT_GU, TILE_SHARED_DOWN, TILE_EXPERT_DOWN };
 
@@ -83,7 +89,7 @@ struct Seg {
   int u0, u1; // routed tiles: units of each row block held in the slot
   int gbase;  // routed tiles: first group held (0 for whole row blocks)
   int acc;    // routed gate/up: accumulator entry of the first row block
-  uint32_t off[4];  // slot byte offset of each range's first valid byte
+  uint32_t off[8];  // slot byte offset of each range's first valid byte
 };
 
 struct TileDesc {
@@ -108,15 +114,15 @@ enum { FLAG_TOPK = NGO, FLAG_SCNT, FLAG_LAST };
 // hf: routed intermediate as A fragments (hi/lo), [pair][group][t][step] x 16 bytes.
 // hx: per (pair, 8-row block of I) sum of hi + lo.
 struct DecodeSmem {
-  size_t ring, bars, desc, xs, xf, xsum, hs, hf, hx, zero, part, cnt, tk_w, tk_i, eptr, tkbuf, res, gam, ypart,
-      ys, hacc, inv, flags, spin, total;
+  size_t ring, bars, desc, xs, xf, xsum, hs, hf, hx, zero, part, cnt, rpart, rcnt, tk_w, tk_i, eptr, tkbuf, res, gam,
+      ypart, ys, hacc, inv, flags, spin, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
 
 __host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int E, int H, int I, int nrows, int nslots,
                                                        uint32_t slot_bytes) {
-  const RoutedGeo gi = routed_geo(I);
+  const RoutedGeo gi = routed_geo(I, 4);
   DecodeSmem s;
   size_t pos = 0;
   s.ring = pos;
@@ -136,13 +142,17 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int E, int 
   s.hf = pos;
   pos = align_up(pos + 4ull * T * K * I, 16);
   s.hx = pos;
-  pos = align_up(pos + 4ull * T * K * (I / 8), 16);
+  pos = align_up(pos + 4ull * T * K * (I / 16), 16);
   s.zero = pos;
   pos = align_up(pos + 64, 16);
   s.part = pos;
-  pos = align_up(pos + 4ull * kAccSlots * kMaxUnits * 16, 16);
+  pos = align_up(pos + 4ull * kAccSlots * kMaxUnits * 32, 16);
   s.cnt = pos;
   pos = align_up(pos + 4ull * kAccSlots, 16);
+  s.rpart = pos;
+  pos = align_up(pos + 4ull * kSlots * kSplitRows * kMaxParts * 2, 16);
+  s.rcnt = pos;
+  pos = align_up(pos + 4ull * kSlots * kSplitRows, 16);
   s.tk_w = pos;
   pos = align_up(pos + sizeof(float) * T * K, 16);
   s.tk_i = pos;
@@ -403,121 +413,140 @@ __device__ __forceinline__ void load_codes<FMT_Q4>(LaneCodes<FMT_Q4>& c, uint32_
 template <>
 __device__ __forceinline__ void load_codes<FMT_Q2>(LaneCodes<FMT_Q2>& c, uint32_t a) { c.w = lds32(a); }
 
-// One unit of a routed tile: windows [u*W, u*W + W) of 8-row block `rbl` of
-// the segment.  GU: gate and up against x (bf16, A rows 0..7); otherwise down
-// against the routed intermediate (hi in A rows 0..7, lo in rows 8..15).
-// afrag: this token's (pair's) A fragments; asum: its group sums (GU) or
-// 8-row partial sums (down); sl, afrag, asum, zero4 are shared-memory
-// addresses.  Returns rows 2t and 2t+1 of the block in res[matrix][0/1]
-// (every lane t, t = lane % 4, holds the sums of its rows).
+// One unit of a routed tile: windows [u*W, u*W + W) of the 16-row block of the
+// segment (its two 8-row halves, codes at sg.off[2m + h], scales at
+// sg.off[2*NM + 2m + h] for matrix m and half h).  The weights are the A
+// operand: lane (g, t) = (lane / 4, lane % 4) holds rows g and g + 8 of a
+// 16-column step, which are exactly its code bytes of the two 8-row halves.
+// The activations are the B operand, one window of groups per pass of steps:
+// GU: column n of B carries group n of the window (x, from bfrag =
+// [group][t][8 words]), zero in the other groups' steps; down: columns 2n and
+// 2n + 1 carry the bf16 hi and lo parts of group n of the intermediate (bfrag
+// = [group][hi/lo][t][8 words]).  After a window, D[r][n] is group n's code
+// dot of row r, and the group's scale and bias are applied to it:
+//   sum_k x_k (q_k s + beta) = s * D + (beta - 128 s) * X.
+// bsum: GU [group] sums of x; down [16-row block] sums of hi + lo.
+// Returns in res[m][0] / res[m][1] the unit's sums of rows g and g + 8 (every
+// lane of lane group g holds them).
 template <int FMT, bool GU>
-__device__ __forceinline__ void routed_unit(uint32_t sl, const Seg& sg, int rbl, int u, const RoutedGeo& geo,
-                                            uint32_t afrag, uint32_t asum, uint32_t zero4, float (&res)[2][2]) {
+__device__ __forceinline__ void routed_unit(uint32_t sl, const Seg& sg, int u, const RoutedGeo& geo, uint32_t bfrag,
+                                            uint32_t bsum, float (&res)[2][2]) {
   constexpr int NM = GU ? 2 : 1;
-  constexpr int NA = GU ? 2 : 4;  // 16-byte A pieces per lane and group
+  constexpr int GPW = GU ? 8 : 4;
   constexpr int CB = LaneCodes<FMT>::kBytes;
   constexpr int BB = 32 * CB;  // code bytes of one 8x64 block
-  const int lane = threadIdx.x & 31, m = lane >> 2, t = lane & 3;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   float acc[NM][2];
 #pragma unroll
   for (int mm = 0; mm < NM; ++mm) acc[mm][0] = acc[mm][1] = 0.f;
   const int wa = u * geo.W, wb = min(wa + geo.W, geo.nwin);
-  const int blk0 = rbl * geo.G - sg.gbase;
-  uint32_t cbase[NM], sbase[NM];
+  uint32_t cbase[NM][2], sbase[NM][2];
 #pragma unroll
-  for (int mm = 0; mm < NM; ++mm) {
-    cbase[mm] = sl + sg.off[mm] + (uint32_t)(blk0 * BB + lane * CB);
-    sbase[mm] = sl + sg.off[NM + mm] + (uint32_t)(blk0 * 32 + t * 8);
-  }
+  for (int mm = 0; mm < NM; ++mm)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      cbase[mm][h] = sl + sg.off[2 * mm + h] + (uint32_t)(lane * CB) - (uint32_t)(sg.gbase * BB);
+      sbase[mm][h] = sl + sg.off[2 * NM + 2 * mm + h] + (uint32_t)(g * 4) - (uint32_t)(sg.gbase * 32);
+    }
+  // this lane's B column: group bg of the window, part bh (down: 0 hi, 1 lo)
+  const int bg = GU ? g : (g >> 1);
 #pragma unroll 1
   for (int w = wa; w < wb; ++w) {
-    const int g0 = 8 * w, nv = min(8, geo.G - g0);
-    float d[NM][4][4];
-#pragma unroll
-    for (int mm = 0; mm < NM; ++mm)
-#pragma unroll
-      for (int s = 0; s < 4; ++s) d[mm][s][0] = d[mm][s][1] = d[mm][s][2] = d[mm][s][3] = 0.f;
-    // lane group m presents group g0 + m's activations in step j == m only
-    const uint32_t a_own = afrag + (uint32_t)(((g0 + m) * 4 + t) * NA * 16);
-    const uint32_t cw = (uint32_t)(g0 * BB);
-#pragma unroll 1
-    for (int j = 0; j < nv; ++j) {
-      const uint32_t ap = (m == j) ? a_own : zero4;
-      uint32_t a[4][4];
-      if constexpr (GU) {
-        const uint4 v0 = lds128(ap), v1 = lds128(ap + 16);
-        a[0][0] = v0.x, a[0][2] = v0.y, a[1][0] = v0.z, a[1][2] = v0.w;
-        a[2][0] = v1.x, a[2][2] = v1.y, a[3][0] = v1.z, a[3][2] = v1.w;
-#pragma unroll
-        for (int s = 0; s < 4; ++s) a[s][1] = a[s][3] = 0u;
-      } else {
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const uint4 v = lds128(ap + 16 * s);
-          a[s][0] = v.x, a[s][1] = v.y, a[s][2] = v.z, a[s][3] = v.w;
-        }
+    const int g0 = GPW * w, nv = min(GPW, geo.G - g0);
+    uint32_t xb[8];
+    {
+      const uint32_t a = GU ? bfrag + (uint32_t)(((g0 + bg) * 4 + t) * 32)
+                            : bfrag + (uint32_t)((((g0 + bg) * 2 + (g & 1)) * 4 + t) * 32);
+      uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+      if (bg < nv) {
+        v0 = lds128(a);
+        v1 = lds128(a + 16);
       }
-      LaneCodes<FMT> c[NM];
+      xb[0] = v0.x, xb[1] = v0.y, xb[2] = v0.z, xb[3] = v0.w;
+      xb[4] = v1.x, xb[5] = v1.y, xb[6] = v1.z, xb[7] = v1.w;
+    }
+    float d[NM][4];
 #pragma unroll
-      for (int mm = 0; mm < NM; ++mm) load_codes<FMT>(c[mm], cbase[mm] + cw + (uint32_t)(j * BB));
+    for (int mm = 0; mm < NM; ++mm) d[mm][0] = d[mm][1] = d[mm][2] = d[mm][3] = 0.f;
 #pragma unroll
-      for (int mm = 0; mm < NM; ++mm) {
-        uint32_t b[4][2];
-        c[mm].frags(b);
+    for (int j = 0; j < GPW; ++j) {
+      if (j < nv) {
+        LaneCodes<FMT> c[NM][2];
 #pragma unroll
-        for (int s = 0; s < 4; ++s) mma_16816(d[mm][s], a[s][0], a[s][1], a[s][2], a[s][3], b[s][0], b[s][1]);
+        for (int mm = 0; mm < NM; ++mm)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) load_codes<FMT>(c[mm][h], cbase[mm][h] + (uint32_t)((g0 + j) * BB));
+        const bool on = bg == j;
+#pragma unroll
+        for (int mm = 0; mm < NM; ++mm) {
+          uint32_t a0[4][2], a1[4][2];
+          c[mm][0].frags(a0);
+          c[mm][1].frags(a1);
+#pragma unroll
+          for (int s = 0; s < 4; ++s)
+            mma_16816(d[mm], a0[s][0], a1[s][0], a0[s][1], a1[s][1], on ? xb[2 * s] : 0u, on ? xb[2 * s + 1] : 0u);
+        }
       }
     }
-    // lane group m owns group g0 + m: rows 2t, 2t+1
-    if (m < nv) {
-      const int g = g0 + m;
-      float X;
-      if constexpr (GU) {
-        X = lds32f(asum + 4 * g);
-      } else {
-        const uint4 p0 = lds128(asum + 32 * g), p1 = lds128(asum + 32 * g + 16);
-        X = ((__uint_as_float(p0.x) + __uint_as_float(p0.y)) + (__uint_as_float(p0.z) + __uint_as_float(p0.w))) +
-            ((__uint_as_float(p1.x) + __uint_as_float(p1.y)) + (__uint_as_float(p1.z) + __uint_as_float(p1.w)));
-      }
+    // epilogue: D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]
+    if constexpr (GU) {
 #pragma unroll
-      for (int mm = 0; mm < NM; ++mm) {
-        const uint2 sw = lds64(sbase[mm] + (uint32_t)(g * 32));
-        float D0 = (d[mm][0][0] + d[mm][1][0]) + (d[mm][2][0] + d[mm][3][0]);
-        float D1 = (d[mm][0][1] + d[mm][1][1]) + (d[mm][2][1] + d[mm][3][1]);
-        if constexpr (!GU) {  // rows m + 8 of D: the lo parts of the intermediate
-          D0 += (d[mm][0][2] + d[mm][1][2]) + (d[mm][2][2] + d[mm][3][2]);
-          D1 += (d[mm][0][3] + d[mm][1][3]) + (d[mm][2][3] + d[mm][3][3]);
+      for (int e = 0; e < 2; ++e) {
+        const int n = 2 * t + e;
+        if (n < nv) {
+          const float X = lds32f(bsum + 4u * (uint32_t)(g0 + n));
+#pragma unroll
+          for (int mm = 0; mm < NM; ++mm) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t sw = lds32(sbase[mm][h] + (uint32_t)((g0 + n) * 32));
+              const float sc = __uint_as_float(sw << 16), bi = __uint_as_float(sw & 0xffff0000u);
+              acc[mm][h] = fmaf(sc, d[mm][2 * h + e], fmaf(fmaf(-128.f, sc, bi), X, acc[mm][h]));
+            }
+          }
         }
-        const float s0 = __uint_as_float(sw.x << 16), b0 = __uint_as_float(sw.x & 0xffff0000u);
-        const float s1 = __uint_as_float(sw.y << 16), b1 = __uint_as_float(sw.y & 0xffff0000u);
-        acc[mm][0] = fmaf(s0, D0, fmaf(fmaf(-128.f, s0, b0), X, acc[mm][0]));
-        acc[mm][1] = fmaf(s1, D1, fmaf(fmaf(-128.f, s1, b1), X, acc[mm][1]));
+      }
+    } else {
+      if (t < nv) {
+        const int gq = g0 + t;  // group of columns 2t (hi) and 2t + 1 (lo)
+        const uint4 hs4 = lds128(bsum + 16u * (uint32_t)gq);
+        const float X = (__uint_as_float(hs4.x) + __uint_as_float(hs4.y)) +
+                        (__uint_as_float(hs4.z) + __uint_as_float(hs4.w));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t sw = lds32(sbase[0][h] + (uint32_t)(gq * 32));
+          const float sc = __uint_as_float(sw << 16), bi = __uint_as_float(sw & 0xffff0000u);
+          acc[0][h] = fmaf(sc, d[0][2 * h] + d[0][2 * h + 1], fmaf(fmaf(-128.f, sc, bi), X, acc[0][h]));
+        }
       }
     }
   }
 #pragma unroll
   for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      float v = mm < NM ? acc[mm < NM ? mm : 0][k] : 0.f;
-      v += __shfl_xor_sync(0xffffffffu, v, 4);
-      v += __shfl_xor_sync(0xffffffffu, v, 8);
-      v += __shfl_xor_sync(0xffffffffu, v, 16);
-      res[mm][k] = v;
+    for (int h = 0; h < 2; ++h) {
+      float v = mm < NM ? acc[mm < NM ? mm : 0][h] : 0.f;
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      res[mm][h] = v;
     }
 }
 
-// A routed gate/up unit is done: store its partial sums in accumulator entry
-// e; the warp that completes the row block's last unit sums the units in
-// order, applies SiLU(gate) * up and publishes the 8 intermediate values as
-// hi/lo A fragments of the down projection, with their sum.
-__device__ __noinline__ void gu_unit_done(float r00, float r01, float r10, float r11, int e, int u, int U,
-                                          float* part, int* cnt, int pair, int rb, int I, uint8_t* hf,
-                                          float* hx) {
+// A routed gate/up unit is done: store its partial sums (rows g and g + 8 of
+// the 16-row block, from the lanes with t = 0) in accumulator entry e; the
+// warp that completes the block's last unit sums the units in order, applies
+// SiLU(gate) * up and publishes the 16 intermediate values as bf16 hi and lo
+// B fragments of the down projection (layout [pair][group][hi/lo][t][8
+// words]: rows 16rb .. 16rb + 15 of I are step rb % 4 of group rb / 4), with
+// their sum.
+__device__ __noinline__ void gu_unit_done(float g0r, float g8r, float u0r, float u8r, int e, int u, int U,
+                                          float* part, int* cnt, int pair, int rb, int I, uint8_t* hf, float* hx) {
   const int lane = threadIdx.x & 31;
-  float* pe = part + (size_t)e * kMaxUnits * 16;
-  if (lane < 4) {
-    *reinterpret_cast<float4*>(pe + u * 16 + 4 * lane) = make_float4(r00, r10, r01, r11);
+  float* pe = part + (size_t)e * kMaxUnits * 32;
+  if ((lane & 3) == 0) {
+    const int g = lane >> 2;
+    *reinterpret_cast<float2*>(pe + u * 32 + 2 * g) = make_float2(g0r, u0r);
+    *reinterpret_cast<float2*>(pe + u * 32 + 2 * (g + 8)) = make_float2(g8r, u8r);
     __threadfence_block();
   }
   __syncwarp();
@@ -529,35 +558,40 @@ __device__ __noinline__ void gu_unit_done(float r00, float r01, float r10, float
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return;
   __threadfence_block();
-  // every lane runs the loop (lanes 8..31 repeat rows 0..7 and are dropped),
-  // so the warp does not diverge around it
-  float g = 0.f, up = 0.f;
-  const volatile float* pp = pe + 2 * (lane & 7);
+  // lane v (v = lane % 16; lanes 16..31 repeat rows 0..15 and are dropped)
+  // sums row v over the units in order, so the warp does not diverge
+  const int v = lane & 15;
+  float gs = 0.f, us = 0.f;
+  const volatile float* pp = pe + 2 * v;
 #pragma unroll 1
   for (int uu = 0; uu < U; ++uu) {
-    g += pp[uu * 16];
-    up += pp[uu * 16 + 1];
+    gs += pp[uu * 32];
+    us += pp[uu * 32 + 1];
   }
   if (lane == 0) cnt[e] = 0;  // entry free for a later row block
-  const float h = silu_mul(g, up);
+  const float h = silu_mul(gs, us);
   const __nv_bfloat16 hi = __float2bfloat16_rn(h);
   const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
-  float hsum = lane < 8 ? __bfloat162float(hi) + __bfloat162float(lo) : 0.f;
+  float hsum = lane < 16 ? __bfloat162float(hi) + __bfloat162float(lo) : 0.f;
   hsum += __shfl_xor_sync(0xffffffffu, hsum, 1);
   hsum += __shfl_xor_sync(0xffffffffu, hsum, 2);
   hsum += __shfl_xor_sync(0xffffffffu, hsum, 4);
+  hsum += __shfl_xor_sync(0xffffffffu, hsum, 8);
   const uint32_t hb = __bfloat16_as_ushort(hi), lb = __bfloat16_as_ushort(lo);
-  const int t = lane & 3;
-  const uint32_t h0 = __shfl_sync(0xffffffffu, hb, 2 * t), h1 = __shfl_sync(0xffffffffu, hb, 2 * t + 1);
-  const uint32_t l0 = __shfl_sync(0xffffffffu, lb, 2 * t), l1 = __shfl_sync(0xffffffffu, lb, 2 * t + 1);
-  // rows 8rb..8rb+7 of I: group rb/8, step (rb%8)/2, first or second 8 columns
+  // lane L < 8 builds word (t' = L % 4, first/second = L / 4) of hi and of lo:
+  // values 8*second + 2t' and 8*second + 2t' + 1 of the 16
+  const int tq = lane & 3, sec = (lane >> 2) & 1;
+  const int src = 8 * sec + 2 * tq;
+  const uint32_t h0 = __shfl_sync(0xffffffffu, hb, src), h1 = __shfl_sync(0xffffffffu, hb, src + 1);
+  const uint32_t l0 = __shfl_sync(0xffffffffu, lb, src), l1 = __shfl_sync(0xffffffffu, lb, src + 1);
   const int Gi = I / 64;
-  const int gq = rb >> 3, sq = (rb & 7) >> 1, half = rb & 1;
-  if (lane < 4) {
-    const size_t off = ((((size_t)pair * Gi + gq) * 4 + lane) * 4 + sq) * 16 + half * 8;
-    *reinterpret_cast<uint2*>(hf + off) = make_uint2(h0 | (h1 << 16), l0 | (l1 << 16));
+  const int gq = rb >> 2, sq = rb & 3;
+  if (lane < 8) {
+    uint32_t* base = reinterpret_cast<uint32_t*>(hf) + (((size_t)pair * Gi + gq) * 2) * 32;
+    base[(0 * 4 + tq) * 8 + 2 * sq + sec] = h0 | (h1 << 16);
+    base[(1 * 4 + tq) * 8 + 2 * sq + sec] = l0 | (l1 << 16);
   }
-  if (lane == 0) hx[(size_t)pair * (I / 8) + rb] = hsum;
+  if (lane == 0) hx[(size_t)pair * (I / 16) + rb] = hsum;
 }
 
 // ---- producer ----------------------------------------------------------------------
@@ -669,7 +703,8 @@ __device__ __forceinline__ void emit_routed(Producer& pr, int type, int bits, co
                                          const size_t* off_scales, const uint8_t* blob, int pair, int rb_a,
                                          int rb_b, int nm, RoutedGeo geo, int max_rb, int* rbseq) {
   const uint32_t bb = 64u * (uint32_t)bits;
-  const uint32_t per_unit = (uint32_t)(8 * geo.W) * (uint32_t)nm * (bb + 32u);
+  // both 8-row halves of every group of the unit's windows, codes and scales
+  const uint32_t per_unit = (uint32_t)(geo.gpw * geo.W) * (uint32_t)nm * 2u * (bb + 32u);
   const uint32_t slack = 64;
 #pragma unroll 1
   for (int rb = rb_a; rb < rb_b; ++rb) {
@@ -681,20 +716,21 @@ __device__ __forceinline__ void emit_routed(Producer& pr, int type, int bits, co
         pr.commit();
       if (!pr.open && !pr.begin(type)) return;
       const int un = min(geo.U - u, max(1, (int)((pr.slot_bytes - pr.fill - slack) / per_unit)));
-      const int ga = 8 * geo.W * u, gb = min(geo.G, 8 * geo.W * (u + un));
+      const int ga = geo.gpw * geo.W * u, gb = min(geo.G, geo.gpw * geo.W * (u + un));
       Seg& s = pr.seg(pair, rb, 1);
       s.u0 = u;
       s.u1 = u + un;
       s.gbase = ga;
       s.acc = e;
-      const size_t b0 = (size_t)rb * geo.G + ga;
 #pragma unroll
-      for (int mm = 0; mm < 4; ++mm) {
-        if (mm < 2 * nm) {
-          const bool sc = mm >= nm;
-          const uint32_t per = sc ? 32u : bb;
-          const size_t base = sc ? (mm - nm == 0 ? off_scales[0] : off_scales[1]) : (mm == 0 ? off_codes[0] : off_codes[1]);
-          s.off[mm] = pr.range(blob + base + b0 * per, (size_t)(gb - ga) * per);
+      for (int mm = 0; mm < 2; ++mm) {
+        if (mm < nm) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const size_t b0 = (size_t)(2 * rb + h) * geo.G + ga;
+            s.off[2 * mm + h] = pr.range(blob + off_codes[mm] + b0 * bb, (size_t)(gb - ga) * bb);
+            s.off[2 * nm + 2 * mm + h] = pr.range(blob + off_scales[mm] + b0 * 32u, (size_t)(gb - ga) * 32u);
+          }
         }
       }
       ++pr.nrb_tile;
@@ -719,9 +755,17 @@ __device__ __forceinline__ void emit_rows(Producer& pr, int type, const uint8_t*
   }
 }
 
+// The expert pointer table is staged in shared memory (in the top-K key
+// buffer, which the register top-K for E <= 512 leaves unused) when it is
+// small and 16-byte aligned.
+__device__ __forceinline__ bool ptab_in_smem(const DecodeParams& p) {
+  return p.L.E <= 512 && (p.L.E & 1) == 0 && (reinterpret_cast<uintptr_t>(p.expert_ptr) & 15u) == 0;
+}
+
 template <bool TRACE>
 __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, uint16_t* res_s, uint16_t* gam_s,
-                             uint64_t* xbar, uint64_t* topkbar, const int* flags, const uint8_t* const* eptr) {
+                             uint64_t* xbar, uint64_t* topkbar, const int* flags, const uint8_t* const* eptr,
+                             uint64_t* ptab) {
   const Layout& L = p.L;
   const int T = p.T, K = L.K, H = L.H, I = L.I, E = L.E;
   const int G = gridDim.x, c = blockIdx.x;
@@ -730,8 +774,12 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
   // the token activations, and this block's rows of the residual and of gamma
   const uint32_t xb = (uint32_t)(2ull * T * H);
   const uint32_t rb = (uint32_t)(2 * (r1 - r0));
-  mbar_expect_tx(xbar, xb + (uint32_t)(T + 1) * rb);
+  // the expert pointer table too, when it fits the top-K key buffer (unused
+  // for E <= 512): the routing then finds its blobs without a global round trip
+  const uint32_t tb = ptab_in_smem(p) ? (uint32_t)(8 * E) : 0u;
+  mbar_expect_tx(xbar, xb + (uint32_t)(T + 1) * rb + tb);
   bulk_g2s(xs, p.x, xb, xbar);
+  if (tb) bulk_g2s(ptab, p.expert_ptr, tb, xbar);
   if (rb > 0) {
 #pragma unroll 1
     for (int t = 0; t < T; ++t) bulk_g2s(res_s + (size_t)t * (r1 - r0), p.res + (size_t)t * H + r0, rb, xbar);
@@ -762,10 +810,10 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
     }
   }
   if (pr.trace) pr.trace[9] = globaltimer_ns();
-  const RoutedGeo gh = routed_geo(H), gi = routed_geo(I);
+  const RoutedGeo gh = routed_geo(H, 8), gi = routed_geo(I, 4);
   const size_t oc[3] = {L.off_codes[0], L.off_codes[1], L.off_codes[2]};
   const size_t os[3] = {L.off_scales[0], L.off_scales[1], L.off_scales[2]};
-  const int nrb_i = I / 8;
+  const int nrb_i = I / kRowBlock;
   int rbseq = 0;
   if (routed) {
     // routed gate/up: this block's share of the T*K*(I/8) (pair, row block) items
@@ -790,7 +838,7 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
   if (routed && r1 > r0) {
 #pragma unroll 1
     for (int pair = 0; pair < T * K && pr.ok; ++pair)
-      emit_routed(pr, TILE_EXPERT_DOWN, L.bits, oc + 2, os + 2, eptr[pair], pair, r0 / 8, r1 / 8, 1, gi, 1 << 20,
+      emit_routed(pr, TILE_EXPERT_DOWN, L.bits, oc + 2, os + 2, eptr[pair], pair, r0 / kRowBlock, r1 / kRowBlock, 1, gi, 1 << 20,
                   &rbseq);
   }
   pr.post(F_END);
@@ -878,7 +926,9 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
 #pragma unroll 1
     for (int j = lane; j < T * K; j += 32) {
       const int e = tk_i[j];
-      const void* bp = (e >= 0 && e < E) ? p.expert_ptr[e] : nullptr;
+      const void* bp = (e >= 0 && e < E) ? (ptab_in_smem(p) ? reinterpret_cast<const void*>(tkbuf[e])
+                                                             : p.expert_ptr[e])
+                                         : nullptr;
       if (bp == nullptr || (reinterpret_cast<uintptr_t>(bp) & 255u)) {
         atomicCAS(p.err, 0u, 2u);
         atomicExch(&ctr[5], 1u);
@@ -911,7 +961,7 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
     flags[GO_E] = ge ? 1 : 0;
     if (ge) {
       fence_proxy_async_global();
-      const uint32_t hfb = (uint32_t)(4ull * T * K * L.I), hxb = (uint32_t)(4ull * T * K * (L.I / 8));
+      const uint32_t hfb = (uint32_t)(4ull * T * K * L.I), hxb = (uint32_t)(4ull * T * K * (L.I / 16));
       mbar_expect_tx(&go[GO_E], hfb + hxb);
       bulk_g2s(hf_s, p.hf, hfb, &go[GO_E]);
       bulk_g2s(hx_s, p.hx, hxb, &go[GO_E]);
@@ -951,6 +1001,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   uint4* zero4 = reinterpret_cast<uint4*>(smem + sp.zero);
   float* part = reinterpret_cast<float*>(smem + sp.part);
   int* cnt = reinterpret_cast<int*>(smem + sp.cnt);
+  float* rpart = reinterpret_cast<float*>(smem + sp.rpart);
+  int* rcnt = reinterpret_cast<int*>(smem + sp.rcnt);
   float* tk_w = reinterpret_cast<float*>(smem + sp.tk_w);
   int* tk_i = reinterpret_cast<int*>(smem + sp.tk_i);
   const uint8_t** eptr = reinterpret_cast<const uint8_t**>(smem + sp.eptr);
@@ -985,6 +1037,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     flags[tid] = 0;
   }
   if (tid < kAccSlots) cnt[tid] = 0;
+  if (tid < kSlots * kSplitRows) rcnt[tid] = 0;
   __syncthreads();
 
   if (warp == kProducerWarp) {
@@ -1011,7 +1064,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       pr.d = descs;
       pr.fill = 0;
       pr.policy = l2_policy_evict_first();
-      run_producer<TRACE>(p, pr, xs, res_s, gam_s, xbar, topkbar, flags, eptr);
+      run_producer<TRACE>(p, pr, xs, res_s, gam_s, xbar, topkbar, flags, eptr, tkbuf);
     }
     __syncwarp();
   } else if (warp == kSyncWarp) {
@@ -1022,7 +1075,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     // Every warp walks every tile; the tile's work items (bf16 rows, or units
     // of packed row blocks) are dealt round-robin to the warps, continuing
     // across tiles, and each warp releases a slot on its own.
-    const RoutedGeo gh = routed_geo(H), gi = routed_geo(I);
+    const RoutedGeo gh = routed_geo(H, 8), gi = routed_geo(I, 4);
     bool ok = warp_wait(xbar, 0, p.timeout_ns, spins ? spins + 2 : nullptr);
     bool have_xf = false;
     int item = 0;  // running count of work items over the compute tiles
@@ -1061,7 +1114,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       for (int si = 0; si < d.nseg; ++si) {
         const Seg& sg = d.seg[si];
         const int nu = sg.u1 - sg.u0;
-        const int nitems = routed_tile ? sg.nrows * nu : sg.nrows;
+        // one-token router / shared gate/up rows: nparts column parts per row
+        const bool split = T == 1 && (type == TILE_ROUTER || type == TILE_SHARED_GU) && d.nseg == 1 &&
+                           sg.nrows <= kSplitRows;
+        const int nparts = split ? min(kMaxParts, kConsumerWarps / sg.nrows) : 1;
+        const int nitems = routed_tile ? sg.nrows * nu : sg.nrows * nparts;
         if (work) {
 #pragma unroll 1
           for (int j = (warp - item % kConsumerWarps + kConsumerWarps) % kConsumerWarps; j < nitems;
@@ -1069,17 +1126,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
             if (routed_tile) {
               // ---- one unit of a packed row block: gate/up, or down ----
               const bool gu = type == TILE_EXPERT_GU;
-              const int rbl = j / nu, u = sg.u0 + (j - rbl * nu);
+              const int u = sg.u0 + j;  // a routed segment holds one 16-row block
               const int pb = gu ? 1 : 2;
               if (tid == 0 && !(probed & pb)) trace_mark<TRACE>(p, gu ? 11 : 13);
               float r[2][2];
               const uint64_t tu0 = TRACE ? globaltimer_ns() : 0;
               if (gu)
-                routed_unit<FMT, true>(smem_u32(sl), sg, rbl, u, gh, smem_u32(xf + (size_t)(sg.pair / K) * gh.G * 8),
-                                       smem_u32(xsum + (size_t)(sg.pair / K) * gh.G), smem_u32(zero4), r);
+                routed_unit<FMT, true>(smem_u32(sl), sg, u, gh, smem_u32(xf + (size_t)(sg.pair / K) * gh.G * 8),
+                                       smem_u32(xsum + (size_t)(sg.pair / K) * gh.G), r);
               else
-                routed_unit<FMT, false>(smem_u32(sl), sg, rbl, u, gi, smem_u32(hf_s + (size_t)sg.pair * gi.G * 256),
-                                        smem_u32(hx_s + (size_t)sg.pair * (I / 8)), smem_u32(zero4), r);
+                routed_unit<FMT, false>(smem_u32(sl), sg, u, gi, smem_u32(hf_s + (size_t)sg.pair * gi.G * 256),
+                                        smem_u32(hx_s + (size_t)sg.pair * (I / kRowBlock)), r);
               if (TRACE && tid == 0 && !(probed & pb)) p.trace[(size_t)c * kTraceEntries + (gu ? 100 : 102)] = globaltimer_after(r[0][0]);
               if (TRACE && tid == 0 && nunit < 8) {
                 p.trace[(size_t)c * kTraceEntries + 104 + 2 * nunit] = tu0;
@@ -1087,12 +1144,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
               }
               if (TRACE) ++nunit;
               if (gu) {
-                gu_unit_done(r[0][0], r[0][1], r[1][0], r[1][1], (sg.acc + rbl) % kAccSlots, u, gh.U, part, cnt,
-                             sg.pair, sg.row0 + rbl, I, p.hf, p.hx);
-              } else if (lane < 4) {
-                float* yp = ypart + (size_t)(sg.pair * gi.U + u) * nrows + 8 * (sg.row0 + rbl) + 2 * lane - r0;
-                yp[0] = r[0][0];
-                yp[1] = r[0][1];
+                gu_unit_done(r[0][0], r[0][1], r[1][0], r[1][1], sg.acc, u, gh.U, part, cnt, sg.pair, sg.row0, I,
+                             p.hf, p.hx);
+              } else if ((lane & 3) == 0) {
+                float* yp = ypart + (size_t)(sg.pair * gi.U + u) * nrows + kRowBlock * sg.row0 - r0;
+                yp[lane >> 2] = r[0][0];
+                yp[(lane >> 2) + 8] = r[0][1];
               }
               if (tid == 0 && !(probed & pb)) {
                 trace_mark<TRACE>(p, gu ? 12 : 14);
@@ -1101,6 +1158,52 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
             } else {
               // ---- one bf16 row (the gate/up pair for the shared expert) ----
               const int cols = down ? I : H;
+              if (split) {
+                // part q of row rl: columns [q*chunk, min(cols, (q+1)*chunk))
+                const int rl = j / nparts, q = j - rl * nparts;
+                const int chunk = ((cols + nparts - 1) / nparts + 7) & ~7;
+                const int c0 = min(cols, q * chunk), nc = min(cols, c0 + chunk) - c0;
+                const int row = sg.row0 + rl;
+                const float rbias = (type == TILE_ROUTER && p.bias && q == 0) ? __ldg(p.bias + row) : 0.f;
+                const uint32_t zs = smem_u32(zero4);
+                const uint32_t wa = smem_u32(sl + sg.off[0] + (size_t)rl * 2 * cols + 2 * c0);
+                float v0, v1 = 0.f;
+                if (type == TILE_SHARED_GU) {
+                  float o[2];
+                  row_dot_t1<2, false>(wa, smem_u32(sl + sg.off[1] + (size_t)rl * 2 * cols + 2 * c0),
+                                       smem_u32(xs) + 2u * c0, nc, zs, o);
+                  v0 = o[0];
+                  v1 = warp_sum(o[1]);
+                } else {
+                  float o[1];
+                  row_dot_t1<1, false>(wa, 0u, smem_u32(xs) + 2u * c0, nc, zs, o);
+                  v0 = o[0];
+                }
+                v0 = warp_sum(v0) + rbias;
+                float* rp = rpart + ((size_t)slot * kSplitRows + rl) * kMaxParts * 2;
+                int last = 0;
+                if (lane == 0) {
+                  rp[2 * q] = v0;
+                  rp[2 * q + 1] = v1;
+                  __threadfence_block();
+                  last = atomicAdd(&rcnt[slot * kSplitRows + rl], 1) == nparts - 1 ? 1 : 0;
+                  if (last) {
+                    __threadfence_block();
+                    const volatile float* vp = rp;
+                    float a0 = 0.f, a1 = 0.f;
+                    for (int k = 0; k < nparts; ++k) {
+                      a0 += vp[2 * k];
+                      a1 += vp[2 * k + 1];
+                    }
+                    rcnt[slot * kSplitRows + rl] = 0;
+                    if (type == TILE_ROUTER)
+                      p.logits[row] = a0;
+                    else
+                      p.hs[row] = silu_mul(a0, a1);
+                  }
+                }
+                continue;
+              }
               const uint8_t* w0 = sl + sg.off[0] + (size_t)j * 2 * cols;
               const int row = sg.row0 + j;
               // the router bias is a global load: issue it before the dot
@@ -1350,10 +1453,10 @@ cudaError_t launch_decode(const DecodeParams& p, int grid, size_t smem, cudaStre
 // *nslots, or returns 0 if no ring fits.
 uint32_t decode_slot_bytes(const Layout& L, int T, int nrows_max, int* nslots) {
   const size_t limit = 227 * 1024;
-  const RoutedGeo gh = routed_geo(L.H), gi = routed_geo(L.I);
+  const RoutedGeo gh = routed_geo(L.H, 8), gi = routed_geo(L.I, 4);
   const size_t per_group = 64ull * L.bits + 32;
   const size_t need[5] = {2ull * L.H + 16, 4ull * L.H + 32, 2ull * L.I + 16,
-                          2ull * 8 * gh.W * per_group + 64, 8ull * gi.W * per_group + 64};
+                          2ull * 2 * 8 * gh.W * per_group + 64, 2ull * 4 * gi.W * per_group + 64};
   for (int ns = kSlots; ns >= 2; --ns) {
     const size_t other = decode_smem_plan(T, L.K, L.E, L.H, L.I, nrows_max, ns, 0).total + 1024;
     if (other >= limit) return 0;

@@ -10,28 +10,34 @@
 namespace moe {
 
 // Geometry of the packed rows of one matrix with `cols` input columns, as the
-// tensor-core dot walks it: G groups of 64 columns, nwin windows of 8 groups,
-// W windows per work unit, U units per 8-row block (U <= kMaxUnits).
+// tensor-core dot walks it: the weights are the A operand of m16n8k16 steps
+// (16 rows, two 8-row blocks of the packed layout), and the 8 columns of B
+// carry a "window" of groups: 8 groups of activations for gate/up (gpw = 8),
+// or 4 groups of the intermediate as bf16 hi and lo columns for down
+// (gpw = 4).  G groups of 64 columns, nwin windows, W windows per work unit,
+// U units per 16-row block (U <= kMaxUnits).
 constexpr int kMaxUnits = 8;
+constexpr int kRowBlock = 16;  // rows of one routed work unit (the mma's M)
 struct RoutedGeo {
-  int G, nwin, W, U;
+  int G, gpw, nwin, W, U;
 };
-__host__ __device__ inline RoutedGeo routed_geo(int cols) {
+__host__ __device__ inline RoutedGeo routed_geo(int cols, int gpw) {
   RoutedGeo g;
   g.G = cols / 64;
-  g.nwin = (g.G + 7) / 8;
+  g.gpw = gpw;
+  g.nwin = (g.G + gpw - 1) / gpw;
   g.W = (g.nwin + kMaxUnits - 1) / kMaxUnits;
   g.U = (g.nwin + g.W - 1) / g.W;
   return g;
 }
 
-// Output rows [r0, r1) of block c of G: whole 8-row blocks, spread evenly.
+// Output rows [r0, r1) of block c of G: whole 16-row blocks, spread evenly.
 __host__ __device__ inline void block_rows(int H, int c, int G, int& r0, int& r1) {
-  const uint32_t nrb = (uint32_t)H / 8u;  // nrb * G < 2^32
-  r0 = (int)(8u * (nrb * (uint32_t)c / (uint32_t)G));
-  r1 = (int)(8u * (nrb * (uint32_t)(c + 1) / (uint32_t)G));
+  const uint32_t nrb = (uint32_t)H / 16u;  // nrb * G < 2^32
+  r0 = (int)(16u * (nrb * (uint32_t)c / (uint32_t)G));
+  r1 = (int)(16u * (nrb * (uint32_t)(c + 1) / (uint32_t)G));
 }
-__host__ __device__ inline int decode_rows_max(int H, int G) { return 8 * ((H / 8 + G - 1) / G); }
+__host__ __device__ inline int decode_rows_max(int H, int G) { return 16 * ((H / 16 + G - 1) / G); }
 
 // Workspace of a layer call: counters and error word first, then fp32
 // intermediates.  ctr[0] router, [1] shared gate/up, [2] routed gate/up,
@@ -59,8 +65,8 @@ struct DecodeParams {
   uint32_t* err;
   float* logits;  // [T][E]
   float* hs;      // [T][I]
-  uint8_t* hf;    // routed intermediate as hi/lo bf16 A fragments, 4*T*K*I bytes
-  float* hx;      // [T*K][I/8] sums of hi + lo over 8-row blocks
+  uint8_t* hf;    // routed intermediate as hi/lo bf16 B fragments, 4*T*K*I bytes
+  float* hx;      // [T*K][I/16] sums of hi + lo over 16-row blocks
   float* ss;      // [grid][T] sums of squares of each block's rows of h
   float* hres;    // [T][H] h in fp32, normalised by the last block to finish
   uint64_t timeout_ns;
@@ -86,5 +92,19 @@ cudaError_t launch_topk(const float* logits, int T, int E, int K, int32_t* idx, 
 // Device packer: e_count experts, fp32 weights [e][I][H], [e][I][H], [e][H][I].
 cudaError_t launch_pack(const Layout& L, const float* wg, const float* wu, const float* wd,
                         int e_count, uint8_t* out, cudaStream_t st);
+
+// ---- batched path (moe_grouped.cu) ----
+struct GemmParams;
+size_t grouped_gemm_smem_bytes(int na, bool packed);
+// ak: 0 dense bf16 A, 4 / 2 packed A; na: A matrices (2 = gate and up);
+// epi: 0 fp32 (+ bias), 1 SwiGLU -> fp16, 2 SwiGLU -> bf16 hi and lo.
+cudaError_t launch_grouped_gemm(int ak, int na, int epi, const GemmParams& p, int grid, cudaStream_t st);
+cudaError_t launch_to_half(const uint16_t* x, void* xh, size_t n, uint32_t* abort_flag, cudaStream_t st);
+cudaError_t launch_group(const int32_t* idx, int TK, int E, int K, int* slot_token, int* pair_slot, int* ch_e,
+                         int* ch_c0, int* ch_n, int* n_chunks, const void* const* expert_ptr, uint32_t* err,
+                         cudaStream_t st);
+cudaError_t launch_combine(const float* Y, const float* Ys, const int* pair_slot, const float* w, const uint16_t* res,
+                           const uint16_t* gamma, int T, int H, int K, float eps, uint16_t* h_out, uint16_t* y_norm,
+                           cudaStream_t st);
 
 }  // namespace moe
