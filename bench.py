@@ -58,6 +58,13 @@ def parse_args(argv=None):
     p.add_argument("--stream-slots", type=int, default=512)
     p.add_argument("--stream-steps", type=int, default=64)
     p.add_argument("--stream-warmup", type=int, default=32)
+    p.add_argument("--store", default="pinned", choices=("pinned", "file"),
+                   help="streaming store: pinned host memory, or a file read with parallel pread")
+    p.add_argument("--direct-io", action="store_true", help="file store: O_DIRECT reads (bypass the page cache)")
+    p.add_argument("--store-path", default="/tmp/moe_expert_store.bin")
+    p.add_argument("--predictor", default="next_router", choices=("next_router", "temporal", "none"),
+                   help="streaming prefetch: the next layer's router on this layer's input, the experts the "
+                        "next layer chose for the previous token, or no prefetch")
     p.add_argument("--batched", default="",
                    help="comma-separated token counts: measure batches of T tokens per step instead")
     return p.parse_args(argv)
@@ -450,23 +457,35 @@ def run_ours(args):
     ms_per_step = elapsed_ms / args.steps
     value = units / (elapsed_ms / 1e3)
 
-    # end to end through the host-buffer entry point: H2D of the step's inputs
-    # from pinned memory and D2H of its outputs inside the timed region
+    # end to end through the host-buffer entry points: every step copies its
+    # inputs from pinned host memory and its outputs back (x|residual and
+    # h_out|y_norm adjacent, one copy each way).  Pipelined: the asynchronous
+    # call for every step, one synchronisation at the end (each replica's
+    # workspace and each step's host buffers serve one call in flight).
+    # Blocking: moe_layer_forward_host, which synchronises every step.
     ne = min(args.e2e_steps, P)
-    xh = xs[:ne].cpu().pin_memory()
-    rh = rs[:ne].cpu().pin_memory()
-    hh = torch.empty((T, s.hidden), dtype=torch.int16).pin_memory()
-    yh = torch.empty((T, s.hidden), dtype=torch.int16).pin_memory()
+    inp = torch.stack([xs[:ne], rs[:ne]], dim=1).cpu().pin_memory()  # [ne][2][T][H]
+    out = torch.empty_like(inp).pin_memory()
     for i in range(5):
-        M.moe_layer_forward_host(cfg, reps[i % R]["wts"], xh[i], rh[i], hh, yh, reps[i % R]["ws"], stream=stream)
+        M.moe_layer_forward_host(cfg, reps[i % R]["wts"], inp[i, 0], inp[i, 1], out[i, 0], out[i, 1],
+                                 reps[i % R]["ws"], stream=stream)
+    torch.cuda.synchronize()
     barrier()
     t0 = time.perf_counter()
     for i in range(ne):
         r = reps[i % R]
-        M.moe_layer_forward_host(cfg, r["wts"], xh[i], rh[i], hh, yh, r["ws"], stream=stream)
+        M.moe_layer_forward_host_packed(cfg, r["wts"], inp[i], out[i], r["ws"], stream=stream)
+    stream.synchronize()
     e2e_ms = (time.perf_counter() - t0) * 1e3
     barrier()
+    t0 = time.perf_counter()
+    for i in range(ne):
+        r = reps[i % R]
+        M.moe_layer_forward_host(cfg, r["wts"], inp[i, 0], inp[i, 1], out[i, 0], out[i, 1], r["ws"], stream=stream)
+    e2e_sync_ms = (time.perf_counter() - t0) * 1e3
+    barrier()
     e2e_ms, e2e_units = aggregate(e2e_ms, float(ne * T), "cuda" if world > 1 else None)
+    e2e_sync_ms, _ = aggregate(e2e_sync_ms, float(ne * T), "cuda" if world > 1 else None)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -499,7 +518,11 @@ def run_ours(args):
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": abytes,
                      "kernel": "moe_decode_kernel"},
         "e2e": {"value": e2e_units / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": 2 * T * s.hidden * 2, "d2h_bytes_per_step": 2 * T * s.hidden * 2},
+                "h2d_bytes_per_step": 2 * T * s.hidden * 2, "d2h_bytes_per_step": 2 * T * s.hidden * 2,
+                "api": "moe_layer_forward_host_packed per step (x|residual in, h_out|y_norm out, one copy "
+                       "each way), one synchronisation at the end",
+                "blocking_value": e2e_units / (e2e_sync_ms / 1e3),
+                "blocking_api": "moe_layer_forward_host (synchronises every step)"},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
         "l2_warm_tokens_per_s": (T / (warm * 1e-3)) if warm else None,
@@ -523,16 +546,30 @@ def run_streaming(args):
     prediction), one device-to-host read of both top-K results,
     moe_stream_resolve, moe_layer_forward_routed, and moe_stream_prefetch of
     the predicted experts on a side stream.  The layer output (y_norm, h_out)
-    is the next layer's (x, residual)."""
+    is the next layer's (x, residual).  The link figure is the bytes copied
+    over the time the copies kept the host-to-device link busy (the union of
+    their event-timed intervals), against a 1 GiB pinned copy on the same
+    box.  After timing, a few more tokens are checked: every layer's outputs
+    must equal, bit for bit, the routed call on the same experts copied
+    straight from the store."""
     import torch
     import quantized_expert_ffn_03_b200 as M
 
     torch.cuda.set_device(0)
     s = workload(args.bits)
-    L, NS, E, K = args.stream_layers, args.stream_slots, s.n_experts, s.top_k
+    E, K = s.n_experts, s.top_k
     cfg = M.config(s.hidden, s.inter, E, K, bits=s.bits, eps=s.eps, has_shared=s.has_shared)
     nb = M.moe_packed_expert_bytes(cfg)
-    store = torch.empty((L * E, nb), dtype=torch.uint8).pin_memory()
+    L_req, NS = args.stream_layers, args.stream_slots
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = None
+    L = L_req
+    if avail is not None:
+        L = max(1, min(L_req, int(0.7 * avail) // (E * nb)))
+    store = torch.empty((L * E, nb), dtype=torch.uint8, pin_memory=True)
     chunk = 32
     buf = torch.empty((chunk, nb), dtype=torch.uint8, device="cuda")
     for l in range(L):
@@ -541,6 +578,7 @@ def run_streaming(args):
             M.moe_pack_experts_device(cfg, wg, wu, wd, buf)
             del wg, wu, wd
             store[l * E + e0:l * E + e0 + chunk].copy_(buf)
+    del buf
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
     dense = []
     for l in range(L):
@@ -571,116 +609,229 @@ def run_streaming(args):
     h2d_peak = 3 * (1 << 30) / (e0.elapsed_time(e1) * 1e-3) / 1e9
     del big, bigd
 
-    cache = M.moe_stream_create(cfg, L, store, NS)
+    if args.store == "file":
+        t_w = time.perf_counter()
+        store.numpy().tofile(args.store_path)
+        write_s = time.perf_counter() - t_w
+        cache = M.moe_stream_create_file(cfg, L, args.store_path, NS, direct_io=args.direct_io,
+                                         n_read_threads=2 * K)
+    else:
+        write_s = None
+        cache = M.moe_stream_create(cfg, L, store, NS)
     gen = torch.Generator(device="cuda")
     gen.manual_seed(4321)
     h = torch.empty((1, s.hidden), dtype=torch.int16, device="cuda")
     y = torch.empty_like(h)
 
-    def token(i):
+    pred = args.predictor
+    last_idx = [None] * L  # experts each layer chose for the previous token (temporal predictor)
+
+    def token(record=None):
         x = torch.randn((1, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
         res = torch.randn((1, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
         for l in range(L):
             d = dense[l]
             M.moe_router_topk(cfg, x, d["wr"], d["bias"], idx_d[0], w_d[0], logits_out=lg[0])
-            if l + 1 < L:
+            if pred == "next_router" and l + 1 < L:
                 dn = dense[l + 1]
                 M.moe_router_topk(cfg, x, dn["wr"], dn["bias"], idx_d[1], w_d[1], logits_out=lg[1])
             idx_h.copy_(idx_d.view(2, K), non_blocking=True)
             comp.synchronize()
             M.moe_stream_resolve(cache, l, idx_h[0].numpy(), table)
             M.moe_layer_forward_routed(cfg, wts[l], x, res, idx_d[0], w_d[0], h, y, ws)
+            if record is not None:
+                record.append((l, x.clone(), res.clone(), idx_d[0].clone(), w_d[0].clone(), h.clone(), y.clone()))
             if l + 1 < L:
-                M.moe_stream_prefetch(cache, l + 1, idx_h[1].numpy(), copy_stream=side)
+                if pred == "next_router":
+                    M.moe_stream_prefetch(cache, l + 1, idx_h[1].numpy(), copy_stream=side)
+                elif pred == "temporal" and last_idx[l + 1] is not None:
+                    M.moe_stream_prefetch(cache, l + 1, last_idx[l + 1], copy_stream=side)
+            last_idx[l] = idx_h[0].numpy().copy()
             x, res = y.clone(), h.clone()
 
+    checked, mismatches = 0, 0
     try:
         for i in range(args.stream_warmup):
-            token(i)
+            token()
         torch.cuda.synchronize()
         st0 = M.moe_stream_stats(cache)
+        fs0 = M.moe_stream_file_stats(cache) if args.store == "file" else None
+        M.moe_stream_copy_timing(cache)  # (enables nothing yet: clears)
+        M.moe_stream_enable_copy_timing(cache, True)
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         wall0 = time.perf_counter()
         t0.record()
         for i in range(args.stream_steps):
-            token(args.stream_warmup + i)
+            token()
         t1.record()
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
         ms = t0.elapsed_time(t1)
         st1 = M.moe_stream_stats(cache)
+        fs1 = M.moe_stream_file_stats(cache) if args.store == "file" else None
+        ct = M.moe_stream_copy_timing(cache)
+        M.moe_stream_enable_copy_timing(cache, False)
         err = M.moe_device_error(ws)[0]
+        # check: two more tokens recorded, then each layer recomputed with its
+        # experts copied straight from the host store
+        rec = []
+        for i in range(2):
+            token(rec)
+        torch.cuda.synchronize()
+        tab2 = torch.zeros(E, dtype=torch.int64, device="cuda")
+        ws2 = torch.zeros_like(ws)
+        M.moe_workspace_init(ws2)
+        blobs = torch.empty((K, nb), dtype=torch.uint8, device="cuda")
+        for l, x, res, idd, wdd, hh, yy in rec:
+            ids = idd.cpu().numpy().ravel()
+            for j, e in enumerate(ids):
+                blobs[j].copy_(store[l * E + int(e)])
+            ptrs = tab2.cpu().numpy()
+            for j, e in enumerate(ids):
+                ptrs[int(e)] = blobs[j].data_ptr()
+            tab2.copy_(torch.from_numpy(ptrs))
+            w2 = M.layer_weights(tab2, None, None, dense[l]["sg"], dense[l]["su"], dense[l]["sd"], dense[l]["gamma"])
+            h2, y2 = torch.empty_like(hh), torch.empty_like(yy)
+            M.moe_layer_forward_routed(cfg, w2, x, res, idd, wdd, h2, y2, ws2)
+            torch.cuda.synchronize()
+            checked += 1
+            if not (torch.equal(h2, hh) and torch.equal(y2, yy)):
+                mismatches += 1
+        err = err or M.moe_device_error(ws2)[0]
     finally:
         torch.cuda.synchronize()
         M.moe_stream_destroy(cache)
     dst = {k: st1[k] - st0[k] for k in st1}
     looked = dst["hits"] + dst["misses"]
     secs = ms * 1e-3
+    link = (ct["bytes"] / (ct["busy_ms"] * 1e-3) / 1e9) if ct["busy_ms"] > 0 else None
     line = {
         "metric": "streaming tier: tokens/s through %d layers, experts in pinned host memory" % L,
         "value": args.stream_steps / secs, "unit": "tokens/s", "impl": "ours", "mode": "streaming",
         "n_gpus": 1, "steps": args.stream_steps, "warmup": args.stream_warmup,
         "ms_per_step": ms / args.stream_steps, "higher_is_better": True, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "%s_x%d_layers" % (s.name, L), "layers": L, "slots": NS,
+        "config": {"workload": "%s_x%d_layers" % (s.name, L), "layers": L, "layers_requested": L_req,
+                   "predictor": pred,
+                   "host_available_gb": (avail / 1e9) if avail else None, "slots": NS,
                    "slot_bytes": nb, "host_store_gb": L * E * nb / 1e9, "device_cache_gb": NS * nb / 1e9,
                    "tokens_per_step": 1, "router_bias": "zipf1.1, a different permutation per layer"},
         "hit_rate": dst["hits"] / looked if looked else None,
         "misses_per_token": dst["misses"] / args.stream_steps,
         "prefetches_per_token": dst["prefetches"] / args.stream_steps,
         "prefetch_hits_per_token": dst["prefetch_hits"] / args.stream_steps,
+        "predictor": pred,
+        "prefetch_unused_per_token": (dst["prefetches"] - dst["prefetch_hits"]) / args.stream_steps,
+        "prefetch_precision": (dst["prefetch_hits"] / dst["prefetches"]) if dst["prefetches"] else None,
         "h2d_gb_per_token": dst["bytes_h2d"] / args.stream_steps / 1e9,
         "h2d_gbs_average": dst["bytes_h2d"] / secs / 1e9,
-        "h2d_peak_gbs": h2d_peak,
+        "link": {"gbs_while_copying": link, "peak_gbs": h2d_peak,
+                 "frac": (link / h2d_peak) if link else None, "busy_ms": ct["busy_ms"],
+                 "copy_ms_sum": ct["copy_ms"], "copies": ct["copies"], "bytes": ct["bytes"],
+                 "busy_share_of_step": ct["busy_ms"] / ms if ms > 0 else None},
+        "ms_per_layer": ms / args.stream_steps / L,
         "wall_ms_per_step": wall * 1e3 / args.stream_steps,
+        "checked_layers": checked, "mismatched_layers": mismatches,
         "device_error": err,
     }
+    if args.store == "file":
+        reads = fs1["reads"] - fs0["reads"]
+        rms = fs1["read_ms"] - fs0["read_ms"]
+        rbytes = fs1["read_bytes"] - fs0["read_bytes"]
+        line["config"].update({"store": "file", "direct_io": bool(args.direct_io), "read_threads": 2 * K,
+                               "store_write_s": write_s})
+        line["file_reads"] = {"reads_per_token": reads / args.stream_steps, "read_ms_per_token": rms / args.stream_steps,
+                              "read_ms_per_layer": rms / args.stream_steps / L,
+                              "read_gbs_while_reading": (rbytes / (rms * 1e-3) / 1e9) if rms > 0 else None}
+        try:
+            os.remove(args.store_path)
+        except OSError:
+            pass
     print(json.dumps(line), flush=True)
-    return 0 if err == 0 else 1
+    return 0 if (err == 0 and mismatches == 0) else 1
 
 
 def run_batched(args):
-    """Batches of T tokens per step (one JSON line per T): moe_layer_forward
-    runs the fused kernel on successive chunks of moe_layer_tokens_per_launch
-    tokens, so each chunk reads the experts its tokens chose.  8 replicas round-robin as in
-    the decode measurement; Zipf router bias."""
+    """Batches of T tokens per step, under uniform and Zipf(1.1) routing, each
+    through both forms of the layer: the batched path (grouped dequant GEMMs
+    on the tensor cores, moe_layer_forward_batched) and the fused decode
+    kernel on chunks of moe_layer_tokens_per_launch tokens
+    (moe_layer_forward_chunked).  One JSON line per (routing, T, path), then
+    one line with the measured crossover (the smallest T from which the
+    batched path is faster).  Replicas round-robin as in the decode
+    measurement; the steps of each measurement are captured in a CUDA graph."""
+    import dataclasses
     import torch
     import quantized_expert_ffn_03_b200 as M
 
     torch.cuda.set_device(0)
-    s = workload(args.bits)
-    R = max(1, args.replicas)
-    reps = [build_replica(M, s, rr, 1) for rr in range(R)]
-    cfg = reps[0]["cfg"]
-    ws = torch.zeros(M.moe_layer_workspace_bytes(cfg, 2048), dtype=torch.uint8, device="cuda")
-    M.moe_workspace_init(ws)
+    base = workload(args.bits)
+    R = max(1, min(args.replicas, 4))
+    Ts = [int(v) for v in args.batched.split(",") if v]
     gen = torch.Generator(device="cuda")
     gen.manual_seed(99)
     rc = 0
-    for T in [int(v) for v in args.batched.split(",") if v]:
-        x = torch.randn((T, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
-        r = torch.randn((T, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
-        h, y = torch.empty_like(x), torch.empty_like(x)
-        steps = max(3, min(50, 4096 // T))
-        for i in range(3):
-            M.moe_layer_forward(cfg, reps[i % R]["wts"], x, r, h, y, workspace=ws)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for i in range(steps):
-            M.moe_layer_forward(cfg, reps[i % R]["wts"], x, r, h, y, workspace=ws)
-        e1.record()
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / steps
-        err = M.moe_device_error(ws)[0]
-        rc = rc or (1 if err else 0)
-        line = {"metric": "batched MoE-layer tokens/s (T tokens per step, fused kernel on chunks)",
-                "value": T / (ms * 1e-3), "unit": "tokens/s", "impl": "ours", "mode": "batched", "n_gpus": 1,
-                "steps": steps, "warmup": 3, "ms_per_step": ms, "higher_is_better": True, "dtype": "f32",
-                "data": "synthetic", "config": {"workload": "%s_T%d" % (s.name, T), "tokens_per_step": T,
-                                                "replicas": R, "router_bias": "zipf1.1"},
-                "launches_per_step": -(-T // max(1, M.moe_layer_tokens_per_launch(cfg))), "device_error": err}
-        print(json.dumps(line), flush=True)
+    results = {}
+    for routing in ("uniform", "zipf"):
+        s = dataclasses.replace(base, routing=routing)
+        reps = [build_replica(M, s, rr, 1) for rr in range(R)]
+        cfg = reps[0]["cfg"]
+        nb = max(M.moe_layer_batched_workspace_bytes(cfg, max(Ts)), M.moe_layer_workspace_bytes(cfg, 8))
+        ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        M.moe_workspace_init(ws)
+        stream = torch.cuda.Stream()
+        for T in Ts:
+            x = torch.randn((T, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
+            r = torch.randn((T, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
+            h, y = torch.empty_like(x), torch.empty_like(x)
+            idx = torch.empty((T, s.top_k), dtype=torch.int32, device="cuda")
+            w = torch.empty((T, s.top_k), dtype=torch.float32, device="cuda")
+            for path in ("batched", "chunked"):
+                fn = M.moe_layer_forward_batched if path == "batched" else M.moe_layer_forward_chunked
+                launches = -(-T // max(1, M.moe_layer_tokens_per_launch(cfg)))
+                steps = max(2, min(20, 2048 // T)) if path == "batched" else max(2, min(20, 256 // launches))
+                with torch.cuda.stream(stream):
+                    for i in range(3):
+                        fn(cfg, reps[i % R]["wts"], x, r, h, y, idx, w, workspace=ws, stream=stream)
+                    torch.cuda.synchronize()
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=stream):
+                        for i in range(steps):
+                            fn(cfg, reps[i % R]["wts"], x, r, h, y, idx, w, workspace=ws, stream=stream)
+                    g.replay()
+                    torch.cuda.synchronize()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    g.replay()
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                    del g
+                ms = e0.elapsed_time(e1) / steps
+                err = M.moe_device_error(ws)[0]
+                rc = rc or (1 if err else 0)
+                ic = idx.cpu().numpy()
+                counts = np.bincount(ic.ravel(), minlength=s.n_experts)
+                results[(routing, T, path)] = ms
+                line = {"metric": "batched MoE-layer tokens/s (T tokens per step)", "value": T / (ms * 1e-3),
+                        "unit": "tokens/s", "impl": "ours", "mode": "batched", "path": path, "n_gpus": 1,
+                        "steps": steps, "warmup": 3, "ms_per_step": ms, "higher_is_better": True,
+                        "dtype": "f16 x f16 -> f32 (routed), bf16 (shared, router)" if path == "batched" else "f32",
+                        "data": "synthetic",
+                        "config": {"workload": "%s_T%d_%s" % (s.name, T, routing), "tokens_per_step": T,
+                                   "routing": routing, "replicas": R, "cuda_graph": True},
+                        "experts_used": int((counts > 0).sum()), "max_tokens_per_expert": int(counts.max()),
+                        "expert_bytes_per_step": int((counts > 0).sum()) * M.moe_packed_expert_bytes(cfg),
+                        "launches_per_step": (8 if path == "batched" else launches), "device_error": err}
+                print(json.dumps(line), flush=True)
+    for routing in ("uniform", "zipf"):
+        cross = None
+        for T in Ts:
+            if results[(routing, T, "batched")] < results[(routing, T, "chunked")]:
+                cross = T
+                break
+        print(json.dumps({"metric": "GEMV/GEMM crossover (smallest measured T where the batched path is faster)",
+                          "mode": "batched", "routing": routing, "crossover_tokens": cross, "measured_T": Ts}),
+              flush=True)
     return rc
 
 

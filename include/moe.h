@@ -172,11 +172,12 @@ moe_status moe_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t str
  * x_bf16, residual_bf16 [T][H]; h_out_bf16, y_norm_bf16 [T][H] (y_norm is
  * computed from the fp32 sum, before h_out is rounded to bf16); idx_out
  * int32 [T][K] and w_out fp32 [T][K] may be NULL.  T == 0 is a no-op.
- * One launch of the fused kernel takes C = moe_layer_tokens_per_launch(cfg)
- * tokens; a larger T runs as successive launches of C tokens on the stream
- * (each token's result depends on that token only, so this is exact; each
- * launch reads the experts its tokens chose).  The workspace of any T is
- * that of min(T, 8) tokens.
+ * For T < 32, one launch of the fused kernel takes C =
+ * moe_layer_tokens_per_launch(cfg) tokens and a larger T runs as successive
+ * launches of C tokens on the stream (each token's result depends on that
+ * token only; each launch reads the experts its tokens chose).  From T = 32
+ * the call takes the batched path (moe_layer_forward_batched) when the shape
+ * allows it.  moe_layer_workspace_bytes covers whichever path runs.
  * A bounded device wait that expires leaves MOE_ERR_TIMEOUT in the
  * workspace (moe_device_error). */
 moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts,
@@ -184,6 +185,56 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts
                              void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
                              float* w_out, void* workspace, size_t ws_bytes,
                              cudaStream_t stream);
+
+/* The batched form of the layer (same arguments and results as
+ * moe_layer_forward), for batches where several tokens share an expert:
+ * router logits as a GEMM, top-K, the T*K (token, expert) pairs grouped by
+ * expert, then per chosen expert and chunk of up to 128 of its tokens a
+ * gate/up GEMM and a down GEMM on the tensor cores with the expert's packed
+ * weights dequantised once per chunk (weights and activations of the routed
+ * experts enter as fp16, accumulation in fp32), the shared expert as bf16
+ * GEMMs (its intermediate as bf16 hi + lo), and one combine + residual +
+ * RMSNorm pass.  Workspace: moe_layer_batched_workspace_bytes (grows with T:
+ * about T * K * (2 I + 4 H) bytes).  n_experts <= 2048.  Expert pointers are
+ * checked (non-null, 256-byte aligned) before any is read; a bad one leaves
+ * MOE_ERR_DEVICE in the workspace (moe_device_error) and the outputs
+X
+size_t moe_layer_batched_workspace_bytes(const moe_config* cfg, int T);
+moe_status moe_layer_forward_batched(const moe_config* cfg, const moe_layer_weights* wts,
+                                     const void* x_bf16, const void* residual_bf16, int T,
+                                     void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
+                                     float* w_out, void* workspace, size_t ws_bytes,
+                                     cudaStream_t stream);
+
+/* The layer through the fused decode kernel only, whatever T: successive
+ * launches of moe_layer_tokens_per_launch tokens (each reads the experts its
+ * tokens chose).  Workspace as moe_layer_forward for T < 32. */
+moe_status moe_layer_forward_chunked(const moe_config* cfg, const moe_layer_weights* wts,
+                                     const void* x_bf16, const void* residual_bf16, int T,
+                                     void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
+                                     float* w_out, void* workspace, size_t ws_bytes,
+                                     cudaStream_t stream);
+
+/* The layer with the RMSNorm before it folded in, taking the residual
+ * stream h_in itself (the normalisation that the per-layer GPU command
+ * before the experts runs together with the router and the shared expert,
+ * hakusoku "パイプライン概要"):
+ *   x[t]      = bf16(h_in[t] / sqrt(mean(h_in[t]^2) + eps) * gamma_pre)
+ *   then moe_layer_forward(x, residual = h_in).
+ * gamma_pre bf16 [H] (device); h_in, x_out, h_out, y_norm bf16 [T][H], three
+ * distinct buffers for h_in, x_out and h_out; x_out receives x.  The same eps
+ * as the norm after the layer (cfg->eps).  The sum of squares is taken in
+ * fp32.  For T < 32 tokens that one launch of the fused kernel takes (its
+ * shared-memory plan then also holds gamma_pre; the count is that of
+ * moe_layer_tokens_per_launch at hidden 4096) the norm runs inside that
+ * kernel: its consumer warps normalise x in shared memory before the router
+ * reads it.  Otherwise a norm kernel runs first, then moe_layer_forward.  Workspace,
+ * errors and the remaining arguments as moe_layer_forward. */
+moe_status moe_layer_forward_prenorm(const moe_config* cfg, const moe_layer_weights* wts,
+                                     const void* gamma_pre_bf16, const void* h_in_bf16, int T,
+                                     void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
+                                     float* w_out, void* x_out_bf16, void* workspace, size_t ws_bytes,
+                                     cudaStream_t stream);
 
 /* Tokens one launch of the fused kernel takes for this shape on the current
  * device: the largest T <= min(8, 64 / K) whose shared-memory plan fits
@@ -278,6 +329,24 @@ moe_status moe_layer_forward_host(const moe_config* cfg, const moe_layer_weights
                                   int T, void* h_out_bf16_host, void* y_norm_bf16_host,
                                   void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* The same without the final synchronisation: the copies and the layer are
+ * enqueued on the stream and the call returns.  The host buffers must stay
+ * valid and untouched, and the outputs are ready, only once the stream has
+ * reached the end of the call (synchronise it, or wait on an event recorded
+ * after it); on one stream, successive calls may share a workspace. */
+moe_status moe_layer_forward_host_async(const moe_config* cfg, const moe_layer_weights* wts,
+                                        const void* x_bf16_host, const void* residual_bf16_host,
+                                        int T, void* h_out_bf16_host, void* y_norm_bf16_host,
+                                        void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* The asynchronous host-buffer call with packed host buffers: xr_bf16_host
+ * [2][T][H] holds x then residual, hy_bf16_host [2][T][H] receives h_out then
+ * y_norm, so that each direction is one copy (when T*H*2 is a multiple of 256
+ * bytes; two otherwise).  Same rules as moe_layer_forward_host_async. */
+moe_status moe_layer_forward_host_packed(const moe_config* cfg, const moe_layer_weights* wts,
+                                         const void* xr_bf16_host, int T, void* hy_bf16_host,
+                                         void* workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* ------------------------------------------------------------------------
  * Expert-streaming tier.  The pages keep all experts on SSD and read the 4
  * chosen ones per layer and token (toolarium, section "Mixture of Experts и
@@ -317,6 +386,29 @@ typedef struct moe_stream_cache moe_stream_cache;
 moe_status moe_stream_create(const moe_config* cfg, int n_layers, const void* host_pinned_experts,
                              size_t store_bytes, int n_slots, moe_stream_cache** out);
 
+/* A cache whose store is a file instead of pinned memory: the file at `path`
+ * holds the same n_layers * n_experts blobs ([layer][expert], each
+ * moe_packed_expert_bytes long) -- the pages' own tier: experts on SSD, the
+ * K chosen ones read with parallel pread per layer ("Flash-MoE: чистый C,
+ * Metal и никакого Python", toolarium.ru; hakusoku.com, section
+ * "パイプライン概要").  Every fill of a prefetch or resolve call is read with
+ * pread on a pool of n_read_threads host threads, in parallel, into one of 16
+ * pinned staging buffers, then copied to its slot on the call's stream; the
+ * call returns once its reads are done (the copies are asynchronous).
+ * direct_io = 1 opens the file with O_DIRECT (bypassing the OS page cache;
+ * needs blobs of a multiple of 4096 bytes), 0 reads through the page cache.
+ * A staging buffer is reused once its copy has completed (the host waits
+ * for that).  MOE_ERR_IO if the file cannot be opened or a read fails (the
+ * slot is left empty); MOE_ERR_INVALID_ARG for a file shorter than the blobs
+ * need.  Everything else as moe_stream_create. */
+moe_status moe_stream_create_file(const moe_config* cfg, int n_layers, const char* path, int direct_io,
+                                  int n_slots, int n_read_threads, moe_stream_cache** out);
+
+/* Reads done by a file-backed cache since create: count, bytes and the host
+ * time the calls spent in them (parallel reads of one call count once). */
+moe_status moe_stream_file_stats(const moe_stream_cache* cache, uint64_t* reads, uint64_t* read_bytes,
+                                 double* read_ms);
+
 /* Enqueues on copy_stream the copies of those of expert_ids_host[0..n)
  * (experts of `layer`) that are not resident, each into the least recently
  * used slot that no resolve call holds; the copy waits for the last kernel
@@ -352,6 +444,19 @@ moe_status moe_stream_stats(const moe_stream_cache* cache, moe_stream_counters* 
 /* Waits for the cache's copies and kernels that may still use its slots
  * (synchronises the device), then frees the slots and events. */
 void moe_stream_destroy(moe_stream_cache* cache);
+
+/* Timing of the host-to-device copies (a measurement aid; none on the
+ * pages): once enabled, every copy the cache issues is bracketed by a pair of
+ * CUDA events on its stream.  moe_stream_copy_timing waits for the timed
+ * copies, returns the time the link was busy with them (the union of their
+ * intervals; copies on the prefetch and compute streams may overlap), the
+ * sum of their durations, their count and bytes, and starts over. */
+typedef struct {
+  double busy_ms, copy_ms;
+  uint64_t copies, bytes;
+} moe_stream_copy_times;
+moe_status moe_stream_enable_copy_timing(moe_stream_cache* cache, int on);
+moe_status moe_stream_copy_timing(moe_stream_cache* cache, moe_stream_copy_times* out);
 
 /* Host-side fault injection for tests of the streaming tier's error paths
  * (no counterpart on the pages; nothing is done to the GPU):

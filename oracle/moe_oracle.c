@@ -422,6 +422,48 @@ void orc_shared_ffn(const orc_cfg* c, const uint16_t* wg, const uint16_t* wu,
   free(a);
 }
 
+/* ---- RMSNorm before the layer --------------------------------------------- */
+
+/* x = h / sqrt(mean(h^2) + eps) * gamma_pre, per token: the normalisation that
+ * the GPU command before the experts runs together with the router and the
+ * shared expert ([hakusoku] "パイプライン概要").  The layer then takes x rounded
+ * to bf16 as its input and h itself as the residual. */
+void orc_prenorm(const orc_cfg* c, const uint16_t* h_bf16, const uint16_t* gamma_bf16, int T,
+                 double* x) {
+  int H = c->hidden;
+  for (int t = 0; t < T; ++t) {
+    double ss = 0.0;
+    for (int r = 0; r < H; ++r) {
+      double v = orc_bf16_to_f64(h_bf16[(size_t)t * H + r]);
+      ss += v * v;
+    }
+    double inv = ORC_MUTANT == 13 ? 1.0 / sqrt(ss + (double)c->eps) : 1.0 / sqrt(ss / H + (double)c->eps);
+    for (int r = 0; r < H; ++r) {
+      double g = ORC_MUTANT == 14 ? 1.0 : orc_bf16_to_f64(gamma_bf16[r]);
+      x[(size_t)t * H + r] = orc_bf16_to_f64(h_bf16[(size_t)t * H + r]) * inv * g;
+    }
+  }
+}
+
+/* Round a double to bf16, to nearest with ties to even, in one step (no
+ * intermediate float).  Finite inputs only. */
+uint16_t orc_f64_to_bf16(double v) {
+  if (v == 0.0) return signbit(v) ? 0x8000u : 0u;
+  int e;
+  (void)frexp(fabs(v), &e); /* |v| = m * 2^e, m in [0.5, 1) */
+  /* bf16 keeps 8 significant bits: units of 2^(e-8) for normal results */
+  int ue = e - 8;
+  if (ue < -133) ue = -133; /* subnormal bf16: units of 2^-133 */
+  double q = ldexp(fabs(v), -ue);
+  double fl = floor(q), fr = q - fl;
+  if (fr > 0.5 || (fr == 0.5 && fmod(fl, 2.0) != 0.0)) fl += 1.0;
+  float f = (float)ldexp(fl, ue); /* exact: at most 9 significant bits */
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  if (v < 0) u |= 0x80000000u;
+  return (uint16_t)(u >> 16);
+}
+
 /* ---- whole layer ---------------------------------------------------------- */
 
 /* h_out = residual + sum_k w_k * expert_{idx_k}(x) + shared(x);

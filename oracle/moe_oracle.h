@@ -65,6 +65,12 @@ void orc_section_offsets(const orc_cfg* c, size_t off[6]);
 /* bf16 helpers (round to nearest even; NaN stays NaN). */
 uint16_t orc_f32_to_bf16(float f);
 double orc_bf16_to_f64(uint16_t h);
+/* Double to bf16 in one rounding (nearest, ties to even; finite inputs). */
+uint16_t orc_f64_to_bf16(double v);
+/* RMSNorm before the layer: x[t] = h[t] / sqrt(mean(h[t]^2) + eps) * gamma_pre,
+ * h and gamma bf16, x double [T][H]. */
+void orc_prenorm(const orc_cfg* c, const uint16_t* h_bf16, const uint16_t* gamma_bf16, int T,
+                 double* x);
 
 /* Quantise one expert from float weights w_gate [I][H], w_up [I][H],
  * w_down [H][I] into blob (orc_expert_bytes bytes, zero padding).  Returns 0. */

@@ -48,6 +48,9 @@ def lib(path=None):
         _lib.orc_f32_to_bf16.argtypes = [C.c_float]
         _lib.orc_bf16_to_f64.restype = C.c_double
         _lib.orc_bf16_to_f64.argtypes = [C.c_uint16]
+        _lib.orc_f64_to_bf16.restype = C.c_uint16
+        _lib.orc_f64_to_bf16.argtypes = [C.c_double]
+        _lib.orc_prenorm.argtypes = [cfgp, P, P, C.c_int, P]
         _lib.orc_quantize_expert.restype = C.c_int
         _lib.orc_quantize_expert.argtypes = [cfgp, P, P, P, P]
         _lib.orc_dequant.restype = C.c_double
@@ -92,6 +95,23 @@ def f32_to_bf16(a):
     a = np.asarray(a, dtype=np.float32)
     f = lib().orc_f32_to_bf16
     return np.array([f(float(v)) for v in a.ravel()], dtype=np.uint16).reshape(a.shape)
+
+
+def f64_to_bf16(a):
+    a = np.asarray(a, dtype=np.float64)
+    f = lib().orc_f64_to_bf16
+    return np.array([f(float(v)) for v in a.ravel()], dtype=np.uint16).reshape(a.shape)
+
+
+def prenorm(c, h_bf16, gamma_bf16):
+    """x = h / sqrt(mean(h^2) + eps) * gamma per token, in double [T][H]."""
+    h = _c(h_bf16, np.uint16)
+    g = _c(gamma_bf16, np.uint16)
+    T = h.shape[0]
+    assert h.shape == (T, c.hidden) and g.shape == (c.hidden,)
+    out = np.zeros((T, c.hidden), dtype=np.float64)
+    lib().orc_prenorm(C.byref(c), _p(h), _p(g), T, _p(out))
+    return out
 
 
 def bf16_to_f64(a):
@@ -197,3 +217,12 @@ def layer_forward(c, experts, wr, bias, shared_gate, shared_up, shared_down, gam
                             _p(x), _p(_c(residual, np.uint16)), T, _p(ii), _p(wi),
                             _p(idx), _p(w), _p(h), _p(yn))
     return idx, w, h, yn
+
+
+def layer_forward_prenorm(c, experts, wr, bias, shared_gate, shared_up, shared_down, gamma,
+                          gamma_pre, h_in):
+    """The layer with the RMSNorm before it: x = bf16(prenorm(h_in)), then
+    the layer on x with h_in as the residual.  Returns (x_bf16, idx, w, h, y)."""
+    x = f64_to_bf16(prenorm(c, h_in, gamma_pre))
+    return (x,) + tuple(layer_forward(c, experts, wr, bias, shared_gate, shared_up, shared_down,
+                                      gamma, x, h_in))

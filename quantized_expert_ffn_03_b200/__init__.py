@@ -70,6 +70,10 @@ EXPORTS = {
     "moe_layer_host_workspace_bytes": (C.c_size_t, [C.c_void_p, C.c_int]),
     "moe_layer_forward_host": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                          C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "moe_layer_forward_host_async": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                               C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "moe_layer_forward_host_packed": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p,
+                                                C.c_void_p, C.c_size_t, C.c_void_p]),
     "moe_layer_trace_blocks": (C.c_int, []),
     "moe_layer_forward_traced": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p,
@@ -77,11 +81,26 @@ EXPORTS = {
     "moe_layer_forward_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                             C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "moe_layer_tokens_per_launch": (C.c_int, [C.c_void_p]),
+    "moe_layer_batched_workspace_bytes": (C.c_size_t, [C.c_void_p, C.c_int]),
+    "moe_layer_forward_batched": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                            C.c_size_t, C.c_void_p]),
+    "moe_layer_forward_chunked": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                            C.c_size_t, C.c_void_p]),
+    "moe_layer_forward_prenorm": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                            C.c_void_p, C.c_size_t, C.c_void_p]),
     "moe_layer_forward_routed": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                            C.c_size_t, C.c_void_p]),
     "moe_stream_create": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_size_t, C.c_int, C.c_void_p]),
     "moe_stream_inject_fault": (C.c_int, [C.c_void_p, C.c_int, C.c_int]),
+    "moe_stream_create_file": (C.c_int, [C.c_void_p, C.c_int, C.c_char_p, C.c_int, C.c_int, C.c_int,
+                                         C.c_void_p]),
+    "moe_stream_file_stats": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "moe_stream_enable_copy_timing": (C.c_int, [C.c_void_p, C.c_int]),
+    "moe_stream_copy_timing": (C.c_int, [C.c_void_p, C.c_void_p]),
     "moe_stream_prefetch": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p]),
     "moe_stream_resolve": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
     "moe_stream_stats": (C.c_int, [C.c_void_p, C.c_void_p]),
@@ -234,6 +253,38 @@ def moe_layer_tokens_per_launch(cfg):
     return _lib.moe_layer_tokens_per_launch(C.byref(cfg))
 
 
+def moe_layer_batched_workspace_bytes(cfg, T):
+    return _lib.moe_layer_batched_workspace_bytes(C.byref(cfg), int(T))
+
+
+def moe_layer_forward_batched(cfg, wts, x, residual, h_out, y_norm, idx_out=None, w_out=None,
+                              workspace=None, stream=None):
+    """The layer through the grouped tensor-core GEMMs (see moe.h)."""
+    T = x.shape[0]
+    _check(_lib.moe_layer_forward_batched(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T, _ptr(h_out),
+                                          _ptr(y_norm), _ptr(idx_out), _ptr(w_out), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_layer_forward_chunked(cfg, wts, x, residual, h_out, y_norm, idx_out=None, w_out=None,
+                              workspace=None, stream=None):
+    """The layer through the fused decode kernel on chunks of tokens (see moe.h)."""
+    T = x.shape[0]
+    _check(_lib.moe_layer_forward_chunked(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T, _ptr(h_out),
+                                          _ptr(y_norm), _ptr(idx_out), _ptr(w_out), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_layer_forward_prenorm(cfg, wts, gamma_pre, h_in, h_out, y_norm, x_out, idx_out=None, w_out=None,
+                              workspace=None, stream=None):
+    """The layer with the RMSNorm before it, on the residual stream h_in (see moe.h)."""
+    T = h_in.shape[0]
+    _check(_lib.moe_layer_forward_prenorm(C.byref(cfg), C.byref(wts), _ptr(gamma_pre), _ptr(h_in), T,
+                                          _ptr(h_out), _ptr(y_norm), _ptr(idx_out), _ptr(w_out), _ptr(x_out),
+                                          _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                          _stream(stream)))
+
+
 def moe_layer_forward_routed(cfg, wts, x, residual, idx, w, h_out, y_norm, workspace, stream=None):
     """The layer with the routing given: idx int32 [T][K], w float32 [T][K] (CUDA)."""
     T = x.shape[0]
@@ -270,6 +321,22 @@ def moe_layer_forward_host(cfg, wts, x, residual, h_out, y_norm, workspace, stre
                                        workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def moe_layer_forward_host_async(cfg, wts, x, residual, h_out, y_norm, workspace, stream=None):
+    """moe_layer_forward_host without the final synchronisation (see moe.h)."""
+    T = x.shape[0]
+    _check(_lib.moe_layer_forward_host_async(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T,
+                                             _ptr(h_out), _ptr(y_norm), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_layer_forward_host_packed(cfg, wts, xr, hy, workspace, stream=None):
+    """xr: pinned host [2][T][H] (x, residual); hy: pinned host [2][T][H]
+    (h_out, y_norm), filled once the stream reaches the end of the call."""
+    T = xr.shape[1]
+    _check(_lib.moe_layer_forward_host_packed(C.byref(cfg), C.byref(wts), _ptr(xr), T, _ptr(hy), _ptr(workspace),
+                                              workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 # ---- expert-streaming tier -------------------------------------------------------
 
 class MoeStreamCounters(C.Structure):
@@ -287,6 +354,21 @@ def moe_stream_create(cfg, n_layers, host_store, n_slots, store_bytes=None):
     _check(_lib.moe_stream_create(C.byref(cfg), int(n_layers), _ptr(host_store), int(store_bytes), int(n_slots),
                                   C.byref(h)))
     return h.value
+
+
+def moe_stream_create_file(cfg, n_layers, path, n_slots, direct_io=False, n_read_threads=4):
+    """A cache whose store is a file of n_layers*E packed blobs (see moe.h).
+    Returns the cache handle (an int)."""
+    h = C.c_void_p(0)
+    _check(_lib.moe_stream_create_file(C.byref(cfg), int(n_layers), os.fsencode(path), 1 if direct_io else 0,
+                                       int(n_slots), int(n_read_threads), C.byref(h)))
+    return h.value
+
+
+def moe_stream_file_stats(cache):
+    reads, nbytes, ms = C.c_uint64(0), C.c_uint64(0), C.c_double(0.0)
+    _check(_lib.moe_stream_file_stats(cache, C.byref(reads), C.byref(nbytes), C.byref(ms)))
+    return {"reads": int(reads.value), "read_bytes": int(nbytes.value), "read_ms": float(ms.value)}
 
 
 MOE_FAULT_NONE, MOE_FAULT_COPY, MOE_FAULT_ALLOC = 0, 1, 2
@@ -316,6 +398,21 @@ def moe_stream_stats(cache):
     out = MoeStreamCounters()
     _check(_lib.moe_stream_stats(cache, C.byref(out)))
     return {f: int(getattr(out, f)) for f, _ in MoeStreamCounters._fields_}
+
+
+class MoeStreamCopyTimes(C.Structure):
+    _fields_ = [("busy_ms", C.c_double), ("copy_ms", C.c_double), ("copies", C.c_uint64), ("bytes", C.c_uint64)]
+
+
+def moe_stream_enable_copy_timing(cache, on=True):
+    _check(_lib.moe_stream_enable_copy_timing(cache, 1 if on else 0))
+
+
+def moe_stream_copy_timing(cache):
+    out = MoeStreamCopyTimes()
+    _check(_lib.moe_stream_copy_timing(cache, C.byref(out)))
+    return {f: (float(getattr(out, f)) if f.endswith("_ms") else int(getattr(out, f)))
+            for f, _ in MoeStreamCopyTimes._fields_}
 
 
 def moe_stream_destroy(cache):

@@ -14,8 +14,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe.so")
-SOURCES = ["moe_abi.cu", "moe_decode.cu", "moe_router.cu", "moe_pack.cu", "moe_noalloc.cu", "moe_stream.cu"]
-HEADERS = ["moe_device.cuh", "moe_kernels.h", "moe_layout.h", "moe_stream_policy.h"]
+SOURCES = ["moe_abi.cu", "moe_decode.cu", "moe_router.cu", "moe_pack.cu", "moe_noalloc.cu", "moe_stream.cu",
+           "moe_grouped.cu"]
+HEADERS = ["moe_device.cuh", "moe_kernels.h", "moe_layout.h", "moe_stream_policy.h", "moe_tc.cuh", "moe_grouped.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

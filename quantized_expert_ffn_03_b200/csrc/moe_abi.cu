@@ -9,6 +9,7 @@
 #include <string>
 
 #include "../../include/moe.h"
+#include "moe_grouped.h"
 #include "moe_kernels.h"
 
 namespace moe {
@@ -96,7 +97,7 @@ moe_status device_info(DeviceInfo* out) {
 }
 
 struct WsPlan {
-  size_t logits, hs, hf, hx, ss, hres, total;
+  size_t logits, hs, hf, hx, ss, total;
 };
 
 // Tokens per launch of the fused kernel: at most kMaxTokensFused, and at
@@ -116,24 +117,78 @@ int tokens_per_launch(const Layout& L, int grid, int max_tokens) {
   return 0;
 }
 
+// The fused kernel publishes its router logits and sums of squares as 64-bit
+// words tagged with the launch's epoch.  Their region follows the 256-byte
+// header in every plan (fused and batched), so no other data of either path
+// is ever written where a later launch looks for its epoch words.
+size_t epoch_region_bytes(const Layout& L) {
+  const size_t C = (size_t)chunk_tokens(L);
+  return round_up_256(sizeof(uint64_t) * C * L.E) + round_up_256(sizeof(uint64_t) * C * kMaxGrid);
+}
+
 WsPlan ws_plan(const Layout& L, int T) {
   WsPlan w;
+  const size_t C = (size_t)chunk_tokens(L);
   size_t pos = 256;
   w.logits = pos;
-  pos = round_up_256(pos + sizeof(float) * (size_t)T * L.E);
+  w.ss = round_up_256(pos + sizeof(uint64_t) * C * L.E);
+  pos = 256 + epoch_region_bytes(L);
   w.hs = pos;
   pos = round_up_256(pos + sizeof(float) * (size_t)T * L.I);
   w.hf = pos;
   pos = round_up_256(pos + 4ull * (size_t)T * L.K * L.I);
   w.hx = pos;
-  pos = round_up_256(pos + sizeof(float) * (size_t)T * L.K * (L.I / 8));
-  w.ss = pos;
-  pos = round_up_256(pos + sizeof(float) * (size_t)T * kMaxGrid);
-  w.hres = pos;
-  pos = round_up_256(pos + sizeof(float) * (size_t)T * L.H);
+  pos = round_up_256(pos + sizeof(float) * (size_t)T * L.K * (L.I / 16));
   w.total = pos;
   return w;
 }
+
+// Workspace of the batched path for T tokens: the 256-byte header (error
+// word, abort flag), then x as fp16, router logits, routing, the grouping
+// (slot -> token, pair -> slot, chunk lists), the routed intermediate (fp16
+// [slot][I]), the routed outputs (fp32 [slot][H]), the shared intermediate
+// (bf16 hi and lo [T][I]) and the shared output (fp32 [T][H]).
+struct BatchPlan {
+  size_t xh, logits, idx, w, slot_token, pair_slot, ch_e, ch_c0, ch_n, nch, hr, y, hs_hi, hs_lo, ys, total;
+  int max_chunks;
+};
+
+constexpr int kBatchedMaxExperts = 2048;
+
+BatchPlan batch_plan(const Layout& L, int T) {
+  BatchPlan b;
+  const size_t TK = (size_t)T * L.K;
+  b.max_chunks = (int)(TK / 128 + (size_t)L.E + 1);
+  size_t pos = 256 + epoch_region_bytes(L);
+  auto take = [&](size_t bytes) {
+    const size_t at = pos;
+    pos = round_up_256(pos + bytes);
+    return at;
+  };
+  b.xh = take(2ull * T * L.H);
+  b.logits = take(4ull * T * L.E);
+  b.idx = take(4 * TK);
+  b.w = take(4 * TK);
+  b.slot_token = take(4 * TK);
+  b.pair_slot = take(4 * TK);
+  b.ch_e = take(4ull * b.max_chunks);
+  b.ch_c0 = take(4ull * b.max_chunks);
+  b.ch_n = take(4ull * b.max_chunks);
+  b.nch = take(16);
+  b.hr = take(2 * TK * L.I);
+  b.y = take(4 * TK * L.H);
+  b.hs_hi = take(2ull * T * L.I);
+  b.hs_lo = take(2ull * T * L.I);
+  b.ys = take(4ull * T * L.H);
+  b.total = pos;
+  return b;
+}
+
+// Tokens from which moe_layer_forward takes the batched path instead of the
+// fused decode kernel on chunks of tokens.
+constexpr int kBatchedMinTokens = 32;
+
+bool batched_ok(const Layout& L) { return L.E <= kBatchedMaxExperts; }
 
 }  // namespace
 
@@ -241,7 +296,21 @@ size_t moe_layer_workspace_bytes(const moe_config* cfg, int T) {
   if (!make_layout(cfg->hidden, cfg->inter, cfg->n_experts, cfg->top_k, cfg->bits, cfg->group,
                    cfg->has_shared, cfg->eps, &L))
     return 0;
-  return ws_plan(L, T < chunk_tokens(L) ? T : chunk_tokens(L)).total;
+  const size_t fused = ws_plan(L, T < chunk_tokens(L) ? T : chunk_tokens(L)).total;
+  if (T >= kBatchedMinTokens && batched_ok(L)) {
+    const size_t b = batch_plan(L, T).total;
+    return b > fused ? b : fused;
+  }
+  return fused;
+}
+
+size_t moe_layer_batched_workspace_bytes(const moe_config* cfg, int T) {
+  Layout L;
+  if (!cfg || T < 0 || cfg->n_experts <= 0 || cfg->top_k <= 0) return 0;
+  if (!make_layout(cfg->hidden, cfg->inter, cfg->n_experts, cfg->top_k, cfg->bits, cfg->group,
+                   cfg->has_shared, cfg->eps, &L) || !batched_ok(L))
+    return 0;
+  return batch_plan(L, T).total;
 }
 
 moe_status moe_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t stream) {
@@ -257,11 +326,15 @@ static moe_status layer_forward_chunk(const moe_config* cfg, const moe_layer_wei
                                       void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
                                       float* w_out, void* workspace, size_t ws_bytes,
                                       void* trace, size_t trace_entries, cudaStream_t stream,
-                                      const int32_t* idx_in, const float* w_in) {
+                                      const int32_t* idx_in, const float* w_in, const void* gamma_pre = nullptr,
+                                      void* x_out = nullptr) {
   Layout L;
   moe_status s = check_cfg(cfg, &L);
   if (s != MOE_OK) return s;
+  L.prenorm = gamma_pre ? 1 : 0;
   if (T > chunk_tokens(L)) return fail(MOE_ERR_UNSUPPORTED, "T=%d: at most %d tokens per launch", T, chunk_tokens(L));
+  if (!aligned(gamma_pre, 16) || !aligned(x_out, 16))
+    return fail(MOE_ERR_INVALID_ARG, "bf16 arrays must be 16-byte aligned");
   const bool given = idx_in != nullptr;  // routing given: the router weights are not read
   if (given && !w_in) return fail(MOE_ERR_INVALID_ARG, "NULL routing weights");
   if (!wts || !wts->expert_ptr || (!given && !wts->router_w) || !wts->gamma || !x_bf16 || !residual_bf16 ||
@@ -301,6 +374,8 @@ static moe_status layer_forward_chunk(const moe_config* cfg, const moe_layer_wei
   p.su = static_cast<const uint16_t*>(wts->shared_up);
   p.sd = static_cast<const uint16_t*>(wts->shared_down);
   p.gamma = static_cast<const uint16_t*>(wts->gamma);
+  p.gamma_pre = static_cast<const uint16_t*>(gamma_pre);
+  p.x_out = static_cast<uint16_t*>(x_out);
   p.x = static_cast<const uint16_t*>(x_bf16);
   p.res = static_cast<const uint16_t*>(residual_bf16);
   p.h_out = static_cast<uint16_t*>(h_out_bf16);
@@ -311,12 +386,11 @@ static moe_status layer_forward_chunk(const moe_config* cfg, const moe_layer_wei
   p.w_in = w_in;
   p.ctr = reinterpret_cast<uint32_t*>(ws);
   p.err = reinterpret_cast<uint32_t*>(ws + 64);
-  p.logits = reinterpret_cast<float*>(ws + wp.logits);
+  p.logits = reinterpret_cast<uint64_t*>(ws + wp.logits);
   p.hs = reinterpret_cast<float*>(ws + wp.hs);
   p.hf = ws + wp.hf;
   p.hx = reinterpret_cast<float*>(ws + wp.hx);
-  p.ss = reinterpret_cast<float*>(ws + wp.ss);
-  p.hres = reinterpret_cast<float*>(ws + wp.hres);
+  p.ss = reinterpret_cast<uint64_t*>(ws + wp.ss);
   if (trace && trace_entries < (size_t)grid * 128)
     return fail(MOE_ERR_INVALID_ARG, "trace needs %d entries", grid * 128);
   p.timeout_ns = kTimeoutNs;
@@ -324,6 +398,141 @@ static moe_status layer_forward_chunk(const moe_config* cfg, const moe_layer_wei
   p.nslots = nslots;
   p.trace = static_cast<uint64_t*>(trace);
   CUDA_TRY(launch_decode(p, grid, smem, stream));
+  return ok();
+}
+
+// The batched path (moe_grouped.cu): router GEMM, top-K, grouping by
+// expert, grouped GEMMs for the routed experts, GEMMs for the shared expert,
+// combine + residual + RMSNorm.
+static moe_status layer_forward_batched(const moe_config* cfg, const moe_layer_weights* wts, const void* x_bf16,
+                                        const void* residual_bf16, int T, void* h_out_bf16, void* y_norm_bf16,
+                                        int32_t* idx_out, float* w_out, void* workspace, size_t ws_bytes,
+                                        cudaStream_t stream) {
+  Layout L;
+  moe_status s = check_cfg(cfg, &L);
+  if (s != MOE_OK) return s;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+  if (T == 0) return ok();
+  if (!batched_ok(L)) return fail(MOE_ERR_UNSUPPORTED, "the batched path takes at most %d experts", kBatchedMaxExperts);
+  if (!wts || !wts->expert_ptr || !wts->router_w || !wts->gamma || !x_bf16 || !residual_bf16 || !h_out_bf16 ||
+      !y_norm_bf16)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (L.has_shared && (!wts->shared_gate || !wts->shared_up || !wts->shared_down))
+    return fail(MOE_ERR_INVALID_ARG, "has_shared=1 but a shared-expert pointer is NULL");
+  const void* a16[] = {x_bf16, residual_bf16, h_out_bf16, y_norm_bf16, wts->router_w, wts->gamma,
+                       L.has_shared ? wts->shared_gate : nullptr, L.has_shared ? wts->shared_up : nullptr,
+                       L.has_shared ? wts->shared_down : nullptr};
+  for (const void* q : a16)
+    if (!aligned(q, 16)) return fail(MOE_ERR_INVALID_ARG, "bf16 arrays must be 16-byte aligned");
+  const BatchPlan bp = batch_plan(L, T);
+  if (!workspace || ws_bytes < bp.total || !aligned(workspace, 256))
+    return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned and >= %zu bytes", bp.total);
+  DeviceInfo di;
+  if ((s = device_info(&di)) != MOE_OK) return s;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws + 64);
+  uint32_t* abort_flag = reinterpret_cast<uint32_t*>(ws) + 5;
+  const int TK = T * L.K;
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + bp.idx);
+  float* w = w_out ? w_out : reinterpret_cast<float*>(ws + bp.w);
+  float* logits = reinterpret_cast<float*>(ws + bp.logits);
+  int* slot_token = reinterpret_cast<int*>(ws + bp.slot_token);
+  int* pair_slot = reinterpret_cast<int*>(ws + bp.pair_slot);
+  int* ch_e = reinterpret_cast<int*>(ws + bp.ch_e);
+  int* ch_c0 = reinterpret_cast<int*>(ws + bp.ch_c0);
+  int* ch_n = reinterpret_cast<int*>(ws + bp.ch_n);
+  int* nch = reinterpret_cast<int*>(ws + bp.nch);
+  const int grid = di.sms;
+  auto tiles = [](int cols, int M) { return ((cols + 127) / 128) * ((M + 127) / 128); };
+
+  CUDA_TRY(launch_to_half(x, ws + bp.xh, (size_t)T * L.H, abort_flag, stream));
+  // router logits (bf16 GEMM, bias in the epilogue), top-K
+  GemmParams g = {};
+  g.err = err;
+  g.abort_flag = abort_flag;
+  g.timeout_ns = kTimeoutNs;
+  {
+    GemmParams r = g;
+    r.M = L.E;
+    r.K = L.H;
+    r.a_dense[0] = static_cast<const uint16_t*>(wts->router_w);
+    r.b = x;
+    r.n_cols = T;
+    r.out = logits;
+    r.bias = wts->router_bias;
+    const int gr = tiles(T, L.E) < grid ? tiles(T, L.E) : grid;
+    CUDA_TRY(launch_grouped_gemm(0, 1, 0, r, gr, stream));
+  }
+  CUDA_TRY(launch_topk(logits, T, L.E, L.K, idx, w, stream));
+  CUDA_TRY(launch_group(idx, TK, L.E, L.K, slot_token, pair_slot, ch_e, ch_c0, ch_n, nch, wts->expert_ptr, err,
+                        stream));
+  // routed gate/up: dequantised weights x the chunk's tokens (fp16), SwiGLU -> hr
+  {
+    GemmParams r = g;
+    r.M = L.I;
+    r.K = L.H;
+    r.bits = L.bits;
+    r.expert_ptr = wts->expert_ptr;
+    r.off_codes[0] = L.off_codes[0];
+    r.off_codes[1] = L.off_codes[1];
+    r.off_scales[0] = L.off_scales[0];
+    r.off_scales[1] = L.off_scales[1];
+    r.b = reinterpret_cast<const uint16_t*>(ws + bp.xh);
+    r.b_rows = slot_token;
+    r.ch_e = ch_e;
+    r.ch_c0 = ch_c0;
+    r.ch_n = ch_n;
+    r.n_chunks_dev = nch;
+    r.out = ws + bp.hr;
+    CUDA_TRY(launch_grouped_gemm(L.bits, 2, 1, r, grid, stream));
+  }
+  // routed down: hr (per slot) -> y (fp32 per slot)
+  {
+    GemmParams r = g;
+    r.M = L.H;
+    r.K = L.I;
+    r.bits = L.bits;
+    r.expert_ptr = wts->expert_ptr;
+    r.off_codes[0] = L.off_codes[2];
+    r.off_scales[0] = L.off_scales[2];
+    r.b = reinterpret_cast<const uint16_t*>(ws + bp.hr);
+    r.ch_e = ch_e;
+    r.ch_c0 = ch_c0;
+    r.ch_n = ch_n;
+    r.n_chunks_dev = nch;
+    r.out = ws + bp.y;
+    CUDA_TRY(launch_grouped_gemm(L.bits, 1, 0, r, grid, stream));
+  }
+  const float* ys = nullptr;
+  if (L.has_shared) {
+    GemmParams r = g;
+    r.M = L.I;
+    r.K = L.H;
+    r.a_dense[0] = static_cast<const uint16_t*>(wts->shared_gate);
+    r.a_dense[1] = static_cast<const uint16_t*>(wts->shared_up);
+    r.b = x;
+    r.n_cols = T;
+    r.out = ws + bp.hs_hi;
+    r.out2 = ws + bp.hs_lo;
+    const int gr = tiles(T, L.I) < grid ? tiles(T, L.I) : grid;
+    CUDA_TRY(launch_grouped_gemm(0, 2, 2, r, gr, stream));
+    GemmParams d = g;
+    d.M = L.H;
+    d.K = L.I;
+    d.a_dense[0] = static_cast<const uint16_t*>(wts->shared_down);
+    d.b = reinterpret_cast<const uint16_t*>(ws + bp.hs_hi);
+    d.b2 = reinterpret_cast<const uint16_t*>(ws + bp.hs_lo);
+    d.n_cols = T;
+    d.out = ws + bp.ys;
+    const int gd = tiles(T, L.H) < grid ? tiles(T, L.H) : grid;
+    CUDA_TRY(launch_grouped_gemm(0, 1, 0, d, gd, stream));
+    ys = reinterpret_cast<const float*>(ws + bp.ys);
+  }
+  CUDA_TRY(launch_combine(reinterpret_cast<const float*>(ws + bp.y), ys, pair_slot, w,
+                          static_cast<const uint16_t*>(residual_bf16), static_cast<const uint16_t*>(wts->gamma), T,
+                          L.H, L.K, L.eps, static_cast<uint16_t*>(h_out_bf16), static_cast<uint16_t*>(y_norm_bf16),
+                          stream));
   return ok();
 }
 
@@ -374,9 +583,18 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
 }
 
 namespace moe {
-// For the library's other translation units: record an error message, and
-// run the fused layer on a given workspace.
+// For the library's other translation units: record an error message, the
+// workspace of the fused kernel's path, and run that path on a given
+// workspace.
 moe_status abi_fail(moe_status s, const char* msg) { return fail(s, "%s", msg); }
+size_t fused_workspace_bytes(const moe_config* cfg, int T) {
+  Layout L;
+  if (!cfg || T < 0 || cfg->n_experts <= 0 || cfg->top_k <= 0) return 0;
+  if (!make_layout(cfg->hidden, cfg->inter, cfg->n_experts, cfg->top_k, cfg->bits, cfg->group,
+                   cfg->has_shared, cfg->eps, &L))
+    return 0;
+  return ws_plan(L, T < chunk_tokens(L) ? T : chunk_tokens(L)).total;
+}
 moe_status layer_forward_on(const moe_config* cfg, const moe_layer_weights* wts, const void* x_bf16,
                             const void* residual_bf16, int T, void* h_out_bf16, void* y_norm_bf16,
                             int32_t* idx_out, float* w_out, void* workspace, size_t ws_bytes,
@@ -413,8 +631,60 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts
                              const void* x_bf16, const void* residual_bf16, int T,
                              void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out, float* w_out,
                              void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  Layout L;
+  if (cfg && T >= kBatchedMinTokens && check_cfg(cfg, &L) == MOE_OK && batched_ok(L))
+    return layer_forward_batched(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out,
+                                 workspace, ws_bytes, stream);
   return layer_forward_impl(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out,
                             workspace, ws_bytes, nullptr, 0, stream);
+}
+
+moe_status moe_layer_forward_batched(const moe_config* cfg, const moe_layer_weights* wts,
+                                     const void* x_bf16, const void* residual_bf16, int T,
+                                     void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out, float* w_out,
+                                     void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  return layer_forward_batched(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out,
+                               workspace, ws_bytes, stream);
+}
+
+moe_status moe_layer_forward_chunked(const moe_config* cfg, const moe_layer_weights* wts,
+                                     const void* x_bf16, const void* residual_bf16, int T,
+                                     void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out, float* w_out,
+                                     void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  return layer_forward_impl(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out,
+                            workspace, ws_bytes, nullptr, 0, stream);
+}
+
+moe_status moe_layer_forward_prenorm(const moe_config* cfg, const moe_layer_weights* wts,
+                                     const void* gamma_pre_bf16, const void* h_in_bf16, int T,
+                                     void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out, float* w_out,
+                                     void* x_out_bf16, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  Layout L;
+  moe_status s = check_cfg(cfg, &L);
+  if (s != MOE_OK) return s;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+  if (T == 0) return ok();
+  if (!gamma_pre_bf16 || !h_in_bf16 || !x_out_bf16) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(gamma_pre_bf16, 16) || !aligned(h_in_bf16, 16) || !aligned(x_out_bf16, 16))
+    return fail(MOE_ERR_INVALID_ARG, "bf16 arrays must be 16-byte aligned");
+  if (x_out_bf16 == h_in_bf16 || x_out_bf16 == h_out_bf16 || h_out_bf16 == h_in_bf16)
+    return fail(MOE_ERR_INVALID_ARG, "h_in, h_out and x_out must be distinct buffers");
+  L.prenorm = 1;
+  if (!(T >= kBatchedMinTokens && batched_ok(L))) {
+    DeviceInfo di;
+    if ((s = device_info(&di)) != MOE_OK) return s;
+    const int C = tokens_per_launch(L, di.sms < kMaxGrid ? di.sms : kMaxGrid, chunk_tokens(L));
+    if (C > 0 && T <= C)
+      return layer_forward_chunk(cfg, wts, h_in_bf16, h_in_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out,
+                                 workspace, ws_bytes, nullptr, 0, stream, nullptr, nullptr, gamma_pre_bf16,
+                                 x_out_bf16);
+  }
+  // more tokens than one fused launch takes: the normalisation as a kernel
+  // of its own, then the layer on its output
+  CUDA_TRY(launch_prenorm(static_cast<const uint16_t*>(h_in_bf16), static_cast<const uint16_t*>(gamma_pre_bf16), T,
+                          L.H, L.eps, static_cast<uint16_t*>(x_out_bf16), stream));
+  return moe_layer_forward(cfg, wts, x_out_bf16, h_in_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out, workspace,
+                           ws_bytes, stream);
 }
 
 int moe_layer_trace_blocks(void) {
@@ -440,14 +710,16 @@ size_t moe_layer_host_workspace_bytes(const moe_config* cfg, int T) {
   return base + 4 * act;
 }
 
-moe_status moe_layer_forward_host(const moe_config* cfg, const moe_layer_weights* wts,
-                                  const void* x_bf16_host, const void* residual_bf16_host, int T,
-                                  void* h_out_bf16_host, void* y_norm_bf16_host, void* workspace,
-                                  size_t ws_bytes, cudaStream_t stream) {
+// Host-buffer forms: x and residual are copied into staging areas of the
+// workspace (one copy when they arrive packed in one host buffer), the layer
+// runs, h_out and y_norm are copied back.
+static moe_status host_path(const moe_config* cfg, const moe_layer_weights* wts, const void* x_host,
+                            const void* res_host, const void* xr_host, int T, void* h_host, void* y_host,
+                            void* hy_host, void* workspace, size_t ws_bytes, cudaStream_t stream) {
   if (!cfg) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
   if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
   if (T == 0) return ok();
-  if (!x_bf16_host || !residual_bf16_host || !h_out_bf16_host || !y_norm_bf16_host)
+  if ((!xr_host && (!x_host || !res_host)) || (!hy_host && (!h_host || !y_host)))
     return fail(MOE_ERR_INVALID_ARG, "NULL host pointer");
   const size_t base = moe_layer_workspace_bytes(cfg, T);
   const size_t need = moe_layer_host_workspace_bytes(cfg, T);
@@ -457,16 +729,61 @@ moe_status moe_layer_forward_host(const moe_config* cfg, const moe_layer_weights
   const size_t bytes = 2ull * (size_t)T * cfg->hidden;
   const size_t act = (size_t)round_up_256(bytes);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  void* dx = ws + base;
-  void* dr = ws + base + act;
-  void* dh = ws + base + 2 * act;
-  void* dy = ws + base + 3 * act;
-  CUDA_TRY(cudaMemcpyAsync(dx, x_bf16_host, bytes, cudaMemcpyHostToDevice, stream));
-  CUDA_TRY(cudaMemcpyAsync(dr, residual_bf16_host, bytes, cudaMemcpyHostToDevice, stream));
+  uint8_t* dx = ws + base;
+  uint8_t* dr = ws + base + act;
+  uint8_t* dh = ws + base + 2 * act;
+  uint8_t* dy = ws + base + 3 * act;
+  if (xr_host) {
+    // staging areas are adjacent exactly when a token block is a multiple of 256 bytes
+    if (act == bytes) {
+      CUDA_TRY(cudaMemcpyAsync(dx, xr_host, 2 * bytes, cudaMemcpyHostToDevice, stream));
+    } else {
+      CUDA_TRY(cudaMemcpyAsync(dx, xr_host, bytes, cudaMemcpyHostToDevice, stream));
+      CUDA_TRY(cudaMemcpyAsync(dr, static_cast<const uint8_t*>(xr_host) + bytes, bytes, cudaMemcpyHostToDevice,
+                               stream));
+    }
+  } else {
+    CUDA_TRY(cudaMemcpyAsync(dx, x_host, bytes, cudaMemcpyHostToDevice, stream));
+    CUDA_TRY(cudaMemcpyAsync(dr, res_host, bytes, cudaMemcpyHostToDevice, stream));
+  }
   moe_status s = moe_layer_forward(cfg, wts, dx, dr, T, dh, dy, nullptr, nullptr, workspace, base, stream);
   if (s != MOE_OK) return s;
-  CUDA_TRY(cudaMemcpyAsync(h_out_bf16_host, dh, bytes, cudaMemcpyDeviceToHost, stream));
-  CUDA_TRY(cudaMemcpyAsync(y_norm_bf16_host, dy, bytes, cudaMemcpyDeviceToHost, stream));
+  if (hy_host) {
+    if (act == bytes) {
+      CUDA_TRY(cudaMemcpyAsync(hy_host, dh, 2 * bytes, cudaMemcpyDeviceToHost, stream));
+    } else {
+      CUDA_TRY(cudaMemcpyAsync(hy_host, dh, bytes, cudaMemcpyDeviceToHost, stream));
+      CUDA_TRY(cudaMemcpyAsync(static_cast<uint8_t*>(hy_host) + bytes, dy, bytes, cudaMemcpyDeviceToHost, stream));
+    }
+  } else {
+    CUDA_TRY(cudaMemcpyAsync(h_host, dh, bytes, cudaMemcpyDeviceToHost, stream));
+    CUDA_TRY(cudaMemcpyAsync(y_host, dy, bytes, cudaMemcpyDeviceToHost, stream));
+  }
+  return ok();
+}
+
+moe_status moe_layer_forward_host_async(const moe_config* cfg, const moe_layer_weights* wts,
+                                        const void* x_bf16_host, const void* residual_bf16_host, int T,
+                                        void* h_out_bf16_host, void* y_norm_bf16_host, void* workspace,
+                                        size_t ws_bytes, cudaStream_t stream) {
+  return host_path(cfg, wts, x_bf16_host, residual_bf16_host, nullptr, T, h_out_bf16_host, y_norm_bf16_host, nullptr,
+                   workspace, ws_bytes, stream);
+}
+
+moe_status moe_layer_forward_host_packed(const moe_config* cfg, const moe_layer_weights* wts,
+                                         const void* xr_bf16_host, int T, void* hy_bf16_host, void* workspace,
+                                         size_t ws_bytes, cudaStream_t stream) {
+  return host_path(cfg, wts, nullptr, nullptr, xr_bf16_host, T, nullptr, nullptr, hy_bf16_host, workspace, ws_bytes,
+                   stream);
+}
+
+moe_status moe_layer_forward_host(const moe_config* cfg, const moe_layer_weights* wts,
+                                  const void* x_bf16_host, const void* residual_bf16_host, int T,
+                                  void* h_out_bf16_host, void* y_norm_bf16_host, void* workspace,
+                                  size_t ws_bytes, cudaStream_t stream) {
+  moe_status s = moe_layer_forward_host_async(cfg, wts, x_bf16_host, residual_bf16_host, T, h_out_bf16_host,
+                                              y_norm_bf16_host, workspace, ws_bytes, stream);
+  if (s != MOE_OK || T == 0) return s;
   CUDA_TRY(cudaStreamSynchronize(stream));
   return ok();
 }

@@ -103,9 +103,9 @@ struct TileDesc {
 // barriers consumers -> sync warp (evt) and sync warp -> consumers (go)
 enum { EVT_R = 0, EVT_S, EVT_E, EVT_D, NEVT };
 enum { GO_S = 0, GO_E, GO_D, NGO };
-// flags[] slots: routing valid; consumer warps past the S tiles; this block
-// finished last
-enum { FLAG_TOPK = NGO, FLAG_SCNT, FLAG_LAST };
+// flags[] slots: routing valid; consumer warps past the S tiles; a sum of
+// squares that never arrived; this launch's epoch
+enum { FLAG_TOPK = NGO, FLAG_SCNT, FLAG_NOSS, FLAG_EPOCH };
 
 // ---- shared-memory plan ------------------------------------------------------
 // xf: x as mma A fragments, [token][group][t][8 words]; word 2s is the bf16
@@ -115,13 +115,13 @@ enum { FLAG_TOPK = NGO, FLAG_SCNT, FLAG_LAST };
 // hx: per (pair, 8-row block of I) sum of hi + lo.
 struct DecodeSmem {
   size_t ring, bars, desc, xs, xf, xsum, hs, hf, hx, zero, part, cnt, rpart, rcnt, tk_w, tk_i, eptr, tkbuf, res, gam,
-      ypart, ys, hacc, inv, flags, spin, total;
+      gpre, ypart, ys, hacc, inv, flags, spin, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
 
 __host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int E, int H, int I, int nrows, int nslots,
-                                                       uint32_t slot_bytes) {
+                                                       uint32_t slot_bytes, int prenorm) {
   const RoutedGeo gi = routed_geo(I, 4);
   DecodeSmem s;
   size_t pos = 0;
@@ -165,6 +165,8 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int E, int 
   pos = align_up(pos + 2ull * T * nrows, 16);
   s.gam = pos;
   pos = align_up(pos + 2ull * nrows, 16);
+  s.gpre = pos;  // pre-norm gamma [H] and the consumer warps' partial sums of squares [14][T]
+  pos = align_up(pos + (prenorm ? 2ull * H + 4ull * kConsumerWarps * T : 0ull), 16);
   s.ypart = pos;
   pos = align_up(pos + sizeof(float) * T * K * gi.U * nrows, 16);
   s.ys = pos;
@@ -182,7 +184,7 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int E, int 
 }
 
 size_t decode_smem_bytes(const Layout& L, int T, int nrows, int nslots, uint32_t slot_bytes) {
-  return decode_smem_plan(T, L.K, L.E, L.H, L.I, nrows, nslots, slot_bytes).total;
+  return decode_smem_plan(T, L.K, L.E, L.H, L.I, nrows, nslots, slot_bytes, L.prenorm).total;
 }
 
 // ---- small helpers ----------------------------------------------------------------
@@ -765,7 +767,7 @@ __device__ __forceinline__ bool ptab_in_smem(const DecodeParams& p) {
 template <bool TRACE>
 __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, uint16_t* res_s, uint16_t* gam_s,
                              uint64_t* xbar, uint64_t* topkbar, const int* flags, const uint8_t* const* eptr,
-                             uint64_t* ptab) {
+                             uint64_t* ptab, uint16_t* gpre_s) {
   const Layout& L = p.L;
   const int T = p.T, K = L.K, H = L.H, I = L.I, E = L.E;
   const int G = gridDim.x, c = blockIdx.x;
@@ -777,9 +779,11 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
   // the expert pointer table too, when it fits the top-K key buffer (unused
   // for E <= 512): the routing then finds its blobs without a global round trip
   const uint32_t tb = ptab_in_smem(p) ? (uint32_t)(8 * E) : 0u;
-  mbar_expect_tx(xbar, xb + (uint32_t)(T + 1) * rb + tb);
+  const uint32_t gb = L.prenorm ? (uint32_t)(2 * H) : 0u;
+  mbar_expect_tx(xbar, xb + (uint32_t)(T + 1) * rb + tb + gb);
   bulk_g2s(xs, p.x, xb, xbar);
   if (tb) bulk_g2s(ptab, p.expert_ptr, tb, xbar);
+  if (gb) bulk_g2s(gpre_s, p.gamma_pre, gb, xbar);
   if (rb > 0) {
 #pragma unroll 1
     for (int t = 0; t < T; ++t) bulk_g2s(res_s + (size_t)t * (r1 - r0), p.res + (size_t)t * H + r0, rb, xbar);
@@ -858,43 +862,12 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
                          uint32_t* spins) {
   const int lane = threadIdx.x & 31;
   const Layout& L = p.L;
-  const int T = p.T, H = L.H, K = L.K, E = L.E, G = gridDim.x;
+  const int T = p.T, K = L.K, E = L.E, G = gridDim.x;
   uint32_t* ctr = p.ctr;
   const uint64_t to = p.timeout_ns;
   uint32_t* sp_evt = spins ? spins + 5 : nullptr;
   uint32_t* sp_grid = spins ? spins + 6 : nullptr;
   bool ok = warp_wait(xbar, 0, to, spins ? spins + 7 : nullptr);
-  if (ok) {
-    // piece q: 8 columns (16 bytes) of one token's x; its four words go to
-    // lanes t = 0..3 of the A fragment of their group and step half
-    const int np = T * H / 8;
-#pragma unroll 1
-    for (int q0 = 0; q0 < np; q0 += 32) {
-      const int q = q0 + lane;
-      float s = 0.f;
-      if (q < np) {
-        const uint4 v = reinterpret_cast<const uint4*>(xs)[q];
-        const int tg = q >> 3, o8 = q & 7;  // tg = token * Gh + group
-        uint32_t* dst = reinterpret_cast<uint32_t*>(xf) + (size_t)tg * 32 + o8;
-        dst[0] = v.x;
-        dst[8] = v.y;
-        dst[16] = v.z;
-        dst[24] = v.w;
-        float xx[8];
-        unpack_bf16x8(v, xx);
-        s = ((xx[0] + xx[1]) + (xx[2] + xx[3])) + ((xx[4] + xx[5]) + (xx[6] + xx[7]));
-      }
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      s += __shfl_xor_sync(0xffffffffu, s, 4);
-      if (q < np && (q & 7) == 0) xsum[q >> 3] = s;
-    }
-  }
-  __syncwarp();
-  if (lane == 0) {
-    mbar_arrive(xfbar);
-    trace_mark<TRACE>(p, 64);
-  }
   int good;
   if (p.idx_in) {
     // the routing is given: no router barrier, no top-K
@@ -906,21 +879,19 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
     __syncwarp();
     good = __all_sync(0xffffffffu, ok) ? 1 : 0;
   } else {
-    // R: arrive once every consumer warp has passed the router tiles.  The
-    // waits up to the top-K are warp-uniform so the top-K runs unsplit.
-    ok = warp_wait(&evt[EVT_R], 0, to, sp_evt) && ok;
-    if (lane == 0) red_release_add(&ctr[0], 1u);
-    __syncwarp();
-    // top-K once every block's router logits are written
-    bool gr = ok && grid_wait_thread(&ctr[0], G, &ctr[5], p.err, to, lane == 0 ? sp_grid : nullptr);
-    good = __all_sync(0xffffffffu, gr) ? 1 : 0;
+    // the router logits of every block carry this launch's epoch once they
+    // are written: polling them is the router barrier and the top-K's loads
+    // in one (warp-uniform, so the top-K runs unsplit)
+    const uint32_t epoch = (uint32_t)flags[FLAG_EPOCH];
     if (lane == 0) trace_mark<TRACE>(p, 65);
-    if (good) {
+    bool gr = ok;
 #pragma unroll 1
-      for (int t = 0; t < T; ++t) warp_topk_keys(p.logits + (size_t)t * E, E, K, tkbuf, tk_i + t * K, tk_w + t * K);
-      __syncwarp();
-      if (lane == 0) trace_mark<TRACE>(p, 66);
-    }
+    for (int t = 0; t < T && gr; ++t)
+      gr = warp_topk_poll(p.logits + (size_t)t * E, epoch, E, K, tkbuf, tk_i + t * K, tk_w + t * K, &ctr[5], p.err,
+                          to, sp_grid);
+    good = __all_sync(0xffffffffu, gr) ? 1 : 0;
+    __syncwarp();
+    if (lane == 0) trace_mark<TRACE>(p, 66);
   }
   if (good) {
 #pragma unroll 1
@@ -982,7 +953,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   block_rows(H, c, G, r0, r1);
   const int nrows = r1 - r0;
   const int nslots = p.nslots;
-  const DecodeSmem sp = decode_smem_plan(T, K, L.E, H, I, decode_rows_max(H, G), nslots, p.slot_bytes);
+  const DecodeSmem sp = decode_smem_plan(T, K, L.E, H, I, decode_rows_max(H, G), nslots, p.slot_bytes, L.prenorm);
   uint8_t* ring = smem + sp.ring;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + sp.bars);
   uint64_t* empty = full + nslots;
@@ -1009,6 +980,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   uint64_t* tkbuf = reinterpret_cast<uint64_t*>(smem + sp.tkbuf);
   uint16_t* res_s = reinterpret_cast<uint16_t*>(smem + sp.res);
   uint16_t* gam_s = reinterpret_cast<uint16_t*>(smem + sp.gam);
+  uint16_t* gpre_s = reinterpret_cast<uint16_t*>(smem + sp.gpre);
+  float* wss = reinterpret_cast<float*>(smem + sp.gpre + 2ull * H);
   float* ypart = reinterpret_cast<float*>(smem + sp.ypart);
   float* ys = reinterpret_cast<float*>(smem + sp.ys);
   float* hacc = reinterpret_cast<float*>(smem + sp.hacc);
@@ -1034,7 +1007,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   if (tid < 16) {
     zero4[tid >> 2] = make_uint4(0u, 0u, 0u, 0u);
     spin_s[tid] = 0u;
-    flags[tid] = 0;
+    if (tid == FLAG_EPOCH) {
+      // this launch's epoch: one past the last launch's (0 is never used)
+      const uint32_t ep = ld_relaxed_gpu(ctr + 6) + 1u;
+      flags[tid] = (int)(ep == 0u ? 1u : ep);
+    } else {
+      flags[tid] = 0;
+    }
   }
   if (tid < kAccSlots) cnt[tid] = 0;
   if (tid < kSlots * kSplitRows) rcnt[tid] = 0;
@@ -1064,7 +1043,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       pr.d = descs;
       pr.fill = 0;
       pr.policy = l2_policy_evict_first();
-      run_producer<TRACE>(p, pr, xs, res_s, gam_s, xbar, topkbar, flags, eptr, tkbuf);
+      run_producer<TRACE>(p, pr, xs, res_s, gam_s, xbar, topkbar, flags, eptr, tkbuf, gpre_s);
     }
     __syncwarp();
   } else if (warp == kSyncWarp) {
@@ -1076,8 +1055,89 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     // of packed row blocks) are dealt round-robin to the warps, continuing
     // across tiles, and each warp releases a slot on its own.
     const RoutedGeo gh = routed_geo(H, 8), gi = routed_geo(I, 4);
+    const uint32_t epoch = (uint32_t)flags[FLAG_EPOCH];
     bool ok = warp_wait(xbar, 0, p.timeout_ns, spins ? spins + 2 : nullptr);
-    bool have_xf = false;
+    if (L.prenorm) {
+      // x is the residual stream: normalise it first, x = bf16(h / sqrt(mean(h^2) + eps) * gamma_pre),
+      // the sum of squares in fixed order (per warp, then over the warps)
+      const int np = T * H / 8;
+      float part[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) part[t] = 0.f;
+#pragma unroll 1
+      for (int q = tid; q < np; q += kConsumers) {
+        float hv[8];
+        unpack_bf16x8(reinterpret_cast<const uint4*>(xs)[q], hv);
+        float sq = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sq = fmaf(hv[i], hv[i], sq);
+        const int t = (8 * q) / H;
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt)
+          if (tt == t) part[tt] += sq;
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const float v = warp_sum(part[t]);
+        if (lane == 0 && t < T) wss[warp * T + t] = v;
+      }
+      consumer_sync();
+      if (tid < T) {
+        float ss = 0.f;
+        for (int w = 0; w < kConsumerWarps; ++w) ss += wss[w * T + tid];
+        inv[tid] = __fdiv_rn(1.f, __fsqrt_rn(__fdiv_rn(ss, (float)H) + L.eps));
+      }
+      consumer_sync();
+#pragma unroll 1
+      for (int q = tid; q < np; q += kConsumers) {
+        float hv[8], gv[8];
+        unpack_bf16x8(reinterpret_cast<const uint4*>(xs)[q], hv);
+        const int t = (8 * q) / H, col = 8 * q - t * H;
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(gpre_s + col), gv);
+        const float iv = inv[t];
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          o[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__fmul_rn(hv[2 * i], iv), gv[2 * i]))) |
+                 ((uint32_t)__bfloat16_as_ushort(
+                      __float2bfloat16_rn(__fmul_rn(__fmul_rn(hv[2 * i + 1], iv), gv[2 * i + 1])))
+                  << 16);
+        const uint4 xo = make_uint4(o[0], o[1], o[2], o[3]);
+        reinterpret_cast<uint4*>(xs)[q] = xo;
+        if (c == 0 && p.x_out) reinterpret_cast<uint4*>(p.x_out)[q] = xo;
+      }
+      consumer_sync();
+    }
+    {
+      // x as tensor-core fragments ([token][group][t][8 words]: word 2s is the
+      // bf16 pair at columns 16s + 2t (+1) of the group, word 2s + 1 the pair at
+      // 16s + 8 + 2t) and its group sums, built by all consumer threads: piece
+      // q is 8 columns of one token, its four words go to t = 0..3
+      const int np = T * H / 8;
+#pragma unroll 1
+      for (int q0 = 0; q0 < np; q0 += kConsumers) {
+        const int q = q0 + tid;
+        float sm = 0.f;
+        if (q < np) {
+          const uint4 v = reinterpret_cast<const uint4*>(xs)[q];
+          const int tg = q >> 3, o8 = q & 7;  // tg = token * Gh + group
+          uint32_t* dst = reinterpret_cast<uint32_t*>(xf) + (size_t)tg * 32 + o8;
+          dst[0] = v.x;
+          dst[8] = v.y;
+          dst[16] = v.z;
+          dst[24] = v.w;
+          float xx[8];
+          unpack_bf16x8(v, xx);
+          sm = ((xx[0] + xx[1]) + (xx[2] + xx[3])) + ((xx[4] + xx[5]) + (xx[6] + xx[7]));
+        }
+        sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+        sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+        sm += __shfl_xor_sync(0xffffffffu, sm, 4);
+        if (q < np && (q & 7) == 0) xsum[q >> 3] = sm;
+      }
+      consumer_sync();
+      if (tid == 0) trace_mark<TRACE>(p, 64);
+    }
     int item = 0;  // running count of work items over the compute tiles
     int probed = 0;  // first routed units traced: bit 0 gate/up, bit 1 down
     int nunit = 0;   // routed units done by this warp (traced launches)
@@ -1104,16 +1164,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         }
       }
       const bool routed_tile = type == TILE_EXPERT_GU || type == TILE_EXPERT_DOWN;
-      if (type == TILE_EXPERT_GU && !have_xf) {
-        ok = warp_wait(xfbar, 0, p.timeout_ns, spins ? spins + 2 : nullptr) && ok;
-        have_xf = true;
-      }
       const bool down = type == TILE_SHARED_DOWN || type == TILE_EXPERT_DOWN;
       const bool work = type != TILE_NONE && (ok || !down);  // down tiles need the staged intermediate
 #pragma unroll 1
       for (int si = 0; si < d.nseg; ++si) {
         const Seg& sg = d.seg[si];
         const int nu = sg.u1 - sg.u0;
+        // router / shared gate/up rows go through the tensor cores in groups
+        // of 16 rows; a tile of one group splits its columns into nparts parts
         // one-token router / shared gate/up rows: nparts column parts per row
         const bool split = T == 1 && (type == TILE_ROUTER || type == TILE_SHARED_GU) && d.nseg == 1 &&
                            sg.nrows <= kSplitRows;
@@ -1197,74 +1255,91 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
                     }
                     rcnt[slot * kSplitRows + rl] = 0;
                     if (type == TILE_ROUTER)
-                      p.logits[row] = a0;
+                      st_relaxed_gpu_b64(p.logits + row, epoch_word(epoch, a0));
                     else
                       p.hs[row] = silu_mul(a0, a1);
                   }
                 }
                 continue;
               }
+              if (type == TILE_ROUTER || type == TILE_SHARED_GU) {
+                // whole rows, one per work item
+                const uint8_t* w0 = sl + sg.off[0] + (size_t)j * 2 * cols;
+                const int row = sg.row0 + j;
+                const float rbias = (type == TILE_ROUTER && p.bias) ? __ldg(p.bias + row) : 0.f;
+                if (T == 1) {
+                  const uint32_t zs = smem_u32(zero4);
+                  float v0, v1 = 0.f;
+                  if (type == TILE_SHARED_GU) {
+                    float o[2];
+                    row_dot_t1<2, false>(smem_u32(w0), smem_u32(sl + sg.off[1] + (size_t)j * 2 * cols), smem_u32(xs),
+                                         H, zs, o);
+                    v0 = o[0];
+                    v1 = warp_sum(o[1]);
+                  } else {
+                    float o[1];
+                    row_dot_t1<1, false>(smem_u32(w0), 0u, smem_u32(xs), H, zs, o);
+                    v0 = o[0];
+                  }
+                  v0 = warp_sum(v0);
+                  if (lane == 0) {
+                    if (type == TILE_ROUTER)
+                      st_relaxed_gpu_b64(p.logits + row, epoch_word(epoch, v0 + rbias));
+                    else
+                      p.hs[row] = silu_mul(v0, v1);
+                  }
+                  continue;
+                }
+#pragma unroll 1
+                for (int t0 = 0; t0 < T; t0 += 4) {
+                  const int nt = min(4, T - t0);
+                  float acc[2][4];
+                  bf16_dot4(w0, type == TILE_SHARED_GU ? sl + sg.off[1] + (size_t)j * 2 * cols : nullptr, H,
+                            reinterpret_cast<const uint8_t*>(xs + (size_t)t0 * H), 2u * H, false, nt, acc);
+#pragma unroll 1
+                  for (int tt = 0; tt < nt; ++tt) {
+                    const int t = t0 + tt;
+                    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq)
+                      if (qq == tt) a0 = acc[0][qq], a1 = acc[1][qq];
+                    a0 = warp_sum(a0);
+                    if (type == TILE_SHARED_GU) a1 = warp_sum(a1);
+                    if (lane == 0) {
+                      if (type == TILE_ROUTER)
+                        st_relaxed_gpu_b64(p.logits + (size_t)t * L.E + row, epoch_word(epoch, a0 + rbias));
+                      else
+                        p.hs[(size_t)t * I + row] = silu_mul(a0, a1);
+                    }
+                  }
+                }
+                continue;
+              }
+              // ---- one bf16 row of the shared expert's down projection ----
               const uint8_t* w0 = sl + sg.off[0] + (size_t)j * 2 * cols;
               const int row = sg.row0 + j;
-              // the router bias is a global load: issue it before the dot
-              const float rbias = (type == TILE_ROUTER && p.bias) ? __ldg(p.bias + row) : 0.f;
               if (T == 1) {
                 // one token: the chunked dot, no per-token branches
-                const uint32_t zs = smem_u32(zero4);
-                float v0, v1 = 0.f;
-                if (down) {
-                  float o[1];
-                  row_dot_t1<1, true>(smem_u32(w0), 0u, smem_u32(hs_s), I, zs, o);
-                  v0 = o[0];
-                } else if (type == TILE_SHARED_GU) {
-                  float o[2];
-                  row_dot_t1<2, false>(smem_u32(w0), smem_u32(sl + sg.off[1] + (size_t)j * 2 * cols), smem_u32(xs),
-                                       H, zs, o);
-                  v0 = o[0];
-                  v1 = warp_sum(o[1]);
-                } else {
-                  float o[1];
-                  row_dot_t1<1, false>(smem_u32(w0), 0u, smem_u32(xs), H, zs, o);
-                  v0 = o[0];
-                }
-                v0 = warp_sum(v0);
-                if (lane == 0) {
-                  if (type == TILE_ROUTER)
-                    p.logits[row] = v0 + rbias;
-                  else if (type == TILE_SHARED_GU)
-                    p.hs[row] = silu_mul(v0, v1);
-                  else
-                    ys[row - r0] = v0;
-                }
+                float o[1];
+                row_dot_t1<1, true>(smem_u32(w0), 0u, smem_u32(hs_s), I, smem_u32(zero4), o);
+                const float v0 = warp_sum(o[0]);
+                if (lane == 0) ys[row - r0] = v0;
                 continue;
               }
 #pragma unroll 1
               for (int t0 = 0; t0 < T; t0 += 4) {
                 const int nt = min(4, T - t0);
                 float acc[2][4];
-                if (down)
-                  bf16_dot4(w0, nullptr, I, reinterpret_cast<const uint8_t*>(hs_s + (size_t)t0 * I), 4u * I, true,
-                            nt, acc);
-                else
-                  bf16_dot4(w0, type == TILE_SHARED_GU ? sl + sg.off[1] + (size_t)j * 2 * cols : nullptr, H,
-                            reinterpret_cast<const uint8_t*>(xs + (size_t)t0 * H), 2u * H, false, nt, acc);
+                bf16_dot4(w0, nullptr, I, reinterpret_cast<const uint8_t*>(hs_s + (size_t)t0 * I), 4u * I, true, nt,
+                          acc);
 #pragma unroll 1
                 for (int tt = 0; tt < nt; ++tt) {
-                  const int t = t0 + tt;
-                  float a0 = 0.f, a1 = 0.f;
+                  float a0 = 0.f;
 #pragma unroll
                   for (int q = 0; q < 4; ++q)
-                    if (q == tt) a0 = acc[0][q], a1 = acc[1][q];
+                    if (q == tt) a0 = acc[0][q];
                   a0 = warp_sum(a0);
-                  if (type == TILE_SHARED_GU) a1 = warp_sum(a1);
-                  if (lane == 0) {
-                    if (type == TILE_ROUTER)
-                      p.logits[(size_t)t * L.E + row] = a0 + rbias;
-                    else if (type == TILE_SHARED_GU)
-                      p.hs[(size_t)t * I + row] = silu_mul(a0, a1);
-                    else
-                      ys[t * nrows + row - r0] = a0;
-                  }
+                  if (lane == 0) ys[(t0 + tt) * nrows + row - r0] = a0;
                 }
               }
             }
@@ -1345,74 +1420,90 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         if (L.has_shared) h += ys[q];
         hacc[q] = h;
         p.h_out[(size_t)t * H + r0 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
-        p.hres[(size_t)t * H + r0 + j] = h;
       }
       consumer_sync();
+      // publish this block's sum of squares per token as an epoch word
       if (warp < T) {
         float s = 0.f;
 #pragma unroll 1
         for (int j = lane; j < nrows; j += 32) s = fmaf(hacc[warp * nrows + j], hacc[warp * nrows + j], s);
         s = warp_sum(s);
-        if (lane == 0) p.ss[(size_t)c * T + warp] = s;
+        if (lane == 0) st_relaxed_gpu_b64(p.ss + (size_t)c * T + warp, epoch_word(epoch, s));
+      }
+      // RMSNorm: every block polls all blocks' sums of squares (the words are
+      // complete once they carry this launch's epoch), sums them in block
+      // order and normalises its own rows of h
+      bool got = true;
+      if (warp < T) {
+        float s = 0.f;
+        uint64_t t0 = 0;
+        uint32_t it = 0;
+#pragma unroll 1
+        for (int b0 = 0; b0 < G && got; b0 += 32) {
+          const int bk = b0 + lane;
+          float v = 0.f;
+          bool have = bk >= G;
+          for (;; ++it) {
+            if (!have) {
+              const uint64_t wd = ld_relaxed_gpu_b64(p.ss + (size_t)bk * T + warp);
+              if ((uint32_t)(wd >> 32) == epoch) {
+                have = true;
+                v = __uint_as_float((uint32_t)wd);
+              }
+            }
+            if (__all_sync(0xffffffffu, have)) break;
+            if ((it & 63u) == 63u) {
+              int stop = 0;
+              if (lane == 0) {
+                if (t0 == 0) t0 = globaltimer_ns();
+                if (ld_relaxed_gpu(&ctr[5]) != 0u) {
+                  stop = 1;
+                } else if (globaltimer_ns() - t0 > p.timeout_ns) {
+                  atomicCAS(p.err, 0u, 1u);
+                  atomicExch(&ctr[5], 1u);
+                  stop = 1;
+                }
+              }
+              if (__shfl_sync(0xffffffffu, stop, 0)) {
+                got = false;
+                break;
+              }
+            }
+          }
+          s += v;
+        }
+        s = warp_sum(s);
+        if (lane == 0) {
+          inv[warp] = rsqrtf(__fdividef(s, (float)H) + L.eps);
+          if (!got) flags[FLAG_NOSS] = 1;  // some block's sum of squares never came
+        }
+      }
+      consumer_sync();
+      if (flags[FLAG_NOSS] == 0) {
+#pragma unroll 1
+        for (int q = tid; q < T * nrows; q += kConsumers) {
+          const int t = q / nrows, j = q - t * nrows;
+          const float g = __bfloat162float(__ushort_as_bfloat16(gam_s[j]));
+          p.y_norm[(size_t)t * H + r0 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(hacc[q] * inv[t] * g));
+        }
       }
     }
   }
 
-  // ---- exit: RMSNorm needs every block's sum of squares, so the last block
-  // to finish its rows of h normalises all of them; it also resets the
-  // counters for the next launch (every other block is past its last wait) ----
+  // ---- exit: the block that arrives last on the final counter resets the
+  // counters and records this launch's epoch for the next launch (every other
+  // block is past its last use of them) ----
   __syncthreads();
   if (tid == 0) {
     if constexpr (TRACE)
       for (int k = 0; k < 8; ++k) p.trace[(size_t)c * kTraceEntries + 80 + k] = spin_s[k];
-    flags[FLAG_LAST] = atom_add_acq_rel_gpu(&ctr[3], 1u) == (uint32_t)G - 1u ? 1 : 0;
     trace_mark<TRACE>(p, 7);
-  }
-  __syncthreads();
-  if (flags[FLAG_LAST]) {
-    // eight columns of one token per thread and pass; the first pass's loads,
-    // the sums of squares and the error word are all in flight together
-    const float4* hr = reinterpret_cast<const float4*>(p.hres);
-    const int n8 = T * H / 8;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-    uint4 gw = make_uint4(0u, 0u, 0u, 0u);
-    if (tid < n8) {
-      a = __ldcg(hr + 2 * tid);
-      b = __ldcg(hr + 2 * tid + 1);
-      gw = __ldg(reinterpret_cast<const uint4*>(p.gamma + (8 * tid) % H));
+    if (atomicAdd(&ctr[3], 1u) == (uint32_t)G - 1u) {
+      // plain stores: the next launch reads them after this one ends
+      volatile uint32_t* vc = reinterpret_cast<volatile uint32_t*>(ctr);
+      for (int k = 0; k < 6; ++k) vc[k] = 0u;
+      vc[6] = (uint32_t)flags[FLAG_EPOCH];
     }
-    const bool good = flags[FLAG_TOPK] != 0 && ld_relaxed_gpu(p.err) == 0u;
-    if (warp < T) {
-      float s = 0.f;
-#pragma unroll 1
-      for (int bk = lane; bk < G; bk += 32) s += __ldcg(p.ss + (size_t)bk * T + warp);
-      s = warp_sum(s);
-      if (lane == 0) inv[warp] = rsqrtf(__fdividef(s, (float)H) + L.eps);
-    }
-    __syncthreads();
-    if (good) {
-#pragma unroll 1
-      for (int q = tid; q < n8; q += kDecodeThreads) {
-        const int t = (8 * q) / H, col = 8 * q - t * H;
-        if (q != tid) {
-          a = __ldcg(hr + 2 * q);
-          b = __ldcg(hr + 2 * q + 1);
-          gw = __ldg(reinterpret_cast<const uint4*>(p.gamma + col));
-        }
-        float gm[8];
-        unpack_bf16x8(gw, gm);
-        const float hv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        const float iv = inv[t];
-        uint32_t o[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          o[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[2 * i] * iv * gm[2 * i])) |
-                 ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[2 * i + 1] * iv * gm[2 * i + 1])) << 16);
-        reinterpret_cast<uint4*>(p.y_norm)[q] = make_uint4(o[0], o[1], o[2], o[3]);
-      }
-    }
-    // plain stores: the next launch reads the counters after this one ends
-    if (tid < 6) reinterpret_cast<volatile uint32_t*>(ctr)[tid] = 0u;
   }
   if (tid == 0) trace_mark<TRACE>(p, 8);
 }
@@ -1458,7 +1549,7 @@ uint32_t decode_slot_bytes(const Layout& L, int T, int nrows_max, int* nslots) {
   const size_t need[5] = {2ull * L.H + 16, 4ull * L.H + 32, 2ull * L.I + 16,
                           2ull * 2 * 8 * gh.W * per_group + 64, 2ull * 4 * gi.W * per_group + 64};
   for (int ns = kSlots; ns >= 2; --ns) {
-    const size_t other = decode_smem_plan(T, L.K, L.E, L.H, L.I, nrows_max, ns, 0).total + 1024;
+    const size_t other = decode_smem_plan(T, L.K, L.E, L.H, L.I, nrows_max, ns, 0, L.prenorm).total + 1024;
     if (other >= limit) return 0;
     size_t slot = (limit - other) / ns;
     slot = slot / 1024 * 1024;

@@ -63,6 +63,21 @@ __device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
   return v;
 }
 
+// 64-bit words that carry their own launch number: a value published as
+// (epoch << 32 | value bits) with one relaxed store is complete once a
+// reader sees the current epoch in it, without a separate flag or fence.
+__device__ __forceinline__ void st_relaxed_gpu_b64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_relaxed_gpu_b64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t epoch_word(uint32_t epoch, float v) {
+  return ((uint64_t)epoch << 32) | __float_as_uint(v);
+}
+
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -269,6 +284,127 @@ static __device__ __noinline__ void warp_topk_keys(const float* logits, int E, i
     }
   }
   topk_weights(K, w);
+}
+
+// The same for logits that other blocks of this launch publish as epoch
+// words (epoch_word): every lane polls its words (one load each, all in
+// flight) until each carries `epoch`, then the K rounds run as above.
+// epoch == 0 accepts any word (a dry run over whatever the buffer holds).
+// Gives up, returning false, when *abort_flag is raised or the time limit
+// passes (recording MOE device error 1 and raising the flag).  E <= 512:
+// keys in registers; larger E: staged in `keys` (E entries of shared memory).
+static __device__ __noinline__ bool warp_topk_poll(const uint64_t* words, uint32_t epoch, int E, int K,
+                                                   uint64_t* keys, int32_t* idx, float* w, uint32_t* abort_flag,
+                                                   uint32_t* err, uint64_t timeout_ns, uint32_t* polls) {
+  const int lane = threadIdx.x & 31;
+  uint64_t t0 = 0;
+  uint32_t nit = 0;
+  bool ok = true;
+  // poll words [e0, e0 + 512) into v[]: lane's i-th word is e0 + lane + 32 i
+  auto poll = [&](int e0, float (&v)[16]) -> bool {
+    uint32_t need = 0, have = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (e0 + lane + 32 * i < E) need |= 1u << i;
+    for (uint32_t it = 0;; ++it) {
+      uint64_t wv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        wv[i] = ((need & ~have) >> i & 1u) ? ld_relaxed_gpu_b64(words + e0 + lane + 32 * i) : 0ull;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (((need & ~have) >> i & 1u) && (epoch == 0u || (uint32_t)(wv[i] >> 32) == epoch)) {
+          have |= 1u << i;
+          v[i] = __uint_as_float((uint32_t)wv[i]);
+        }
+      ++nit;
+      if (__all_sync(0xffffffffu, have == need)) return true;
+      if ((it & 31u) == 31u) {
+        int stop = 0;
+        if (lane == 0) {
+          if (t0 == 0) t0 = globaltimer_ns();
+          if (ld_relaxed_gpu(abort_flag) != 0u) {
+            stop = 1;
+          } else if (globaltimer_ns() - t0 > timeout_ns) {
+            atomicCAS(err, 0u, 1u);
+            atomicExch(abort_flag, 1u);
+            stop = 1;
+          }
+        }
+        if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+      }
+    }
+  };
+  if (E <= 512) {
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+    ok = poll(0, v);
+    if (polls && lane == 0) atomicAdd(polls, nit);
+    if (!ok) return false;
+    uint64_t kr[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = lane + 32 * i;
+      kr[i] = e < E ? topk_key(v[i], e) : 0ull;
+    }
+    uint64_t mine = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mine = kr[i] > mine ? kr[i] : mine;
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+      const uint32_t hi = (uint32_t)(mine >> 32);
+      const uint32_t hmax = __reduce_max_sync(0xffffffffu, hi);
+      const uint32_t lmax = __reduce_max_sync(0xffffffffu, hi == hmax ? (uint32_t)mine : 0u);
+      const uint64_t best = ((uint64_t)hmax << 32) | lmax;
+      if (lane == 0) {
+        idx[k] = (int)~lmax;
+        w[k] = topk_key_value(best);
+      }
+      if (mine == best) {
+        uint64_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = (kr[i] < best && kr[i] > m) ? kr[i] : m;
+        mine = m;
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int e0 = 0; e0 < E && ok; e0 += 512) {
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      ok = poll(e0, v);
+      if (ok) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int e = e0 + lane + 32 * i;
+          if (e < E) keys[e] = topk_key(v[i], e);
+        }
+      }
+    }
+    if (polls && lane == 0) atomicAdd(polls, nit);
+    if (!ok) return false;
+    __syncwarp();
+    uint64_t prev = ~0ull;
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+      uint64_t best = 0;
+#pragma unroll 4
+      for (int e = lane; e < E; e += 32) {
+        const uint64_t key = keys[e];
+        best = (key < prev && key > best) ? key : best;
+      }
+      best = warp_max_u64(best);
+      if (lane == 0) {
+        idx[k] = (int)~(uint32_t)best;
+        w[k] = topk_key_value(best);
+      }
+      prev = best;
+    }
+  }
+  topk_weights(K, w);
+  return true;
 }
 
 // SiLU(g) * u with a fast division (relative error of a few ulp).

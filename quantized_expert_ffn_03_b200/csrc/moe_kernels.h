@@ -39,10 +39,11 @@ __host__ __device__ inline void block_rows(int H, int c, int G, int& r0, int& r1
 }
 __host__ __device__ inline int decode_rows_max(int H, int G) { return 16 * ((H / 16 + G - 1) / G); }
 
-// Workspace of a layer call: counters and error word first, then fp32
-// intermediates.  ctr[0] router, [1] shared gate/up, [2] routed gate/up,
-// [3] blocks that finished their rows of h, [4] unused, [5] abort flag of
-// the running launch.
+// Workspace of a layer call: counters and error word first, then the
+// intermediates.  ctr[1] shared gate/up, [2] routed gate/up, [3] blocks that
+// finished, [5] abort flag of the running launch, [6] the last launch's
+// epoch (each launch publishes its router logits and sums of squares as
+// 64-bit words tagged with its own epoch, ctr[6] + 1).
 struct DecodeParams {
   Layout L;
   int T;
@@ -53,6 +54,8 @@ struct DecodeParams {
   const uint16_t* su;
   const uint16_t* sd;
   const uint16_t* gamma;
+  const uint16_t* gamma_pre;  // L.prenorm: bf16 [H] weight of the RMSNorm applied to x first
+  uint16_t* x_out;            // L.prenorm: the normalised x, bf16 [T][H] (block 0 writes it), or null
   const uint16_t* x;
   const uint16_t* res;
   uint16_t* h_out;
@@ -63,12 +66,11 @@ struct DecodeParams {
   const float* w_in;
   uint32_t* ctr;
   uint32_t* err;
-  float* logits;  // [T][E]
-  float* hs;      // [T][I]
-  uint8_t* hf;    // routed intermediate as hi/lo bf16 B fragments, 4*T*K*I bytes
-  float* hx;      // [T*K][I/16] sums of hi + lo over 16-row blocks
-  float* ss;      // [grid][T] sums of squares of each block's rows of h
-  float* hres;    // [T][H] h in fp32, normalised by the last block to finish
+  uint64_t* logits;  // [T][E] router logits as epoch words (epoch << 32 | float bits)
+  float* hs;         // [T][I]
+  uint8_t* hf;       // routed intermediate as hi/lo bf16 B fragments, 4*T*K*I bytes
+  float* hx;         // [T*K][I/16] sums of hi + lo over 16-row blocks
+  uint64_t* ss;      // [grid][T] each block's sum of squares of its rows of h, as epoch words
   uint64_t timeout_ns;
   uint32_t slot_bytes;  // bytes per shared-memory ring slot
   int nslots;           // ring slots (2..4)
@@ -99,6 +101,8 @@ size_t grouped_gemm_smem_bytes(int na, bool packed);
 // ak: 0 dense bf16 A, 4 / 2 packed A; na: A matrices (2 = gate and up);
 // epi: 0 fp32 (+ bias), 1 SwiGLU -> fp16, 2 SwiGLU -> bf16 hi and lo.
 cudaError_t launch_grouped_gemm(int ak, int na, int epi, const GemmParams& p, int grid, cudaStream_t st);
+cudaError_t launch_prenorm(const uint16_t* h, const uint16_t* gamma, int T, int H, float eps, uint16_t* x,
+                           cudaStream_t st);
 cudaError_t launch_to_half(const uint16_t* x, void* xh, size_t n, uint32_t* abort_flag, cudaStream_t st);
 cudaError_t launch_group(const int32_t* idx, int TK, int E, int K, int* slot_token, int* pair_slot, int* ch_e,
                          int* ch_c0, int* ch_n, int* n_chunks, const void* const* expert_ptr, uint32_t* err,

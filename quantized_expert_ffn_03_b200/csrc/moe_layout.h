@@ -28,6 +28,7 @@ struct Layout {
   int H, I, E, K, bits;
   int has_shared;
   float eps;
+  int prenorm;  // 1: the layer's x is its residual stream, RMS-normalised with a second gamma first
   uint32_t off_codes[3];
   uint32_t off_scales[3];
   uint32_t code_row_bytes[3];
@@ -50,6 +51,7 @@ inline bool make_layout(int H, int I, int E, int K, int bits, int group, int has
   L->bits = bits;
   L->has_shared = has_shared;
   L->eps = eps;
+  L->prenorm = 0;
   const uint64_t rows[3] = {(uint64_t)I, (uint64_t)I, (uint64_t)H};
   const uint64_t cols[3] = {(uint64_t)H, (uint64_t)H, (uint64_t)I};
   uint64_t pos = 0;

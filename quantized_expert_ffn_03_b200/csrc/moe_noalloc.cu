@@ -31,6 +31,7 @@
 
 namespace moe {
 moe_status abi_fail(moe_status s, const char* msg);
+size_t fused_workspace_bytes(const moe_config* cfg, int T);
 moe_status layer_forward_on(const moe_config* cfg, const moe_layer_weights* wts, const void* x_bf16,
                             const void* residual_bf16, int T, void* h_out_bf16, void* y_norm_bf16,
                             int32_t* idx_out, float* w_out, void* workspace, size_t ws_bytes,
@@ -73,7 +74,7 @@ extern "C" moe_status moe_layer_forward_noalloc(const moe_config* cfg, const moe
                                                 float* w_out, cudaStream_t stream) {
   if (!cfg) return moe::abi_fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
   if (T < 0) return moe::abi_fail(MOE_ERR_INVALID_ARG, "T < 0");
-  const size_t need = moe_layer_workspace_bytes(cfg, T);
+  const size_t need = moe::fused_workspace_bytes(cfg, T);
   if (need == 0)
     return moe::abi_fail(MOE_ERR_UNSUPPORTED,
                          "unsupported shape (bits 2 or 4, group 64, hidden and inter positive multiples of 64)");

@@ -33,10 +33,22 @@
 // the GPU).
 #include <cuda_runtime.h>
 
+#include <fcntl.h>
+#include <sys/stat.h>
+#include <unistd.h>
+
+#include <algorithm>
+#include <cerrno>
+#include <chrono>
+#include <condition_variable>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <deque>
+#include <functional>
 #include <mutex>
+#include <thread>
+#include <utility>
 #include <vector>
 
 #include "../../include/moe.h"
@@ -62,11 +74,89 @@ moe_status failf(moe_status s, const char* fmt, ...) {
 
 }  // namespace
 
+namespace {
+
+// A fixed pool of host threads that run the reads of one call in parallel
+// (the pages read the K chosen experts of a layer with parallel pread).
+struct IoPool {
+  std::vector<std::thread> th;
+  std::mutex m;
+  std::condition_variable cv, done;
+  std::deque<std::function<void()>> q;
+  int pending = 0;
+  bool stop = false;
+
+  void start(int n) {
+    for (int i = 0; i < n; ++i)
+      th.emplace_back([this] {
+        for (;;) {
+          std::function<void()> job;
+          {
+            std::unique_lock<std::mutex> lk(m);
+            cv.wait(lk, [this] { return stop || !q.empty(); });
+            if (stop && q.empty()) return;
+            job = std::move(q.front());
+            q.pop_front();
+          }
+          job();
+          std::lock_guard<std::mutex> lk(m);
+          if (--pending == 0) done.notify_all();
+        }
+      });
+  }
+  // runs the jobs on the pool and returns when all of them have finished
+  void run(std::vector<std::function<void()>>& jobs) {
+    if (jobs.empty()) return;
+    {
+      std::lock_guard<std::mutex> lk(m);
+      for (auto& j : jobs) q.push_back(std::move(j));
+      pending += (int)jobs.size();
+    }
+    cv.notify_all();
+    std::unique_lock<std::mutex> lk(m);
+    done.wait(lk, [this] { return pending == 0; });
+  }
+  void shutdown() {
+    {
+      std::lock_guard<std::mutex> lk(m);
+      stop = true;
+    }
+    cv.notify_all();
+    for (auto& t : th) t.join();
+    th.clear();
+  }
+};
+
+// Reads `bytes` at `off` of fd into dst, retrying short reads; false on error.
+bool read_full(int fd, uint8_t* dst, size_t bytes, off_t off) {
+  size_t got = 0;
+  while (got < bytes) {
+    const ssize_t r = pread(fd, dst + got, bytes - got, off + (off_t)got);
+    if (r < 0 && errno == EINTR) continue;
+    if (r <= 0) return false;
+    got += (size_t)r;
+  }
+  return true;
+}
+
+constexpr int kFileStage = 16;  // pinned staging buffers of a file-backed store
+
+}  // namespace
+
 struct moe_stream_cache {
   int L = 0, E = 0, S = 0;
   size_t blob = 0;
   int device = 0;
-  const uint8_t* host = nullptr;
+  const uint8_t* host = nullptr;  // pinned host store, or null for a file store
+  // file store: the file, pinned staging buffers (each reused once the copy
+  // that last read it is done), the read pool, and read statistics
+  int fd = -1;
+  uint8_t* fstage[kFileStage] = {};
+  cudaEvent_t fstage_ev[kFileStage] = {};
+  bool fstage_used[kFileStage] = {};
+  int fstage_next = 0;
+  IoPool io;
+  uint64_t reads = 0, read_ns = 0, read_bytes = 0;
   uint8_t* slots = nullptr;
   moe::StreamPolicy pol;
   std::vector<cudaEvent_t> ready, used;
@@ -76,6 +166,13 @@ struct moe_stream_cache {
   int stage_next = 0;
   uint64_t bytes_h2d = 0;
   int fault_copy = -1;  // injected: copies left before one fails (-1: none)
+  // optional copy timing: an event pair around each copy, relative to `ref`
+  bool timing = false;
+  bool ref_recorded = false;
+  cudaEvent_t ref = nullptr;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> timed;
+  std::vector<cudaEvent_t> spare;
+  uint64_t timed_bytes = 0;
   std::mutex mu;
 };
 
@@ -86,7 +183,33 @@ std::mutex g_fault_mu;
 
 namespace {
 
+cudaEvent_t take_event(moe_stream_cache* c) {
+  if (!c->spare.empty()) {
+    cudaEvent_t e = c->spare.back();
+    c->spare.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+
 void destroy_parts(moe_stream_cache* c) {
+  c->io.shutdown();
+  for (int i = 0; i < kFileStage; ++i) {
+    if (c->fstage_ev[i]) cudaEventDestroy(c->fstage_ev[i]);
+    if (c->fstage[i]) cudaFreeHost(c->fstage[i]);
+  }
+  if (c->fd >= 0) close(c->fd);
+  for (auto& pr : c->timed) {
+    cudaEventDestroy(pr.first);
+    cudaEventDestroy(pr.second);
+  }
+  for (cudaEvent_t e : c->spare) cudaEventDestroy(e);
+  if (c->ref) cudaEventDestroy(c->ref);
   for (cudaEvent_t e : c->ready)
     if (e) cudaEventDestroy(e);
   for (cudaEvent_t e : c->used)
@@ -100,16 +223,34 @@ void destroy_parts(moe_stream_cache* c) {
 
 // Enqueue the copy of (layer, e) into slot s on stream st (see the ordering
 // rules at the top of the file); the policy has already assigned the slot.
-moe_status fill_slot(moe_stream_cache* c, int s, int layer, int e, cudaStream_t st) {
+moe_status fill_slot(moe_stream_cache* c, int s, int layer, int e, cudaStream_t st, const uint8_t* src_stage = nullptr) {
   cudaError_t err = cudaStreamWaitEvent(st, c->used[s], 0);
   if (err == cudaSuccess) err = cudaStreamWaitEvent(st, c->ready[s], 0);
   if (err != cudaSuccess) return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
-  const uint8_t* src = c->host + ((size_t)layer * c->E + e) * c->blob;
+  const uint8_t* src = src_stage ? src_stage : c->host + ((size_t)layer * c->E + e) * c->blob;
   if (c->fault_copy >= 0 && c->fault_copy-- == 0) {
     c->pol.evict(s);
     return failf(MOE_ERR_IO, "copy of expert %d of layer %d from the host store failed: injected fault", e, layer);
   }
+  cudaEvent_t tb = nullptr, te = nullptr;
+  if (c->timing) {
+    if (!c->ref_recorded && cudaEventRecord(c->ref, st) == cudaSuccess) c->ref_recorded = true;
+    tb = take_event(c);
+    te = take_event(c);
+    if (tb && te && c->ref_recorded) {
+      cudaEventRecord(tb, st);
+    } else {
+      if (tb) c->spare.push_back(tb);
+      if (te) c->spare.push_back(te);
+      tb = te = nullptr;
+    }
+  }
   err = cudaMemcpyAsync(c->slots + (size_t)s * c->blob, src, c->blob, cudaMemcpyHostToDevice, st);
+  if (tb) {
+    cudaEventRecord(te, st);
+    c->timed.emplace_back(tb, te);
+    c->timed_bytes += c->blob;
+  }
   if (err != cudaSuccess) {
     c->pol.evict(s);
     return failf(MOE_ERR_IO, "copy of expert %d of layer %d from the host store failed: %s", e, layer,
@@ -118,6 +259,84 @@ moe_status fill_slot(moe_stream_cache* c, int s, int layer, int e, cudaStream_t 
   err = cudaEventRecord(c->ready[s], st);
   if (err != cudaSuccess) return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
   c->bytes_h2d += c->blob;
+  return MOE_OK;
+}
+
+struct Fill {
+  int slot, layer, e;
+};
+
+// Issues the fills of one call.  A pinned store is copied from directly.  A
+// file store first reads every blob of the call into its own pinned staging
+// buffer, in parallel on the read pool, then enqueues the copies; a staging
+// buffer is reused once the copy that last read it has completed (the host
+// waits for that).  On failure, the slots of the fills not issued are left
+// empty and *issued says how many fills were enqueued.
+moe_status do_fills(moe_stream_cache* c, const std::vector<Fill>& fills, cudaStream_t st, int* issued) {
+  *issued = 0;
+  if (c->fd < 0) {
+    for (const Fill& f : fills) {
+      const moe_status s = fill_slot(c, f.slot, f.layer, f.e, st);
+      if (s != MOE_OK) {
+        for (size_t k = *issued + 1; k < fills.size(); ++k) c->pol.evict(fills[k].slot);
+        return s;
+      }
+      ++*issued;
+    }
+    return MOE_OK;
+  }
+  for (size_t b0 = 0; b0 < fills.size(); b0 += kFileStage) {
+    const size_t nb = std::min(fills.size() - b0, (size_t)kFileStage);
+    std::vector<int> sb(nb);
+    for (size_t k = 0; k < nb; ++k) {
+      const int i = c->fstage_next;
+      c->fstage_next = (i + 1) % kFileStage;
+      if (c->fstage_used[i]) {
+        const cudaError_t err = cudaEventSynchronize(c->fstage_ev[i]);
+        if (err != cudaSuccess) return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
+      }
+      sb[k] = i;
+    }
+    std::vector<char> okv(nb, 0);
+    std::vector<std::function<void()>> jobs;
+    const uint64_t t0 = (uint64_t)std::chrono::duration_cast<std::chrono::nanoseconds>(
+                            std::chrono::steady_clock::now().time_since_epoch()).count();
+    for (size_t k = 0; k < nb; ++k) {
+      const Fill f = fills[b0 + k];
+      uint8_t* dst = c->fstage[sb[k]];
+      const off_t off = (off_t)(((size_t)f.layer * c->E + f.e) * c->blob);
+      const int fd = c->fd;
+      const size_t bytes = c->blob;
+      char* okp = &okv[k];
+      jobs.push_back([fd, dst, bytes, off, okp] { *okp = read_full(fd, dst, bytes, off) ? 1 : 0; });
+    }
+    c->io.run(jobs);
+    const uint64_t t1 = (uint64_t)std::chrono::duration_cast<std::chrono::nanoseconds>(
+                            std::chrono::steady_clock::now().time_since_epoch()).count();
+    c->reads += nb;
+    c->read_bytes += nb * c->blob;
+    c->read_ns += t1 - t0;
+    for (size_t k = 0; k < nb; ++k) {
+      const Fill& f = fills[b0 + k];
+      moe_status s = MOE_OK;
+      if (!okv[k]) {
+        c->pol.evict(f.slot);
+        s = failf(MOE_ERR_IO, "read of expert %d of layer %d from the store file failed", f.e, f.layer);
+      } else {
+        s = fill_slot(c, f.slot, f.layer, f.e, st, c->fstage[sb[k]]);
+      }
+      if (s == MOE_OK) {
+        const cudaError_t err = cudaEventRecord(c->fstage_ev[sb[k]], st);
+        if (err != cudaSuccess) s = failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
+        c->fstage_used[sb[k]] = true;
+      }
+      if (s != MOE_OK) {
+        for (size_t j = b0 + k + 1; j < fills.size(); ++j) c->pol.evict(fills[j].slot);
+        return s;
+      }
+      ++*issued;
+    }
+  }
   return MOE_OK;
 }
 
@@ -140,37 +359,16 @@ struct DeviceGuard {
   }
 };
 
-}  // namespace
-
-extern "C" {
-
-moe_status moe_stream_create(const moe_config* cfg, int n_layers, const void* host_pinned_experts,
-                             size_t store_bytes, int n_slots, moe_stream_cache** out) {
-  if (!out) return failf(MOE_ERR_INVALID_ARG, "out is NULL");
-  *out = nullptr;
-  if (!cfg) return failf(MOE_ERR_INVALID_ARG, "cfg is NULL");
+// The part of creating a cache common to both stores: the policy, the slots
+// (the library's one device allocation), the per-slot events and the pinned
+// staging ring of the pointer table.  Takes ownership of c.
+moe_status finish_create(moe_stream_cache* c, const moe_config* cfg, int n_layers, int n_slots,
+                         moe_stream_cache** out) {
   const size_t blob = moe_packed_expert_bytes(cfg);
-  if (blob == 0 || cfg->n_experts <= 0) return failf(MOE_ERR_UNSUPPORTED, "unsupported shape");
-  if (n_layers < 1 || n_slots < 1) return failf(MOE_ERR_INVALID_ARG, "n_layers and n_slots must be >= 1");
-  if (!host_pinned_experts) return failf(MOE_ERR_INVALID_ARG, "host store is NULL");
-  const size_t need = blob * (size_t)cfg->n_experts * (size_t)n_layers;
-  if (store_bytes < need)
-    return failf(MOE_ERR_INVALID_ARG, "the host store holds %zu bytes; %d layers of %d experts need %zu", store_bytes,
-                 n_layers, cfg->n_experts, need);
-  // both ends of the store must be page-locked memory
-  cudaPointerAttributes attr, attr_end;
-  const uint8_t* last_byte = static_cast<const uint8_t*>(host_pinned_experts) + need - 1;
-  if (cudaPointerGetAttributes(&attr, host_pinned_experts) != cudaSuccess || attr.type != cudaMemoryTypeHost ||
-      cudaPointerGetAttributes(&attr_end, last_byte) != cudaSuccess || attr_end.type != cudaMemoryTypeHost) {
-    cudaGetLastError();
-    return failf(MOE_ERR_INVALID_ARG, "the host store must be page-locked (cudaHostAlloc or cudaHostRegister)");
-  }
-  moe_stream_cache* c = new moe_stream_cache;
   c->L = n_layers;
   c->E = cfg->n_experts;
   c->S = n_slots;
   c->blob = blob;
-  c->host = static_cast<const uint8_t*>(host_pinned_experts);
   cudaGetDevice(&c->device);
   c->pol.init(n_layers, cfg->n_experts, n_slots);
   bool alloc_fault = false;
@@ -206,20 +404,98 @@ moe_status moe_stream_create(const moe_config* cfg, int n_layers, const void* ho
   return MOE_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+moe_status moe_stream_create(const moe_config* cfg, int n_layers, const void* host_pinned_experts,
+                             size_t store_bytes, int n_slots, moe_stream_cache** out) {
+  if (!out) return failf(MOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!cfg) return failf(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  const size_t blob = moe_packed_expert_bytes(cfg);
+  if (blob == 0 || cfg->n_experts <= 0) return failf(MOE_ERR_UNSUPPORTED, "unsupported shape");
+  if (n_layers < 1 || n_slots < 1) return failf(MOE_ERR_INVALID_ARG, "n_layers and n_slots must be >= 1");
+  if (!host_pinned_experts) return failf(MOE_ERR_INVALID_ARG, "host store is NULL");
+  const size_t need = blob * (size_t)cfg->n_experts * (size_t)n_layers;
+  if (store_bytes < need)
+    return failf(MOE_ERR_INVALID_ARG, "the host store holds %zu bytes; %d layers of %d experts need %zu", store_bytes,
+                 n_layers, cfg->n_experts, need);
+  // both ends of the store must be page-locked memory
+  cudaPointerAttributes attr, attr_end;
+  const uint8_t* last_byte = static_cast<const uint8_t*>(host_pinned_experts) + need - 1;
+  if (cudaPointerGetAttributes(&attr, host_pinned_experts) != cudaSuccess || attr.type != cudaMemoryTypeHost ||
+      cudaPointerGetAttributes(&attr_end, last_byte) != cudaSuccess || attr_end.type != cudaMemoryTypeHost) {
+    cudaGetLastError();
+    return failf(MOE_ERR_INVALID_ARG, "the host store must be page-locked (cudaHostAlloc or cudaHostRegister)");
+  }
+  moe_stream_cache* c = new moe_stream_cache;
+  c->host = static_cast<const uint8_t*>(host_pinned_experts);
+  return finish_create(c, cfg, n_layers, n_slots, out);
+}
+
+moe_status moe_stream_create_file(const moe_config* cfg, int n_layers, const char* path, int direct_io, int n_slots,
+                                  int n_read_threads, moe_stream_cache** out) {
+  if (!out) return failf(MOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!cfg) return failf(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  const size_t blob = moe_packed_expert_bytes(cfg);
+  if (blob == 0 || cfg->n_experts <= 0) return failf(MOE_ERR_UNSUPPORTED, "unsupported shape");
+  if (n_layers < 1 || n_slots < 1 || n_read_threads < 1 || n_read_threads > 64)
+    return failf(MOE_ERR_INVALID_ARG, "n_layers and n_slots must be >= 1, n_read_threads in [1, 64]");
+  if (!path) return failf(MOE_ERR_INVALID_ARG, "path is NULL");
+  if (direct_io && blob % 4096)
+    return failf(MOE_ERR_UNSUPPORTED, "direct reads need blobs of a multiple of 4096 bytes (this shape: %zu)", blob);
+  const int fd = open(path, O_RDONLY | (direct_io ? O_DIRECT : 0));
+  if (fd < 0) return failf(MOE_ERR_IO, "cannot open the store file %s: %s", path, strerror(errno));
+  struct stat sb;
+  const size_t need = blob * (size_t)cfg->n_experts * (size_t)n_layers;
+  if (fstat(fd, &sb) != 0 || (size_t)sb.st_size < need) {
+    close(fd);
+    return failf(MOE_ERR_INVALID_ARG, "the store file holds %lld bytes; %d layers of %d experts need %zu",
+                 (long long)sb.st_size, n_layers, cfg->n_experts, need);
+  }
+  moe_stream_cache* c = new moe_stream_cache;
+  c->fd = fd;
+  bool okk = true;
+  for (int i = 0; i < kFileStage && okk; ++i)
+    okk = cudaHostAlloc(reinterpret_cast<void**>(&c->fstage[i]), blob, cudaHostAllocDefault) == cudaSuccess &&
+          cudaEventCreateWithFlags(&c->fstage_ev[i], cudaEventDisableTiming) == cudaSuccess;
+  if (!okk) {
+    cudaGetLastError();
+    destroy_parts(c);
+    delete c;
+    return failf(MOE_ERR_OOM, "could not allocate the store file's pinned staging buffers");
+  }
+  c->io.start(n_read_threads);
+  return finish_create(c, cfg, n_layers, n_slots, out);
+}
+
+moe_status moe_stream_file_stats(const moe_stream_cache* c, uint64_t* reads, uint64_t* read_bytes,
+                                 double* read_ms) {
+  if (!c) return failf(MOE_ERR_INVALID_ARG, "cache is NULL");
+  std::lock_guard<std::mutex> lk(const_cast<moe_stream_cache*>(c)->mu);
+  if (reads) *reads = c->reads;
+  if (read_bytes) *read_bytes = c->read_bytes;
+  if (read_ms) *read_ms = (double)c->read_ns * 1e-6;
+  return MOE_OK;
+}
+
 moe_status moe_stream_prefetch(moe_stream_cache* c, int layer, const int32_t* ids, int n, cudaStream_t copy_stream) {
   if (!c) return failf(MOE_ERR_INVALID_ARG, "cache is NULL");
   std::lock_guard<std::mutex> lk(c->mu);
   moe_status s = check_ids(c, layer, ids, n);
   if (s != MOE_OK) return s;
   DeviceGuard dg(c->device);
+  std::vector<Fill> fills;
   for (int i = 0; i < n; ++i) {
     const int v = c->pol.prefetch(layer, ids[i]);
-    if (v >= 0 && (s = fill_slot(c, v, layer, ids[i], copy_stream)) != MOE_OK) {
-      --c->pol.prefetches;  // not issued
-      return s;
-    }
+    if (v >= 0) fills.push_back(Fill{v, layer, ids[i]});
   }
-  return MOE_OK;
+  int issued = 0;
+  s = do_fills(c, fills, copy_stream, &issued);
+  if (s != MOE_OK) c->pol.prefetches -= (uint64_t)(fills.size() - issued);  // not issued
+  return s;
 }
 
 moe_status moe_stream_resolve(moe_stream_cache* c, int layer, const int32_t* idx, int n, const void** expert_ptr_dev,
@@ -243,24 +519,33 @@ moe_status moe_stream_resolve(moe_stream_cache* c, int layer, const int32_t* idx
     return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
   const void** tab = c->stage[sb];
   std::memset(tab, 0, sizeof(void*) * (size_t)c->E);
+  std::vector<Fill> fills;
   for (int i = 0; i < n; ++i) {
     const int e = idx[i];
     if (tab[e]) continue;  // already resolved in this call
     bool fill = false;
     const int slot = c->pol.resolve(layer, e, &fill);
-    if (slot < 0)
+    if (slot < 0) {
+      for (const Fill& f : fills) c->pol.evict(f.slot);
+      c->pol.misses -= fills.size();
+      c->pol.release();
       return failf(MOE_ERR_OOM, "the cache's %d slots cannot hold the distinct experts of one call", c->S);
+    }
     if (fill) {
-      if ((s = fill_slot(c, slot, layer, e, st)) != MOE_OK) {
-        --c->pol.misses;  // not issued
-        c->pol.release();  // no layer will read this call's slots
-        return s;
-      }
+      fills.push_back(Fill{slot, layer, e});
     } else if ((err = cudaStreamWaitEvent(st, c->ready[slot], 0)) != cudaSuccess) {
+      for (const Fill& f : fills) c->pol.evict(f.slot);
+      c->pol.misses -= fills.size();
       c->pol.release();
       return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
     }
     tab[e] = c->slots + (size_t)slot * c->blob;
+  }
+  int issued = 0;
+  if ((s = do_fills(c, fills, st, &issued)) != MOE_OK) {
+    c->pol.misses -= (uint64_t)(fills.size() - issued);  // not issued
+    c->pol.release();  // no layer will read this call's slots
+    return s;
   }
   if ((err = cudaMemcpyAsync(expert_ptr_dev, tab, sizeof(void*) * (size_t)c->E, cudaMemcpyHostToDevice, st)) !=
           cudaSuccess ||
@@ -292,6 +577,58 @@ moe_status moe_stream_inject_fault(moe_stream_cache* c, int what, int countdown)
     return MOE_OK;
   }
   return failf(MOE_ERR_INVALID_ARG, "unknown fault %d", what);
+}
+
+moe_status moe_stream_enable_copy_timing(moe_stream_cache* c, int on) {
+  if (!c) return failf(MOE_ERR_INVALID_ARG, "cache is NULL");
+  std::lock_guard<std::mutex> lk(c->mu);
+  DeviceGuard dg(c->device);
+  if (on && !c->ref && cudaEventCreate(&c->ref) != cudaSuccess) {
+    cudaGetLastError();
+    return failf(MOE_ERR_OOM, "could not create a timing event");
+  }
+  c->timing = on != 0;
+  return MOE_OK;
+}
+
+moe_status moe_stream_copy_timing(moe_stream_cache* c, moe_stream_copy_times* out) {
+  if (!c || !out) return failf(MOE_ERR_INVALID_ARG, "NULL pointer");
+  std::lock_guard<std::mutex> lk(c->mu);
+  DeviceGuard dg(c->device);
+  std::vector<std::pair<double, double>> iv;
+  double sum = 0.0;
+  for (auto& pr : c->timed) {
+    float a = 0.f, b = 0.f;
+    cudaError_t err = cudaEventSynchronize(pr.second);
+    if (err == cudaSuccess) err = cudaEventElapsedTime(&a, c->ref, pr.first);
+    if (err == cudaSuccess) err = cudaEventElapsedTime(&b, c->ref, pr.second);
+    if (err != cudaSuccess) return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
+    iv.emplace_back(a, b);
+    sum += b - a;
+  }
+  std::sort(iv.begin(), iv.end());
+  double busy = 0.0, cur_a = 0.0, cur_b = -1.0;
+  for (auto& x : iv) {
+    if (x.first > cur_b) {
+      if (cur_b > cur_a) busy += cur_b - cur_a;
+      cur_a = x.first;
+      cur_b = x.second;
+    } else if (x.second > cur_b) {
+      cur_b = x.second;
+    }
+  }
+  if (cur_b > cur_a) busy += cur_b - cur_a;
+  out->busy_ms = busy;
+  out->copy_ms = sum;
+  out->copies = c->timed.size();
+  out->bytes = c->timed_bytes;
+  for (auto& pr : c->timed) {
+    c->spare.push_back(pr.first);
+    c->spare.push_back(pr.second);
+  }
+  c->timed.clear();
+  c->timed_bytes = 0;
+  return MOE_OK;
 }
 
 moe_status moe_stream_stats(const moe_stream_cache* c, moe_stream_counters* out) {

@@ -105,6 +105,19 @@ def activations(s: LayerShape, step: int = 0, tokens: int = None, replica: int =
     return x, res
 
 
+def prenorm_inputs(s: LayerShape, step: int = 0, tokens: int = None, replica: int = 0):
+    """bf16 bit patterns of a residual stream h [T][H] (normal values, a
+    per-token scale e^U(-1, 2), every 64th channel 8x larger) and of the
+    pre-norm weight gamma_pre [H] (1 + 0.02 N(0, 1))."""
+    T = s.tokens if tokens is None else tokens
+    g = rng(s.seed, replica, "prenorm", step, T, s.hidden)
+    h = g.standard_normal((T, s.hidden), dtype=np.float32)
+    h *= np.exp(g.uniform(-1.0, 2.0, (T, 1))).astype(np.float32)
+    h[:, ::64] *= np.float32(8.0)
+    gp = 1.0 + g.standard_normal(s.hidden, dtype=np.float32) * np.float32(0.02)
+    return f32_to_bf16_bits(h), f32_to_bf16_bits(gp)
+
+
 def torch_expert_weights(s: LayerShape, e0: int, n: int, replica: int, device):
     """Device-side fp32 expert weights for experts e0..e0+n-1 (benchmark scale).
 

@@ -109,8 +109,17 @@ def test_argument_checks_without_gpu():
     st = lib.moe_layer_forward_traced(C.byref(good), C.byref(wts), 16, 16, 9, 16, 16, 256, 1 << 20, 16, 1 << 20,
                                       None)
     assert st == 2 and "at most" in M.last_error()
-    # the workspace of a long batch is one chunk's
-    assert lib.moe_layer_workspace_bytes(C.byref(good), 2048) == lib.moe_layer_workspace_bytes(C.byref(good), 8)
+    # below 32 tokens the workspace is one chunk's (the fused kernel's
+    # chunks); from 32 it covers the batched path, which grows with T
+    assert lib.moe_layer_workspace_bytes(C.byref(good), 31) == lib.moe_layer_workspace_bytes(C.byref(good), 8)
+    assert lib.moe_layer_workspace_bytes(C.byref(good), 2048) == lib.moe_layer_batched_workspace_bytes(
+        C.byref(good), 2048)
+    assert lib.moe_layer_batched_workspace_bytes(C.byref(good), 2048) > \
+        2 * lib.moe_layer_batched_workspace_bytes(C.byref(good), 512)
+    # the batched call checks its arguments before any device work too
+    st = lib.moe_layer_forward_batched(C.byref(good), C.byref(wts), 16, 16, 40, 16, 16, None, None, 256, 1 << 20,
+                                       None)
+    assert st == 1 and "NULL" in M.last_error()
     # T == 0 is a no-op that touches nothing
     st = lib.moe_layer_forward(C.byref(good), None, None, None, 0, None, None, None, None, None, 0, None)
     assert st == 0

@@ -140,6 +140,19 @@ def test_layer_is_deterministic_and_host_path_matches(M):
     M.moe_layer_forward_host(dl.cfg, dl.wts, xh, rh, hh, yh, hw)
     assert np.array_equal(hh.numpy().view(np.uint16), a[0])
     assert np.array_equal(yh.numpy().view(np.uint16), a[1])
+    # the asynchronous calls: separate buffers, and x|residual, h_out|y_norm
+    # packed in one host buffer each (one copy each way)
+    hh2, yh2 = torch.zeros_like(hh).pin_memory(), torch.zeros_like(yh).pin_memory()
+    M.moe_layer_forward_host_async(dl.cfg, dl.wts, xh, rh, hh2, yh2, hw)
+    torch.cuda.synchronize()
+    assert np.array_equal(hh2.numpy().view(np.uint16), a[0])
+    assert np.array_equal(yh2.numpy().view(np.uint16), a[1])
+    inp = torch.from_numpy(np.stack([x, res]).view(np.int16)).pin_memory()
+    out = torch.zeros_like(inp).pin_memory()
+    M.moe_layer_forward_host_packed(dl.cfg, dl.wts, inp, out, hw)
+    torch.cuda.synchronize()
+    assert np.array_equal(out[0].numpy().view(np.uint16), a[0])
+    assert np.array_equal(out[1].numpy().view(np.uint16), a[1])
 
 
 def test_layer_uniform_zero_router_picks_lowest_indices(M):

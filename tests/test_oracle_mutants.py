@@ -25,6 +25,8 @@ MUTANTS = {
     10: ("router reads Wr transposed", [P.test_router_hand_worked]),
     11: ("router drops the bias", [P.test_router_hand_worked]),
     12: ("silu replaced by the plain sigmoid", [P.test_expert_ffn_hand_worked, P.test_shared_ffn_hand_worked]),
+    13: ("pre-norm divides by the sum, not the mean", [P.test_prenorm_hand_worked, P.test_prenorm_closed_forms]),
+    14: ("pre-norm drops gamma", [P.test_prenorm_hand_worked, P.test_prenorm_closed_forms]),
 }
 
 

@@ -324,6 +324,72 @@ def test_rmsnorm_closed_form():
     np.testing.assert_allclose(yn[1], np.where(np.arange(H) % 2 == 0, -cval, cval) * inv * g, rtol=1e-14)
 
 
+# ---- RMSNorm before the layer ------------------------------------------------
+
+def test_prenorm_hand_worked():
+    # H = 64, eps = 0: h = (1, 2, 2, 4, 0, ...), sum of squares 25, mean 25/64,
+    # root 5/8, so inv = 1.6; gamma = 1 on the first two columns, 0.5 after
+    c = O.cfg(64, 64, 4, 2, eps=0.0)
+    h = np.zeros((1, 64), np.float32)
+    h[0, :4] = [1, 2, 2, 4]
+    g = np.full(64, 0.5, np.float32)
+    g[:2] = 1.0
+    x = O.prenorm(c, S.f32_to_bf16_bits(h), S.f32_to_bf16_bits(g))
+    want = np.zeros(64)
+    want[:4] = [1.6, 3.2, 1.6, 3.2]
+    np.testing.assert_allclose(x[0], want, rtol=1e-15, atol=0)
+
+
+def test_prenorm_closed_forms():
+    H = 128
+    c = O.cfg(H, 64, 4, 2)
+    eps = np.float64(np.float32(1e-6))
+    gamma = S.f32_to_bf16_bits(np.linspace(0.5, 2.0, H).astype(np.float32))
+    g = O.bf16_to_f64(gamma)
+    # one-hot token: x_j = a / sqrt(a^2 / H + eps) * gamma_j, zero elsewhere
+    a, j = 3.0, 17
+    h1 = np.zeros(H, np.float32)
+    h1[j] = a
+    # constant token: x = v / sqrt(v^2 + eps) * gamma
+    v = -0.375
+    h2 = np.full(H, v, np.float32)
+    x = O.prenorm(c, S.f32_to_bf16_bits(np.stack([h1, h2])), gamma)
+    want1 = np.zeros(H)
+    want1[j] = a / np.sqrt(a * a / H + eps) * g[j]
+    np.testing.assert_allclose(x[0], want1, rtol=1e-14, atol=0)
+    np.testing.assert_allclose(x[1], v / np.sqrt(v * v + eps) * g, rtol=1e-14)
+
+
+def test_f64_to_bf16_single_rounding():
+    # bf16 keeps 8 significant bits: steps of 2^-7 just above 1
+    u = 2.0**-8
+    cases = {1.0: 0x3F80, 1.0 + u: 0x3F80,          # tie, to even (down)
+             1.0 + 3 * u: 0x3F82,                    # tie, to even (up)
+             1.0 + u + 2.0**-40: 0x3F81,             # just above the tie: up
+             -2.0: 0xC000, 0.0: 0x0000, 2.0**-130: 0x0008,  # subnormal: 8 units of 2^-133
+             3.0e38: 0x7F62}
+    for v, want in cases.items():
+        assert int(O.f64_to_bf16(np.array([v]))[0]) == want, v
+    # on values that are floats, the same as the float rounding
+    rng = np.random.default_rng(5)
+    f = (rng.standard_normal(2000) * np.exp(rng.uniform(-20, 20, 2000))).astype(np.float32)
+    np.testing.assert_array_equal(O.f64_to_bf16(f.astype(np.float64)), S.f32_to_bf16_bits(f))
+
+
+def test_prenorm_layer_composes():
+    # the prenorm layer is the plain layer on x = bf16(prenorm(h)) with residual h
+    s, c, blobs, d, x, res = _tiny_layer()
+    gp = S.f32_to_bf16_bits(np.linspace(0.8, 1.2, c.hidden).astype(np.float32))
+    xn, idx, w, h, yn = O.layer_forward_prenorm(c, blobs, d["wr"], None, d["shared_gate"], d["shared_up"],
+                                                d["shared_down"], d["gamma"], gp, res)
+    xr = O.prenorm(c, res, gp)
+    assert np.all(np.abs(O.bf16_to_f64(xn) - xr) <= np.abs(xr) * 2.0**-8)
+    idx2, w2, h2, yn2 = O.layer_forward(c, blobs, d["wr"], None, d["shared_gate"], d["shared_up"],
+                                        d["shared_down"], d["gamma"], xn, res)
+    np.testing.assert_array_equal(idx, idx2)
+    np.testing.assert_array_equal(h, h2)
+
+
 def test_given_routing_overrides():
     s, c, blobs, d, x, res = _tiny_layer()
     idx_in = np.array([[3, 4], [5, 6], [7, 8]], np.int32)

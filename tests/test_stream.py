@@ -476,3 +476,75 @@ def test_stream_copy_failure_is_reported_and_the_cache_recovers(M):
         M.moe_stream_inject_fault(cache, M.MOE_FAULT_NONE)
         torch.cuda.synchronize()
         M.moe_stream_destroy(cache)
+
+
+# ---- file-backed store (the pages' SSD tier) -------------------------------------------
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("direct", [False, True], ids=["page_cache", "direct_io"])
+def test_file_store_matches_resident(M, tmp_path, direct):
+    """The same multi-layer run with the cache's store in a file (parallel
+    pread into pinned staging, then the copy to the slot): every layer's
+    outputs equal the resident routed call's bit for bit, and the reads
+    counted equal the misses plus the prefetches."""
+    import torch
+    if direct:
+        s = replace(S.QWEN_4BIT, name="h4096_e16_k4_i1024_4bit", n_experts=16, tokens=1)  # 4096-byte blobs
+    else:
+        s = replace(S.TINY, tokens=2)
+    lay = _Layers(M, s, n_layers=2, device_pack=direct)
+    path = tmp_path / "experts.bin"
+    lay.store.numpy().tofile(str(path))
+    try:
+        cache = M.moe_stream_create_file(lay.cfg, 2, str(path), 6, direct_io=direct, n_read_threads=4)
+    except M.MoeError as e:
+        if direct and e.status == M.STATUS_BY_NAME["MOE_ERR_IO"]:
+            pytest.skip("O_DIRECT is not available on this file system: %s" % e)
+        raise
+    E = s.n_experts
+    table = torch.zeros(E, dtype=torch.int64, device="cuda")
+    ws = torch.zeros(M.moe_layer_workspace_bytes(lay.cfg, 8), dtype=torch.uint8, device="cuda")
+    M.moe_workspace_init(ws)
+    side = torch.cuda.Stream()
+    try:
+        for step in range(3):
+            for l in range(2):
+                dl = lay.layers[l]
+                x, res = S.activations(s, step=step, replica=l)
+                _, idx, w = dl.router(x)
+                xd, rd, idd, wd = to_dev_bits(x), to_dev_bits(res), _dev(idx), _dev(w)
+                h1, y1 = torch.empty_like(xd), torch.empty_like(xd)
+                M.moe_layer_forward_routed(lay.cfg, dl.wts, xd, rd, idd, wd, h1, y1, dl.ws)
+                M.moe_stream_resolve(cache, l, idx.ravel(), table)
+                wts = M.layer_weights(table, None, None, dl.sg, dl.su, dl.sd, dl.gamma)
+                h2, y2 = torch.empty_like(xd), torch.empty_like(xd)
+                M.moe_layer_forward_routed(lay.cfg, wts, xd, rd, idd, wd, h2, y2, ws)
+                if l == 0:
+                    _, pred, _ = lay.layers[1].router(x)
+                    M.moe_stream_prefetch(cache, 1, pred.ravel(), copy_stream=side)
+                torch.cuda.synchronize()
+                assert M.moe_device_error(ws)[0] == 0
+                assert np.array_equal(from_dev_bits(h1), from_dev_bits(h2)), (step, l)
+                assert np.array_equal(from_dev_bits(y1), from_dev_bits(y2)), (step, l)
+        st = M.moe_stream_stats(cache)
+        fs = M.moe_stream_file_stats(cache)
+        assert fs["reads"] == st["misses"] + st["prefetches"] and fs["reads"] > 0
+        assert fs["read_bytes"] == fs["reads"] * lay.nb
+    finally:
+        torch.cuda.synchronize()
+        M.moe_stream_destroy(cache)
+
+
+@pytest.mark.gpu
+def test_file_store_rejects_a_short_or_missing_file(M, tmp_path):
+    s = replace(S.TINY, tokens=2)
+    cfg = mcfg(s)
+    nb = M.moe_packed_expert_bytes(cfg)
+    path = tmp_path / "short.bin"
+    np.zeros(2 * s.n_experts * nb - 1, np.uint8).tofile(str(path))
+    with pytest.raises(M.MoeError) as ei:
+        M.moe_stream_create_file(cfg, 2, str(path), 4)
+    assert ei.value.status == M.STATUS_BY_NAME["MOE_ERR_INVALID_ARG"] and "file holds" in str(ei.value)
+    with pytest.raises(M.MoeError) as ei:
+        M.moe_stream_create_file(cfg, 1, str(tmp_path / "missing.bin"), 4)
+    assert ei.value.status == M.STATUS_BY_NAME["MOE_ERR_IO"]
