@@ -470,14 +470,21 @@ uint16_t orc_f64_to_bf16(double v) {
  * y_norm = h_out / sqrt(mean(h_out^2) + eps) * gamma.
  * The pages fuse "combine + residual + normalization" into one GPU kernel
  * whose output feeds the next layer ([toolarium] "Оптимизации, которые
- * сработали"; [hakusoku] "主要技術", deferred expert computation). */
-void orc_layer_forward(const orc_cfg* c, const uint8_t* const* experts,
-                       const uint16_t* wr_bf16, const float* bias,
-                       const uint16_t* shared_gate, const uint16_t* shared_up,
-                       const uint16_t* shared_down, const uint16_t* gamma_bf16,
-                       const uint16_t* x_bf16, const uint16_t* residual_bf16, int T,
-                       const int32_t* idx_in, const double* w_in, int32_t* idx,
-                       float* w, double* h_out, double* y_norm) {
+ * сработали"; [hakusoku] "主要技術", deferred expert computation).
+ * The shared expert is the bf16 FFN, or, when shared_blob is given, the same
+ * FFN with packed weights as the routed experts; when shared_gate_w (bf16
+ * [H]) is given its output is scaled by sigmoid(x . shared_gate_w) (the
+ * pages name the shared expert next to the K routed ones and compute it in
+ * the command with the router, [hakusoku] "モデルアーキテクチャ",
+ * "パイプライン概要"; neither form is printed there). */
+void orc_layer_forward_ex(const orc_cfg* c, const uint8_t* const* experts,
+                          const uint16_t* wr_bf16, const float* bias,
+                          const uint16_t* shared_gate, const uint16_t* shared_up,
+                          const uint16_t* shared_down, const uint8_t* shared_blob,
+                          const uint16_t* shared_gate_w, const uint16_t* gamma_bf16,
+                          const uint16_t* x_bf16, const uint16_t* residual_bf16, int T,
+                          const int32_t* idx_in, const double* w_in, int32_t* idx,
+                          float* w, double* h_out, double* y_norm) {
   int H = c->hidden, E = c->n_experts, K = c->top_k;
   int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)T * K + 4);
   double* wsel = (double*)malloc(sizeof(double) * (size_t)T * K + 8);
@@ -507,8 +514,17 @@ void orc_layer_forward(const orc_cfg* c, const uint8_t* const* experts,
       for (int r = 0; r < H; ++r) h[r] += wsel[(size_t)t * K + k] * y[r];
     }
     if (c->has_shared) {
-      orc_shared_ffn(c, shared_gate, shared_up, shared_down, x, y);
-      for (int r = 0; r < H; ++r) h[r] += y[r];
+      if (shared_blob && ORC_MUTANT != 17)
+        orc_expert_ffn(c, shared_blob, x, y);
+      else
+        orc_shared_ffn(c, shared_gate, shared_up, shared_down, x, y);
+      double gs = 1.0;
+      if (shared_gate_w) {
+        double z = 0.0;
+        for (int r = 0; r < H; ++r) z += x[r] * orc_bf16_to_f64(shared_gate_w[r]);
+        gs = ORC_MUTANT == 15 ? z / (1.0 + exp(-z)) : 1.0 / (1.0 + exp(-z));
+      }
+      for (int r = 0; r < H; ++r) h[r] += (ORC_MUTANT == 16 ? 1.0 : gs) * y[r];
     }
     double ss = 0.0;
     for (int r = 0; r < H; ++r) ss += h[r] * h[r];
@@ -524,4 +540,15 @@ void orc_layer_forward(const orc_cfg* c, const uint8_t* const* experts,
   free(x);
   free(wsel);
   free(sel);
+}
+
+void orc_layer_forward(const orc_cfg* c, const uint8_t* const* experts,
+                       const uint16_t* wr_bf16, const float* bias,
+                       const uint16_t* shared_gate, const uint16_t* shared_up,
+                       const uint16_t* shared_down, const uint16_t* gamma_bf16,
+                       const uint16_t* x_bf16, const uint16_t* residual_bf16, int T,
+                       const int32_t* idx_in, const double* w_in, int32_t* idx,
+                       float* w, double* h_out, double* y_norm) {
+  orc_layer_forward_ex(c, experts, wr_bf16, bias, shared_gate, shared_up, shared_down, NULL, NULL,
+                       gamma_bf16, x_bf16, residual_bf16, T, idx_in, w_in, idx, w, h_out, y_norm);
 }

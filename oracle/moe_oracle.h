@@ -117,6 +117,18 @@ void orc_layer_forward(const orc_cfg* c, const uint8_t* const* experts,
                        const uint16_t* x_bf16, const uint16_t* residual_bf16, int T,
                        const int32_t* idx_in, const double* w_in, int32_t* idx,
                        float* w, double* h_out, double* y_norm);
+/* The same layer with the shared expert's two optional forms: shared_blob
+ * (a packed blob like the routed experts') replaces the bf16 weights, and
+ * shared_gate_w (bf16 [H]) scales the shared output by sigmoid(x . g).
+ * Either may be NULL; with both NULL this is orc_layer_forward. */
+void orc_layer_forward_ex(const orc_cfg* c, const uint8_t* const* experts,
+                          const uint16_t* wr_bf16, const float* bias,
+                          const uint16_t* shared_gate, const uint16_t* shared_up,
+                          const uint16_t* shared_down, const uint8_t* shared_blob,
+                          const uint16_t* shared_gate_w, const uint16_t* gamma_bf16,
+                          const uint16_t* x_bf16, const uint16_t* residual_bf16, int T,
+                          const int32_t* idx_in, const double* w_in, int32_t* idx,
+                          float* w, double* h_out, double* y_norm);
 
 #ifdef __cplusplus
 }

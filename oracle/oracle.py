@@ -66,6 +66,8 @@ def lib(path=None):
         _lib.orc_shared_ffn.argtypes = [cfgp, P, P, P, P, P]
         _lib.orc_layer_forward.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, C.c_int,
                                            P, P, P, P, P, P]
+        _lib.orc_layer_forward_ex.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, C.c_int,
+                                              P, P, P, P, P, P]
     return _lib
 
 
@@ -196,8 +198,11 @@ def shared_ffn(c, wg, wu, wd, x):
 
 
 def layer_forward(c, experts, wr, bias, shared_gate, shared_up, shared_down, gamma,
-                  x, residual, idx_in=None, w_in=None):
-    """experts: list (length E) of uint8 blobs (entries may repeat)."""
+                  x, residual, idx_in=None, w_in=None, shared_blob=None, shared_gate_w=None):
+    """experts: list (length E) of uint8 blobs (entries may repeat).
+    shared_blob: the shared expert packed like the routed ones (replaces the
+    bf16 weights); shared_gate_w: bf16 [H], the shared output scaled by
+    sigmoid(x . shared_gate_w)."""
     x = _c(x, np.uint16)
     T = x.shape[0]
     blobs = [_c(b, np.uint8) for b in experts]
@@ -212,10 +217,12 @@ def layer_forward(c, experts, wr, bias, shared_gate, shared_up, shared_down, gam
     bb = None if bias is None else _c(bias, np.float32)
     ii = None if idx_in is None else _c(idx_in, np.int32)
     wi = None if w_in is None else _c(w_in, np.float64)
-    lib().orc_layer_forward(C.byref(c), C.cast(ptrs, C.c_void_p), _p(_c(wr, np.uint16)),
-                            _p(bb), _p(sg), _p(su), _p(sd), _p(_c(gamma, np.uint16)),
-                            _p(x), _p(_c(residual, np.uint16)), T, _p(ii), _p(wi),
-                            _p(idx), _p(w), _p(h), _p(yn))
+    sb = None if shared_blob is None else _c(shared_blob, np.uint8)
+    sgw = None if shared_gate_w is None else _c(shared_gate_w, np.uint16)
+    lib().orc_layer_forward_ex(C.byref(c), C.cast(ptrs, C.c_void_p), _p(_c(wr, np.uint16)),
+                               _p(bb), _p(sg), _p(su), _p(sd), _p(sb), _p(sgw), _p(_c(gamma, np.uint16)),
+                               _p(x), _p(_c(residual, np.uint16)), T, _p(ii), _p(wi),
+                               _p(idx), _p(w), _p(h), _p(yn))
     return idx, w, h, yn
 
 

@@ -27,6 +27,9 @@ MUTANTS = {
     12: ("silu replaced by the plain sigmoid", [P.test_expert_ffn_hand_worked, P.test_shared_ffn_hand_worked]),
     13: ("pre-norm divides by the sum, not the mean", [P.test_prenorm_hand_worked, P.test_prenorm_closed_forms]),
     14: ("pre-norm drops gamma", [P.test_prenorm_hand_worked, P.test_prenorm_closed_forms]),
+    15: ("shared gate uses silu, not the sigmoid", [P.test_shared_gate_closed_forms]),
+    16: ("shared gate ignored", [P.test_shared_gate_closed_forms]),
+    17: ("packed shared expert ignored for the bf16 weights", [P.test_packed_shared_is_an_expert]),
 }
 
 

@@ -324,6 +324,48 @@ def test_rmsnorm_closed_form():
     np.testing.assert_allclose(yn[1], np.where(np.arange(H) % 2 == 0, -cval, cval) * inv * g, rtol=1e-14)
 
 
+# ---- the shared expert's gate and packed form ---------------------------------
+
+def _shared_variants(gate_w=None, shared_blob=None, has_shared=1):
+    s, c, blobs, d, x, res = _tiny_layer()
+    c = O.cfg(c.hidden, c.inter, c.n_experts, c.top_k, bits=c.bits, has_shared=has_shared)
+    idx_in = np.array([[1, 2], [3, 4], [5, 0]], np.int32)
+    w_in = np.array([[0.6, 0.4], [0.25, 0.75], [0.5, 0.5]])
+    _, _, h, _ = O.layer_forward(c, blobs, d["wr"], None, d["shared_gate"], d["shared_up"], d["shared_down"],
+                                 d["gamma"], x, res, idx_in=idx_in, w_in=w_in, shared_blob=shared_blob,
+                                 shared_gate_w=gate_w)
+    return h, x, blobs
+
+
+def test_shared_gate_closed_forms():
+    # the gate scales the shared output by sigmoid(x . g): 1/2 at g = 0;
+    # with g = +-sign(x) the logit is +-sum|x| (about 200 here), so the
+    # gate is 1 (the ungated layer) or 0 (the layer without a shared expert)
+    h_plain, x, _ = _shared_variants()
+    h_none, _, _ = _shared_variants(has_shared=0)
+    H = x.shape[1]
+    h_half, _, _ = _shared_variants(gate_w=np.zeros(H, np.uint16))
+    np.testing.assert_allclose(h_half, h_none + 0.5 * (h_plain - h_none), rtol=1e-12, atol=1e-13)
+    for t in range(x.shape[0]):
+        sgn = np.where(O.bf16_to_f64(x[t]) >= 0, 1.0, -1.0).astype(np.float32)
+        up, _, _ = _shared_variants(gate_w=S.f32_to_bf16_bits(sgn))
+        dn, _, _ = _shared_variants(gate_w=S.f32_to_bf16_bits(-sgn))
+        assert np.sum(np.abs(O.bf16_to_f64(x[t]))) > 100
+        np.testing.assert_allclose(up[t], h_plain[t], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(dn[t], h_none[t], rtol=1e-12, atol=1e-13)
+
+
+def test_packed_shared_is_an_expert():
+    # the packed shared expert adds expert_ffn(blob, x) with weight 1
+    _, x, blobs = _shared_variants()
+    h_none, _, _ = _shared_variants(has_shared=0)
+    h_pk, _, _ = _shared_variants(shared_blob=blobs[9])
+    c = O.cfg(256, 128, 16, 2)
+    for t in range(x.shape[0]):
+        ys = O.expert_ffn(c, blobs[9], O.bf16_to_f64(x[t]))
+        np.testing.assert_allclose(h_pk[t], h_none[t] + ys, rtol=1e-12, atol=1e-13)
+
+
 # ---- RMSNorm before the layer ------------------------------------------------
 
 def test_prenorm_hand_worked():
