@@ -155,6 +155,15 @@ typedef struct {
   const void* shared_up;         /* bf16 [I][H] */
   const void* shared_down;       /* bf16 [H][I] */
   const void* gamma;             /* bf16 [H], RMSNorm weight */
+  /* Optional forms of the shared expert (both NULL: the bf16 FFN above with
+   * weight 1).  The pages name a shared expert next to the K routed ones and
+   * compute it in the GPU command with the router (hakusoku
+   * "モデルアーキテクチャ", "パイプライン概要") without printing its form. */
+  const void* shared_out_gate;   /* bf16 [H] or NULL: the shared output is scaled by
+                                    sigmoid(x . shared_out_gate) (fp32 dot) */
+  const void* shared_packed;     /* device blob in the routed experts' packed format
+                                    (moe_pack_experts, 256-B aligned) or NULL: when set it
+                                    replaces shared_gate/up/down, which may then be NULL */
 } moe_layer_weights;
 
 /* Workspace for moe_layer_forward with T tokens (device memory, 256-B

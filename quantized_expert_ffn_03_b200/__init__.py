@@ -46,7 +46,7 @@ class MoeConfig(C.Structure):
 class MoeLayerWeights(C.Structure):
     _fields_ = [("expert_ptr", C.c_void_p), ("router_w", C.c_void_p), ("router_bias", C.c_void_p),
                 ("shared_gate", C.c_void_p), ("shared_up", C.c_void_p), ("shared_down", C.c_void_p),
-                ("gamma", C.c_void_p)]
+                ("gamma", C.c_void_p), ("shared_out_gate", C.c_void_p), ("shared_packed", C.c_void_p)]
 
 
 EXPORTS = {
@@ -235,10 +235,13 @@ def moe_workspace_init(workspace, stream=None):
                                    _stream(stream)))
 
 
-def layer_weights(expert_ptr, router_w, router_bias, shared_gate, shared_up, shared_down, gamma):
-    """expert_ptr: int64 CUDA tensor [E] of blob addresses; the rest CUDA tensors or None."""
+def layer_weights(expert_ptr, router_w, router_bias, shared_gate, shared_up, shared_down, gamma,
+                  shared_out_gate=None, shared_packed=None):
+    """expert_ptr: int64 CUDA tensor [E] of blob addresses; the rest CUDA tensors or None
+    (shared_packed: a uint8 CUDA tensor holding one packed blob)."""
     return MoeLayerWeights(_ptr(expert_ptr), _ptr(router_w), _ptr(router_bias), _ptr(shared_gate),
-                           _ptr(shared_up), _ptr(shared_down), _ptr(gamma))
+                           _ptr(shared_up), _ptr(shared_down), _ptr(gamma), _ptr(shared_out_gate),
+                           _ptr(shared_packed))
 
 
 def moe_layer_forward(cfg, wts, x, residual, h_out, y_norm, idx_out=None, w_out=None,

@@ -53,10 +53,16 @@ moe_status ok() {
       return fail(MOE_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));             \
   } while (0)
 
-constexpr int kMaxGrid = 1024;
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per bounded wait
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The optional forms of the shared expert that a weight set selects.
+void weight_opts(const moe_layer_weights* wts, Layout* L) {
+  L->sgate = (wts && L->has_shared && wts->shared_out_gate) ? 1 : 0;
+  L->spacked = (wts && L->has_shared && wts->shared_packed) ? 1 : 0;
+  L->KP = L->K + L->spacked;
+}
 
 moe_status check_cfg(const moe_config* cfg, Layout* L) {
   if (!cfg) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
@@ -135,10 +141,13 @@ WsPlan ws_plan(const Layout& L, int T) {
   pos = 256 + epoch_region_bytes(L);
   w.hs = pos;
   pos = round_up_256(pos + sizeof(float) * (size_t)T * L.I);
+  // the routed intermediate of K pairs per token, one more when a shared
+  // expert exists (the workspace size does not depend on its form)
+  const size_t kp = (size_t)L.K + (L.has_shared ? 1 : 0);
   w.hf = pos;
-  pos = round_up_256(pos + 4ull * (size_t)T * L.K * L.I);
+  pos = round_up_256(pos + 4ull * (size_t)T * kp * L.I);
   w.hx = pos;
-  pos = round_up_256(pos + sizeof(float) * (size_t)T * L.K * (L.I / 16));
+  pos = round_up_256(pos + sizeof(float) * (size_t)T * kp * (L.I / 16));
   w.total = pos;
   return w;
 }
@@ -149,7 +158,7 @@ WsPlan ws_plan(const Layout& L, int T) {
 // [slot][I]), the routed outputs (fp32 [slot][H]), the shared intermediate
 // (bf16 hi and lo [T][I]) and the shared output (fp32 [T][H]).
 struct BatchPlan {
-  size_t xh, logits, idx, w, slot_token, pair_slot, ch_e, ch_c0, ch_n, nch, hr, y, hs_hi, hs_lo, ys, total;
+  size_t xh, logits, idx, w, slot_token, pair_slot, ch_e, ch_c0, ch_n, nch, sptr, hr, y, hs_hi, hs_lo, ys, total;
   int max_chunks;
 };
 
@@ -175,6 +184,7 @@ BatchPlan batch_plan(const Layout& L, int T) {
   b.ch_c0 = take(4ull * b.max_chunks);
   b.ch_n = take(4ull * b.max_chunks);
   b.nch = take(16);
+  b.sptr = take(16);  // a one-entry pointer table: the packed shared expert
   b.hr = take(2 * TK * L.I);
   b.y = take(4 * TK * L.H);
   b.hs_hi = take(2ull * T * L.I);
@@ -332,22 +342,25 @@ static moe_status layer_forward_chunk(const moe_config* cfg, const moe_layer_wei
   moe_status s = check_cfg(cfg, &L);
   if (s != MOE_OK) return s;
   L.prenorm = gamma_pre ? 1 : 0;
+  weight_opts(wts, &L);
   if (T > chunk_tokens(L)) return fail(MOE_ERR_UNSUPPORTED, "T=%d: at most %d tokens per launch", T, chunk_tokens(L));
-  if (!aligned(gamma_pre, 16) || !aligned(x_out, 16))
+  if (!aligned(gamma_pre, 16) || !aligned(x_out, 16) || (L.sgate && !aligned(wts->shared_out_gate, 16)))
     return fail(MOE_ERR_INVALID_ARG, "bf16 arrays must be 16-byte aligned");
   const bool given = idx_in != nullptr;  // routing given: the router weights are not read
   if (given && !w_in) return fail(MOE_ERR_INVALID_ARG, "NULL routing weights");
   if (!wts || !wts->expert_ptr || (!given && !wts->router_w) || !wts->gamma || !x_bf16 || !residual_bf16 ||
       !h_out_bf16 || !y_norm_bf16)
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  if (L.has_shared && (!wts->shared_gate || !wts->shared_up || !wts->shared_down))
+  if (L.has_shared && !L.spacked && (!wts->shared_gate || !wts->shared_up || !wts->shared_down))
     return fail(MOE_ERR_INVALID_ARG, "has_shared=1 but a shared-expert pointer is NULL");
+  if (L.spacked && !aligned(wts->shared_packed, 256))
+    return fail(MOE_ERR_INVALID_ARG, "the packed shared expert must be 256-byte aligned");
   const void* a16[] = {x_bf16, residual_bf16, h_out_bf16, y_norm_bf16, given ? nullptr : wts->router_w,
                        wts->gamma};
   for (const void* p : a16)
     if (!aligned(p, 16)) return fail(MOE_ERR_INVALID_ARG, "bf16 arrays must be 16-byte aligned");
-  if (L.has_shared && (!aligned(wts->shared_gate, 16) || !aligned(wts->shared_up, 16) ||
-                       !aligned(wts->shared_down, 16)))
+  if (L.has_shared && !L.spacked && (!aligned(wts->shared_gate, 16) || !aligned(wts->shared_up, 16) ||
+                                     !aligned(wts->shared_down, 16)))
     return fail(MOE_ERR_INVALID_ARG, "shared-expert weights must be 16-byte aligned");
   const WsPlan wp = ws_plan(L, T);
   if (!workspace || ws_bytes < wp.total || !aligned(workspace, 256))
@@ -376,6 +389,8 @@ static moe_status layer_forward_chunk(const moe_config* cfg, const moe_layer_wei
   p.gamma = static_cast<const uint16_t*>(wts->gamma);
   p.gamma_pre = static_cast<const uint16_t*>(gamma_pre);
   p.x_out = static_cast<uint16_t*>(x_out);
+  p.sgate = L.sgate ? static_cast<const uint16_t*>(wts->shared_out_gate) : nullptr;
+  p.spacked = L.spacked ? static_cast<const uint8_t*>(wts->shared_packed) : nullptr;
   p.x = static_cast<const uint16_t*>(x_bf16);
   p.res = static_cast<const uint16_t*>(residual_bf16);
   p.h_out = static_cast<uint16_t*>(h_out_bf16);
@@ -417,11 +432,15 @@ static moe_status layer_forward_batched(const moe_config* cfg, const moe_layer_w
   if (!wts || !wts->expert_ptr || !wts->router_w || !wts->gamma || !x_bf16 || !residual_bf16 || !h_out_bf16 ||
       !y_norm_bf16)
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  if (L.has_shared && (!wts->shared_gate || !wts->shared_up || !wts->shared_down))
+  weight_opts(wts, &L);
+  const bool bf16_shared = L.has_shared && !L.spacked;
+  if (bf16_shared && (!wts->shared_gate || !wts->shared_up || !wts->shared_down))
     return fail(MOE_ERR_INVALID_ARG, "has_shared=1 but a shared-expert pointer is NULL");
+  if (L.spacked && !aligned(wts->shared_packed, 256))
+    return fail(MOE_ERR_INVALID_ARG, "the packed shared expert must be 256-byte aligned");
   const void* a16[] = {x_bf16, residual_bf16, h_out_bf16, y_norm_bf16, wts->router_w, wts->gamma,
-                       L.has_shared ? wts->shared_gate : nullptr, L.has_shared ? wts->shared_up : nullptr,
-                       L.has_shared ? wts->shared_down : nullptr};
+                       bf16_shared ? wts->shared_gate : nullptr, bf16_shared ? wts->shared_up : nullptr,
+                       bf16_shared ? wts->shared_down : nullptr, L.sgate ? wts->shared_out_gate : nullptr};
   for (const void* q : a16)
     if (!aligned(q, 16)) return fail(MOE_ERR_INVALID_ARG, "bf16 arrays must be 16-byte aligned");
   const BatchPlan bp = batch_plan(L, T);
@@ -505,7 +524,38 @@ static moe_status layer_forward_batched(const moe_config* cfg, const moe_layer_w
     CUDA_TRY(launch_grouped_gemm(L.bits, 1, 0, r, grid, stream));
   }
   const float* ys = nullptr;
-  if (L.has_shared) {
+  if (L.spacked) {
+    // the packed shared expert on every token: the same dequant GEMMs over
+    // dense chunks of the T tokens, with a one-entry pointer table
+    CUDA_TRY(launch_set_ptr(reinterpret_cast<const void**>(ws + bp.sptr), wts->shared_packed, stream));
+    GemmParams r = g;
+    r.M = L.I;
+    r.K = L.H;
+    r.bits = L.bits;
+    r.expert_ptr = reinterpret_cast<const void* const*>(ws + bp.sptr);
+    r.off_codes[0] = L.off_codes[0];
+    r.off_codes[1] = L.off_codes[1];
+    r.off_scales[0] = L.off_scales[0];
+    r.off_scales[1] = L.off_scales[1];
+    r.b = reinterpret_cast<const uint16_t*>(ws + bp.xh);
+    r.n_cols = T;
+    r.out = ws + bp.hs_hi;  // fp16 [T][I]
+    const int gr = tiles(T, L.I) < grid ? tiles(T, L.I) : grid;
+    CUDA_TRY(launch_grouped_gemm(L.bits, 2, 1, r, gr, stream));
+    GemmParams d = g;
+    d.M = L.H;
+    d.K = L.I;
+    d.bits = L.bits;
+    d.expert_ptr = reinterpret_cast<const void* const*>(ws + bp.sptr);
+    d.off_codes[0] = L.off_codes[2];
+    d.off_scales[0] = L.off_scales[2];
+    d.b = reinterpret_cast<const uint16_t*>(ws + bp.hs_hi);
+    d.n_cols = T;
+    d.out = ws + bp.ys;
+    const int gd = tiles(T, L.H) < grid ? tiles(T, L.H) : grid;
+    CUDA_TRY(launch_grouped_gemm(L.bits, 1, 0, d, gd, stream));
+    ys = reinterpret_cast<const float*>(ws + bp.ys);
+  } else if (L.has_shared) {
     GemmParams r = g;
     r.M = L.I;
     r.K = L.H;
@@ -529,10 +579,12 @@ static moe_status layer_forward_batched(const moe_config* cfg, const moe_layer_w
     CUDA_TRY(launch_grouped_gemm(0, 1, 0, d, gd, stream));
     ys = reinterpret_cast<const float*>(ws + bp.ys);
   }
+  const bool sgate = L.sgate != 0;
   CUDA_TRY(launch_combine(reinterpret_cast<const float*>(ws + bp.y), ys, pair_slot, w,
                           static_cast<const uint16_t*>(residual_bf16), static_cast<const uint16_t*>(wts->gamma), T,
-                          L.H, L.K, L.eps, static_cast<uint16_t*>(h_out_bf16), static_cast<uint16_t*>(y_norm_bf16),
-                          stream));
+                          L.H, L.K, L.eps, static_cast<const uint16_t*>(x_bf16),
+                          sgate ? static_cast<const uint16_t*>(wts->shared_out_gate) : nullptr,
+                          static_cast<uint16_t*>(h_out_bf16), static_cast<uint16_t*>(y_norm_bf16), stream));
   return ok();
 }
 
@@ -559,6 +611,7 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
   if (!wts || !wts->expert_ptr || (!given && !wts->router_w) || !wts->gamma || !x_bf16 || !residual_bf16 ||
       !h_out_bf16 || !y_norm_bf16)
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  weight_opts(wts, &L);
   DeviceInfo di;
   if ((s = device_info(&di)) != MOE_OK) return s;
   const int C = tokens_per_launch(L, di.sms < kMaxGrid ? di.sms : kMaxGrid, chunk_tokens(L));
@@ -670,6 +723,7 @@ moe_status moe_layer_forward_prenorm(const moe_config* cfg, const moe_layer_weig
   if (x_out_bf16 == h_in_bf16 || x_out_bf16 == h_out_bf16 || h_out_bf16 == h_in_bf16)
     return fail(MOE_ERR_INVALID_ARG, "h_in, h_out and x_out must be distinct buffers");
   L.prenorm = 1;
+  weight_opts(wts, &L);
   if (!(T >= kBatchedMinTokens && batched_ok(L))) {
     DeviceInfo di;
     if ((s = device_info(&di)) != MOE_OK) return s;

@@ -42,6 +42,8 @@
 // "Оптимизации, которые сработали").
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "moe_kernels.h"
 #include "moe_device.cuh"
 
@@ -115,13 +117,17 @@ enum { FLAG_TOPK = NGO, FLAG_SCNT, FLAG_NOSS, FLAG_EPOCH };
 // hx: per (pair, 8-row block of I) sum of hi + lo.
 struct DecodeSmem {
   size_t ring, bars, desc, xs, xf, xsum, hs, hf, hx, zero, part, cnt, rpart, rcnt, tk_w, tk_i, eptr, tkbuf, res, gam,
-      gpre, ypart, ys, hacc, inv, flags, spin, total;
+      gpre, sgv, ypart, ys, hacc, inv, flags, spin, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
 
+// Optional shared-memory regions of a layout: bit 0 the pre-norm, bit 1 the
+// shared output gate.
+__host__ __device__ inline int smem_opts(const Layout& L) { return (L.prenorm ? 1 : 0) | (L.sgate ? 2 : 0); }
+
 __host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int E, int H, int I, int nrows, int nslots,
-                                                       uint32_t slot_bytes, int prenorm) {
+                                                       uint32_t slot_bytes, int opts) {
   const RoutedGeo gi = routed_geo(I, 4);
   DecodeSmem s;
   size_t pos = 0;
@@ -166,7 +172,9 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int E, int 
   s.gam = pos;
   pos = align_up(pos + 2ull * nrows, 16);
   s.gpre = pos;  // pre-norm gamma [H] and the consumer warps' partial sums of squares [14][T]
-  pos = align_up(pos + (prenorm ? 2ull * H + 4ull * kConsumerWarps * T : 0ull), 16);
+  pos = align_up(pos + ((opts & 1) ? 2ull * H + 4ull * kConsumerWarps * T : 0ull), 16);
+  s.sgv = pos;  // shared output gate [H], the consumer warps' partial dots [14][T], the gates [T]
+  pos = align_up(pos + ((opts & 2) ? 2ull * H + 4ull * (kConsumerWarps + 1) * T : 0ull), 16);
   s.ypart = pos;
   pos = align_up(pos + sizeof(float) * T * K * gi.U * nrows, 16);
   s.ys = pos;
@@ -184,7 +192,7 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int E, int 
 }
 
 size_t decode_smem_bytes(const Layout& L, int T, int nrows, int nslots, uint32_t slot_bytes) {
-  return decode_smem_plan(T, L.K, L.E, L.H, L.I, nrows, nslots, slot_bytes, L.prenorm).total;
+  return decode_smem_plan(T, L.KP, L.E, L.H, L.I, nrows, nslots, slot_bytes, smem_opts(L)).total;
 }
 
 // ---- small helpers ----------------------------------------------------------------
@@ -767,9 +775,9 @@ __device__ __forceinline__ bool ptab_in_smem(const DecodeParams& p) {
 template <bool TRACE>
 __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, uint16_t* res_s, uint16_t* gam_s,
                              uint64_t* xbar, uint64_t* topkbar, const int* flags, const uint8_t* const* eptr,
-                             uint64_t* ptab, uint16_t* gpre_s) {
+                             uint64_t* ptab, uint16_t* gpre_s, uint16_t* sgv_s) {
   const Layout& L = p.L;
-  const int T = p.T, K = L.K, H = L.H, I = L.I, E = L.E;
+  const int T = p.T, H = L.H, I = L.I, E = L.E;
   const int G = gridDim.x, c = blockIdx.x;
   int r0, r1;
   block_rows(H, c, G, r0, r1);
@@ -780,10 +788,12 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
   // for E <= 512): the routing then finds its blobs without a global round trip
   const uint32_t tb = ptab_in_smem(p) ? (uint32_t)(8 * E) : 0u;
   const uint32_t gb = L.prenorm ? (uint32_t)(2 * H) : 0u;
-  mbar_expect_tx(xbar, xb + (uint32_t)(T + 1) * rb + tb + gb);
+  const uint32_t sb = L.sgate ? (uint32_t)(2 * H) : 0u;
+  mbar_expect_tx(xbar, xb + (uint32_t)(T + 1) * rb + tb + gb + sb);
   bulk_g2s(xs, p.x, xb, xbar);
   if (tb) bulk_g2s(ptab, p.expert_ptr, tb, xbar);
   if (gb) bulk_g2s(gpre_s, p.gamma_pre, gb, xbar);
+  if (sb) bulk_g2s(sgv_s, p.sgate, sb, xbar);
   if (rb > 0) {
 #pragma unroll 1
     for (int t = 0; t < T; ++t) bulk_g2s(res_s + (size_t)t * (r1 - r0), p.res + (size_t)t * H + r0, rb, xbar);
@@ -796,7 +806,8 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
     emit_rows(pr, TILE_ROUTER, reinterpret_cast<const uint8_t*>(p.wr), nullptr, 2u * H, a, b);
   }
   pr.post(F_ARRIVE_R);
-  if (L.has_shared) {
+  const bool bf16_shared = L.has_shared && !L.spacked;
+  if (bf16_shared) {
     range_of(I, c, G, a, b);
     emit_rows(pr, TILE_SHARED_GU, reinterpret_cast<const uint8_t*>(p.sg), reinterpret_cast<const uint8_t*>(p.su),
               2u * H, a, b);
@@ -819,9 +830,10 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
   const size_t os[3] = {L.off_scales[0], L.off_scales[1], L.off_scales[2]};
   const int nrb_i = I / kRowBlock;
   int rbseq = 0;
+  const int KP = L.KP;  // pairs per token (the packed shared expert is pair K)
   if (routed) {
-    // routed gate/up: this block's share of the T*K*(I/8) (pair, row block) items
-    range_of(T * K * nrb_i, c, G, a, b);
+    // routed gate/up: this block's share of the T*KP*(I/16) (pair, row block) items
+    range_of(T * KP * nrb_i, c, G, a, b);
 #pragma unroll 1
     for (int q = a; q < b && pr.ok;) {
       const int pair = q / nrb_i, rb0 = q - pair * nrb_i;
@@ -834,14 +846,14 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
   // the shared expert's down rows of this block: every block's shared
   // intermediate (S) was staged while the routing was found, so they run
   // while the routed intermediate (E) is being completed
-  if (L.has_shared) {
+  if (bf16_shared) {
     pr.pre(F_WAIT_S);
     emit_rows(pr, TILE_SHARED_DOWN, reinterpret_cast<const uint8_t*>(p.sd), nullptr, 2u * I, r0, r1);
   }
   pr.pre(F_WAIT_E);
   if (routed && r1 > r0) {
 #pragma unroll 1
-    for (int pair = 0; pair < T * K && pr.ok; ++pair)
+    for (int pair = 0; pair < T * KP && pr.ok; ++pair)
       emit_routed(pr, TILE_EXPERT_DOWN, L.bits, oc + 2, os + 2, eptr[pair], pair, r0 / kRowBlock, r1 / kRowBlock, 1, gi, 1 << 20,
                   &rbseq);
   }
@@ -862,7 +874,7 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
                          uint32_t* spins) {
   const int lane = threadIdx.x & 31;
   const Layout& L = p.L;
-  const int T = p.T, K = L.K, E = L.E, G = gridDim.x;
+  const int T = p.T, K = L.K, KP = L.KP, E = L.E, G = gridDim.x;
   uint32_t* ctr = p.ctr;
   const uint64_t to = p.timeout_ns;
   uint32_t* sp_evt = spins ? spins + 5 : nullptr;
@@ -873,8 +885,9 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
     // the routing is given: no router barrier, no top-K
 #pragma unroll 1
     for (int j = lane; j < T * K; j += 32) {
-      tk_i[j] = __ldg(p.idx_in + j);
-      tk_w[j] = __ldg(p.w_in + j);
+      const int t = j / K, k = j - t * K;
+      tk_i[t * KP + k] = __ldg(p.idx_in + j);
+      tk_w[t * KP + k] = __ldg(p.w_in + j);
     }
     __syncwarp();
     good = __all_sync(0xffffffffu, ok) ? 1 : 0;
@@ -887,19 +900,28 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
     bool gr = ok;
 #pragma unroll 1
     for (int t = 0; t < T && gr; ++t)
-      gr = warp_topk_poll(p.logits + (size_t)t * E, epoch, E, K, tkbuf, tk_i + t * K, tk_w + t * K, &ctr[5], p.err,
-                          to, sp_grid);
+      gr = warp_topk_poll(p.logits + (size_t)t * E, epoch, E, K, tkbuf, tk_i + t * KP, tk_w + t * KP, &ctr[5], p.err,
+                          to, sp_grid, TRACE ? p.trace + (size_t)blockIdx.x * kTraceEntries + 73 : nullptr);
     good = __all_sync(0xffffffffu, gr) ? 1 : 0;
     __syncwarp();
     if (lane == 0) trace_mark<TRACE>(p, 66);
   }
   if (good) {
 #pragma unroll 1
-    for (int j = lane; j < T * K; j += 32) {
-      const int e = tk_i[j];
-      const void* bp = (e >= 0 && e < E) ? (ptab_in_smem(p) ? reinterpret_cast<const void*>(tkbuf[e])
-                                                             : p.expert_ptr[e])
-                                         : nullptr;
+    for (int j = lane; j < T * KP; j += 32) {
+      // pair K of a token is the packed shared expert (weight 1: its gate,
+      // if any, is applied in the combine)
+      const int t = j / KP, k = j - t * KP;
+      const bool shp = k == K;
+      if (shp) {
+        tk_i[j] = -1;
+        tk_w[j] = 1.f;
+      }
+      const int e = shp ? 0 : tk_i[j];
+      const void* bp = shp ? reinterpret_cast<const void*>(p.spacked)
+                           : (e >= 0 && e < E) ? (ptab_in_smem(p) ? reinterpret_cast<const void*>(tkbuf[e])
+                                                                  : p.expert_ptr[e])
+                                               : nullptr;
       if (bp == nullptr || (reinterpret_cast<uintptr_t>(bp) & 255u)) {
         atomicCAS(p.err, 0u, 2u);
         atomicExch(&ctr[5], 1u);
@@ -907,9 +929,9 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
         good = 0;
       }
       eptr[j] = reinterpret_cast<const uint8_t*>(bp);
-      if (blockIdx.x == 0) {
-        if (p.idx_out) p.idx_out[j] = e;
-        if (p.w_out) p.w_out[j] = tk_w[j];
+      if (blockIdx.x == 0 && !shp) {
+        if (p.idx_out) p.idx_out[t * K + k] = e;
+        if (p.w_out) p.w_out[t * K + k] = tk_w[j];
       }
     }
     good = __all_sync(0xffffffffu, good != 0) ? 1 : 0;
@@ -932,7 +954,7 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
     flags[GO_E] = ge ? 1 : 0;
     if (ge) {
       fence_proxy_async_global();
-      const uint32_t hfb = (uint32_t)(4ull * T * K * L.I), hxb = (uint32_t)(4ull * T * K * (L.I / 16));
+      const uint32_t hfb = (uint32_t)(4ull * T * KP * L.I), hxb = (uint32_t)(4ull * T * KP * (L.I / 16));
       mbar_expect_tx(&go[GO_E], hfb + hxb);
       bulk_g2s(hf_s, p.hf, hfb, &go[GO_E]);
       bulk_g2s(hx_s, p.hx, hxb, &go[GO_E]);
@@ -953,7 +975,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   block_rows(H, c, G, r0, r1);
   const int nrows = r1 - r0;
   const int nslots = p.nslots;
-  const DecodeSmem sp = decode_smem_plan(T, K, L.E, H, I, decode_rows_max(H, G), nslots, p.slot_bytes, L.prenorm);
+  const DecodeSmem sp = decode_smem_plan(T, L.KP, L.E, H, I, decode_rows_max(H, G), nslots, p.slot_bytes, smem_opts(L));
   uint8_t* ring = smem + sp.ring;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + sp.bars);
   uint64_t* empty = full + nslots;
@@ -982,6 +1004,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   uint16_t* gam_s = reinterpret_cast<uint16_t*>(smem + sp.gam);
   uint16_t* gpre_s = reinterpret_cast<uint16_t*>(smem + sp.gpre);
   float* wss = reinterpret_cast<float*>(smem + sp.gpre + 2ull * H);
+  uint16_t* sgv_s = reinterpret_cast<uint16_t*>(smem + sp.sgv);
+  float* sgp = reinterpret_cast<float*>(smem + sp.sgv + 2ull * H);  // [14][T] partial dots, then [T] gates
+  float* sgt = sgp + kConsumerWarps * T;
   float* ypart = reinterpret_cast<float*>(smem + sp.ypart);
   float* ys = reinterpret_cast<float*>(smem + sp.ys);
   float* hacc = reinterpret_cast<float*>(smem + sp.hacc);
@@ -1043,7 +1068,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       pr.d = descs;
       pr.fill = 0;
       pr.policy = l2_policy_evict_first();
-      run_producer<TRACE>(p, pr, xs, res_s, gam_s, xbar, topkbar, flags, eptr, tkbuf, gpre_s);
+      run_producer<TRACE>(p, pr, xs, res_s, gam_s, xbar, topkbar, flags, eptr, tkbuf, gpre_s, sgv_s);
     }
     __syncwarp();
   } else if (warp == kSyncWarp) {
@@ -1136,6 +1161,39 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         if (q < np && (q & 7) == 0) xsum[q >> 3] = sm;
       }
       consumer_sync();
+      if (L.sgate) {
+        // the shared output gate of each token: sigmoid(x . g), the dot in
+        // fp32 in a fixed order (per thread over its pieces, per warp, then
+        // over the warps in order)
+        float part[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) part[t] = 0.f;
+#pragma unroll 1
+        for (int q = tid; q < np; q += kConsumers) {
+          float xv[8], gv[8];
+          const int t = (8 * q) / H, col = 8 * q - t * H;
+          unpack_bf16x8(reinterpret_cast<const uint4*>(xs)[q], xv);
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(sgv_s + col), gv);
+          float d = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) d = fmaf(xv[i], gv[i], d);
+#pragma unroll
+          for (int tt = 0; tt < 8; ++tt)
+            if (tt == t) part[tt] += d;
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const float v = warp_sum(part[t]);
+          if (lane == 0 && t < T) sgp[warp * T + t] = v;
+        }
+        consumer_sync();
+        if (tid < T) {
+          float z = 0.f;
+          for (int w = 0; w < kConsumerWarps; ++w) z += sgp[w * T + tid];
+          sgt[tid] = 1.f / (1.f + expf(-z));
+        }
+        // read after the later consumer barriers (the combine)
+      }
       if (tid == 0) trace_mark<TRACE>(p, 64);
     }
     int item = 0;  // running count of work items over the compute tiles
@@ -1190,8 +1248,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
               float r[2][2];
               const uint64_t tu0 = TRACE ? globaltimer_ns() : 0;
               if (gu)
-                routed_unit<FMT, true>(smem_u32(sl), sg, u, gh, smem_u32(xf + (size_t)(sg.pair / K) * gh.G * 8),
-                                       smem_u32(xsum + (size_t)(sg.pair / K) * gh.G), r);
+                routed_unit<FMT, true>(smem_u32(sl), sg, u, gh, smem_u32(xf + (size_t)(sg.pair / L.KP) * gh.G * 8),
+                                       smem_u32(xsum + (size_t)(sg.pair / L.KP) * gh.G), r);
               else
                 routed_unit<FMT, false>(smem_u32(sl), sg, u, gi, smem_u32(hf_s + (size_t)sg.pair * gi.G * 256),
                                         smem_u32(hx_s + (size_t)sg.pair * (I / kRowBlock)), r);
@@ -1218,6 +1276,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
               const int cols = down ? I : H;
               if (split) {
                 // part q of row rl: columns [q*chunk, min(cols, (q+1)*chunk))
+                const bool probe = TRACE && warp == 0 && type == TILE_SHARED_GU && !(probed & 4);
+                if (probe && lane == 0) p.trace[(size_t)c * kTraceEntries + 75] = globaltimer_ns();
                 const int rl = j / nparts, q = j - rl * nparts;
                 const int chunk = ((cols + nparts - 1) / nparts + 7) & ~7;
                 const int c0 = min(cols, q * chunk), nc = min(cols, c0 + chunk) - c0;
@@ -1238,6 +1298,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
                   v0 = o[0];
                 }
                 v0 = warp_sum(v0) + rbias;
+                if (probe && lane == 0) p.trace[(size_t)c * kTraceEntries + 76] = globaltimer_after(v0 + v1);
                 float* rp = rpart + ((size_t)slot * kSplitRows + rl) * kMaxParts * 2;
                 int last = 0;
                 if (lane == 0) {
@@ -1254,11 +1315,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
                       a1 += vp[2 * k + 1];
                     }
                     rcnt[slot * kSplitRows + rl] = 0;
-                    if (type == TILE_ROUTER)
+                    if (type == TILE_ROUTER) {
                       st_relaxed_gpu_b64(p.logits + row, epoch_word(epoch, a0));
-                    else
+                      if (TRACE)
+                        atomicMax(reinterpret_cast<unsigned long long*>(p.trace + (size_t)c * kTraceEntries + 72),
+                                  (unsigned long long)globaltimer_ns());
+                    } else {
                       p.hs[row] = silu_mul(a0, a1);
+                    }
                   }
+                }
+                if (probe) {
+                  if (lane == 0) p.trace[(size_t)c * kTraceEntries + 77] = globaltimer_ns();
+                  probed |= 4;
                 }
                 continue;
               }
@@ -1283,10 +1352,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
                   }
                   v0 = warp_sum(v0);
                   if (lane == 0) {
-                    if (type == TILE_ROUTER)
+                    if (type == TILE_ROUTER) {
                       st_relaxed_gpu_b64(p.logits + row, epoch_word(epoch, v0 + rbias));
-                    else
+                      if (TRACE)
+                        atomicMax(reinterpret_cast<unsigned long long*>(p.trace + (size_t)c * kTraceEntries + 72),
+                                  (unsigned long long)globaltimer_ns());
+                    } else {
                       p.hs[row] = silu_mul(v0, v1);
+                    }
                   }
                   continue;
                 }
@@ -1376,7 +1449,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
             trace_mark<TRACE>(p, 68);
           }
           __syncwarp();
-          const bool need = L.has_shared != 0;
+          const bool need = L.has_shared && !L.spacked;  // the bf16 shared expert's intermediate
           const bool gw = ok && (!need || grid_wait_thread(&ctr[1], G, &ctr[5], p.err, p.timeout_ns));
           const bool gs = __all_sync(0xffffffffu, gw);
           if (lane == 0) {
@@ -1409,15 +1482,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         const int t = q / nrows, j = q - t * nrows;
         float acc = 0.f;
 #pragma unroll 1
-        for (int k = 0; k < K; ++k) {
-          const int pair = t * K + k;
+        for (int k = 0; k < L.KP; ++k) {
+          const int pair = t * L.KP + k;
           float yk = 0.f;
 #pragma unroll 1
           for (int u = 0; u < gi.U; ++u) yk += ypart[(size_t)(pair * gi.U + u) * nrows + j];
-          acc = fmaf(tk_w[pair], yk, acc);
+          // pair K: the packed shared expert, scaled by its gate if any
+          const float wk = k < K ? tk_w[pair] : (L.sgate ? sgt[t] : 1.f);
+          acc = fmaf(wk, yk, acc);
         }
         float h = __bfloat162float(__ushort_as_bfloat16(res_s[q])) + acc;
-        if (L.has_shared) h += ys[q];
+        if (L.has_shared && !L.spacked) h += L.sgate ? sgt[t] * ys[q] : ys[q];
         hacc[q] = h;
         p.h_out[(size_t)t * H + r0 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
       }
@@ -1429,49 +1504,67 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         for (int j = lane; j < nrows; j += 32) s = fmaf(hacc[warp * nrows + j], hacc[warp * nrows + j], s);
         s = warp_sum(s);
         if (lane == 0) st_relaxed_gpu_b64(p.ss + (size_t)c * T + warp, epoch_word(epoch, s));
+        if (TRACE && lane == 0 && warp == 0) p.trace[(size_t)c * kTraceEntries + 99] = globaltimer_ns();
       }
       // RMSNorm: every block polls all blocks' sums of squares (the words are
       // complete once they carry this launch's epoch), sums them in block
       // order and normalises its own rows of h
       bool got = true;
       if (warp < T) {
-        float s = 0.f;
+        // lane l holds blocks l, l + 32, ...: every pass loads all the words
+        // still missing at once, so a pass costs one round trip
+        constexpr int kMaxPer = (kMaxGrid + 31) / 32;
+        float v[kMaxPer];
+        uint32_t need = 0;
+#pragma unroll
+        for (int i = 0; i < kMaxPer; ++i) {
+          v[i] = 0.f;
+          if (lane + 32 * i < G) need |= 1u << i;
+        }
         uint64_t t0 = 0;
-        uint32_t it = 0;
 #pragma unroll 1
-        for (int b0 = 0; b0 < G && got; b0 += 32) {
-          const int bk = b0 + lane;
-          float v = 0.f;
-          bool have = bk >= G;
-          for (;; ++it) {
-            if (!have) {
-              const uint64_t wd = ld_relaxed_gpu_b64(p.ss + (size_t)bk * T + warp);
-              if ((uint32_t)(wd >> 32) == epoch) {
-                have = true;
-                v = __uint_as_float((uint32_t)wd);
+        for (uint32_t it = 0;; ++it) {
+          if (TRACE && lane == 0 && warp == 0) {
+            const uint64_t now = globaltimer_ns();
+            if (it < 8) p.trace[(size_t)c * kTraceEntries + 120 + it] = now;
+            p.trace[(size_t)c * kTraceEntries + 97] = it + 1;
+          }
+          uint64_t wd[kMaxPer];
+#pragma unroll
+          for (int i = 0; i < kMaxPer; ++i)
+            wd[i] = (need >> i & 1u) ? ld_relaxed_gpu_b64(p.ss + (size_t)(lane + 32 * i) * T + warp) : 0ull;
+          if (TRACE && lane == 0 && warp == 0)
+            p.trace[(size_t)c * kTraceEntries + 98] = globaltimer_after((float)(wd[0] + wd[kMaxPer - 1]));
+#pragma unroll
+          for (int i = 0; i < kMaxPer; ++i)
+            if ((need >> i & 1u) && (uint32_t)(wd[i] >> 32) == epoch) {
+              need &= ~(1u << i);
+              v[i] = __uint_as_float((uint32_t)wd[i]);
+            }
+          if (__all_sync(0xffffffffu, need == 0u)) break;
+          if ((it & 15u) == 15u) {
+            int stop = 0;
+            if (lane == 0) {
+              if (t0 == 0) t0 = globaltimer_ns();
+              if (ld_relaxed_gpu(&ctr[5]) != 0u) {
+                stop = 1;
+              } else if (globaltimer_ns() - t0 > p.timeout_ns) {
+                atomicCAS(p.err, 0u, 1u);
+                atomicExch(&ctr[5], 1u);
+                stop = 1;
               }
             }
-            if (__all_sync(0xffffffffu, have)) break;
-            if ((it & 63u) == 63u) {
-              int stop = 0;
-              if (lane == 0) {
-                if (t0 == 0) t0 = globaltimer_ns();
-                if (ld_relaxed_gpu(&ctr[5]) != 0u) {
-                  stop = 1;
-                } else if (globaltimer_ns() - t0 > p.timeout_ns) {
-                  atomicCAS(p.err, 0u, 1u);
-                  atomicExch(&ctr[5], 1u);
-                  stop = 1;
-                }
-              }
-              if (__shfl_sync(0xffffffffu, stop, 0)) {
-                got = false;
-                break;
-              }
+            if (__shfl_sync(0xffffffffu, stop, 0)) {
+              got = false;
+              break;
             }
           }
-          s += v;
         }
+        // the sum in block order: lane partials over i, then across lanes
+        // (a fixed order whatever the arrival order)
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMaxPer; ++i) s += v[i];
         s = warp_sum(s);
         if (lane == 0) {
           inv[warp] = rsqrtf(__fdividef(s, (float)H) + L.eps);
@@ -1508,16 +1601,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   if (tid == 0) trace_mark<TRACE>(p, 8);
 }
 
+// The kernel's dynamic shared-memory limit is raised per device to the
+// largest size any launch asked for; the check and the set happen under one
+// lock, so host threads launching different sizes cannot leave the cached
+// value above the attribute.
 template <int FMT, bool TRACE>
 static cudaError_t launch_one(const DecodeParams& p, int grid, size_t smem, cudaStream_t st) {
   static size_t attr_set[64] = {};
+  static std::mutex mu;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && attr_set[dev] < smem) {
-    cudaError_t e =
-        cudaFuncSetAttribute(moe_decode_kernel<FMT, TRACE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = smem;
+  if (dev >= 0 && dev < 64) {
+    std::lock_guard<std::mutex> lk(mu);
+    if (attr_set[dev] < smem) {
+      const cudaError_t e = cudaFuncSetAttribute(moe_decode_kernel<FMT, TRACE>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = smem;
+    }
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -1549,7 +1650,7 @@ uint32_t decode_slot_bytes(const Layout& L, int T, int nrows_max, int* nslots) {
   const size_t need[5] = {2ull * L.H + 16, 4ull * L.H + 32, 2ull * L.I + 16,
                           2ull * 2 * 8 * gh.W * per_group + 64, 2ull * 4 * gi.W * per_group + 64};
   for (int ns = kSlots; ns >= 2; --ns) {
-    const size_t other = decode_smem_plan(T, L.K, L.E, L.H, L.I, nrows_max, ns, 0, L.prenorm).total + 1024;
+    const size_t other = decode_smem_plan(T, L.KP, L.E, L.H, L.I, nrows_max, ns, 0, smem_opts(L)).total + 1024;
     if (other >= limit) return 0;
     size_t slot = (limit - other) / ns;
     slot = slot / 1024 * 1024;

@@ -295,18 +295,26 @@ static __device__ __noinline__ void warp_topk_keys(const float* logits, int E, i
 // keys in registers; larger E: staged in `keys` (E entries of shared memory).
 static __device__ __noinline__ bool warp_topk_poll(const uint64_t* words, uint32_t epoch, int E, int K,
                                                    uint64_t* keys, int32_t* idx, float* w, uint32_t* abort_flag,
-                                                   uint32_t* err, uint64_t timeout_ns, uint32_t* polls) {
+                                                   uint32_t* err, uint64_t timeout_ns, uint32_t* polls,
+                                                   uint64_t* tr = nullptr) {
   const int lane = threadIdx.x & 31;
   uint64_t t0 = 0;
   uint32_t nit = 0;
   bool ok = true;
   // poll words [e0, e0 + 512) into v[]: lane's i-th word is e0 + lane + 32 i
+  // (tr, traced launches: start time of the last pass and the number of passes)
   auto poll = [&](int e0, float (&v)[16]) -> bool {
     uint32_t need = 0, have = 0;
 #pragma unroll
     for (int i = 0; i < 16; ++i)
       if (e0 + lane + 32 * i < E) need |= 1u << i;
     for (uint32_t it = 0;; ++it) {
+      if (tr && lane == 0) {
+        const uint64_t now = globaltimer_ns();
+        tr[0] = now;
+        tr[1] = it + 1;
+        if (it < 8) tr[15 + it] = now;  // start of each of the first 8 passes
+      }
       uint64_t wv[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i)
@@ -318,6 +326,7 @@ static __device__ __noinline__ bool warp_topk_poll(const uint64_t* words, uint32
           v[i] = __uint_as_float((uint32_t)wv[i]);
         }
       ++nit;
+      if (tr && lane == 0) tr[23] = globaltimer_after(wv[0] + wv[15]);  // this pass's loads returned
       if (__all_sync(0xffffffffu, have == need)) return true;
       if ((it & 31u) == 31u) {
         int stop = 0;

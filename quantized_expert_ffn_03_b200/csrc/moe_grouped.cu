@@ -554,12 +554,13 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__
 // The second pass recomputes h in the same order (its inputs are in L2).
 __device__ __forceinline__ float combine_h(const float* __restrict__ Y, const float* __restrict__ Ys,
                                            const int* __restrict__ pair_slot, const float* __restrict__ w,
-                                           const uint16_t* __restrict__ res, int t, int c, int H, int K) {
+                                           const uint16_t* __restrict__ res, int t, int c, int H, int K,
+                                           float sg) {
   float h = __uint_as_float((uint32_t)res[(size_t)t * H + c] << 16);
   float acc = 0.f;
   for (int k = 0; k < K; ++k) acc = fmaf(w[t * K + k], Y[(size_t)pair_slot[t * K + k] * H + c], acc);
   h += acc;
-  if (Ys) h += Ys[(size_t)t * H + c];
+  if (Ys) h += sg * Ys[(size_t)t * H + c];
   return h;
 }
 
@@ -567,13 +568,32 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
                                                       const int* __restrict__ pair_slot, const float* __restrict__ w,
                                                       const uint16_t* __restrict__ res,
                                                       const uint16_t* __restrict__ gamma, int H, int K, float eps,
+                                                      const uint16_t* __restrict__ x,
+                                                      const uint16_t* __restrict__ sgate,
                                                       uint16_t* __restrict__ h_out, uint16_t* __restrict__ y_norm) {
   const int t = blockIdx.x;
   __shared__ float red[8];
-  __shared__ float inv_s;
+  __shared__ float inv_s, sg_s;
+  // the shared output gate sigmoid(x . g) of this token, when given
+  float sg = 1.f;
+  if (sgate) {
+    float d = 0.f;
+    for (int c = threadIdx.x; c < H; c += blockDim.x)
+      d = fmaf(__uint_as_float((uint32_t)x[(size_t)t * H + c] << 16), __uint_as_float((uint32_t)sgate[c] << 16), d);
+    d = warp_sum(d);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = d;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float z = 0.f;
+      for (int i = 0; i < (int)(blockDim.x >> 5); ++i) z += red[i];
+      sg_s = 1.f / (1.f + expf(-z));
+    }
+    __syncthreads();
+    sg = sg_s;
+  }
   float ss = 0.f;
   for (int c = threadIdx.x; c < H; c += blockDim.x) {
-    const float h = combine_h(Y, Ys, pair_slot, w, res, t, c, H, K);
+    const float h = combine_h(Y, Ys, pair_slot, w, res, t, c, H, K, sg);
     ss = fmaf(h, h, ss);
     h_out[(size_t)t * H + c] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
   }
@@ -588,7 +608,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   __syncthreads();
   const float inv = inv_s;
   for (int c = threadIdx.x; c < H; c += blockDim.x) {
-    const float h = combine_h(Y, Ys, pair_slot, w, res, t, c, H, K);
+    const float h = combine_h(Y, Ys, pair_slot, w, res, t, c, H, K, sg);
     const float g = __uint_as_float((uint32_t)gamma[c] << 16);
     y_norm[(size_t)t * H + c] = __bfloat16_as_ushort(__float2bfloat16_rn(h * inv * g));
   }
@@ -645,6 +665,15 @@ cudaError_t launch_prenorm(const uint16_t* h, const uint16_t* gamma, int T, int 
   return cudaGetLastError();
 }
 
+__global__ void set_ptr_kernel(const void** dst, const void* v) { *dst = v; }
+
+// Writes one pointer value into device memory (stream-ordered, and usable
+// under stream capture, unlike a copy from a host variable).
+cudaError_t launch_set_ptr(const void** dst, const void* v, cudaStream_t st) {
+  set_ptr_kernel<<<1, 1, 0, st>>>(dst, v);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_to_half(const uint16_t* x, void* xh, size_t n, uint32_t* abort_flag, cudaStream_t st) {
   const size_t n8 = n / 8;
   const int grid = (int)((n8 + 255) / 256 < 1184 ? (n8 + 255) / 256 : 1184);
@@ -661,9 +690,9 @@ cudaError_t launch_group(const int32_t* idx, int TK, int E, int K, int* slot_tok
 }
 
 cudaError_t launch_combine(const float* Y, const float* Ys, const int* pair_slot, const float* w, const uint16_t* res,
-                           const uint16_t* gamma, int T, int H, int K, float eps, uint16_t* h_out, uint16_t* y_norm,
-                           cudaStream_t st) {
-  combine_kernel<<<T, 256, 0, st>>>(Y, Ys, pair_slot, w, res, gamma, H, K, eps, h_out, y_norm);
+                           const uint16_t* gamma, int T, int H, int K, float eps, const uint16_t* x,
+                           const uint16_t* sgate, uint16_t* h_out, uint16_t* y_norm, cudaStream_t st) {
+  combine_kernel<<<T, 256, 0, st>>>(Y, Ys, pair_slot, w, res, gamma, H, K, eps, x, sgate, h_out, y_norm);
   return cudaGetLastError();
 }
 

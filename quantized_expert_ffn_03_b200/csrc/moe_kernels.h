@@ -18,6 +18,7 @@ namespace moe {
 // U units per 16-row block (U <= kMaxUnits).
 constexpr int kMaxUnits = 8;
 constexpr int kRowBlock = 16;  // rows of one routed work unit (the mma's M)
+constexpr int kMaxGrid = 256;  // most blocks of a fused-kernel launch (one per SM)
 struct RoutedGeo {
   int G, gpw, nwin, W, U;
 };
@@ -56,6 +57,8 @@ struct DecodeParams {
   const uint16_t* gamma;
   const uint16_t* gamma_pre;  // L.prenorm: bf16 [H] weight of the RMSNorm applied to x first
   uint16_t* x_out;            // L.prenorm: the normalised x, bf16 [T][H] (block 0 writes it), or null
+  const uint16_t* sgate;      // L.sgate: bf16 [H], the shared expert's output gate
+  const uint8_t* spacked;     // L.spacked: the shared expert's packed blob (pair K of each token)
   const uint16_t* x;
   const uint16_t* res;
   uint16_t* h_out;
@@ -101,6 +104,7 @@ size_t grouped_gemm_smem_bytes(int na, bool packed);
 // ak: 0 dense bf16 A, 4 / 2 packed A; na: A matrices (2 = gate and up);
 // epi: 0 fp32 (+ bias), 1 SwiGLU -> fp16, 2 SwiGLU -> bf16 hi and lo.
 cudaError_t launch_grouped_gemm(int ak, int na, int epi, const GemmParams& p, int grid, cudaStream_t st);
+cudaError_t launch_set_ptr(const void** dst, const void* v, cudaStream_t st);
 cudaError_t launch_prenorm(const uint16_t* h, const uint16_t* gamma, int T, int H, float eps, uint16_t* x,
                            cudaStream_t st);
 cudaError_t launch_to_half(const uint16_t* x, void* xh, size_t n, uint32_t* abort_flag, cudaStream_t st);
@@ -108,7 +112,7 @@ cudaError_t launch_group(const int32_t* idx, int TK, int E, int K, int* slot_tok
                          int* ch_c0, int* ch_n, int* n_chunks, const void* const* expert_ptr, uint32_t* err,
                          cudaStream_t st);
 cudaError_t launch_combine(const float* Y, const float* Ys, const int* pair_slot, const float* w, const uint16_t* res,
-                           const uint16_t* gamma, int T, int H, int K, float eps, uint16_t* h_out, uint16_t* y_norm,
-                           cudaStream_t st);
+                           const uint16_t* gamma, int T, int H, int K, float eps, const uint16_t* x,
+                           const uint16_t* sgate, uint16_t* h_out, uint16_t* y_norm, cudaStream_t st);
 
 }  // namespace moe

@@ -29,6 +29,9 @@ struct Layout {
   int has_shared;
   float eps;
   int prenorm;  // 1: the layer's x is its residual stream, RMS-normalised with a second gamma first
+  int sgate;    // 1: the shared expert's output is scaled by sigmoid(x . g), g bf16 [H]
+  int spacked;  // 1: the shared expert is a packed blob, run as pair K of every token
+  int KP;       // (token, expert) pairs per token: K, or K + 1 with a packed shared expert
   uint32_t off_codes[3];
   uint32_t off_scales[3];
   uint32_t code_row_bytes[3];
@@ -52,6 +55,9 @@ inline bool make_layout(int H, int I, int E, int K, int bits, int group, int has
   L->has_shared = has_shared;
   L->eps = eps;
   L->prenorm = 0;
+  L->sgate = 0;
+  L->spacked = 0;
+  L->KP = K;
   const uint64_t rows[3] = {(uint64_t)I, (uint64_t)I, (uint64_t)H};
   const uint64_t cols[3] = {(uint64_t)H, (uint64_t)H, (uint64_t)I};
   uint64_t pos = 0;

@@ -89,8 +89,11 @@ def check_prenorm_layer(M, dl, h_bits, gp_bits, blobs=None):
         np.testing.assert_allclose(w[t], wk, rtol=8 * bound[t].max() + 2e-6, atol=1e-7)
     blobs = dl.oracle_blobs() if blobs is None else blobs
     _, _, h_ref, y_ref = oracle_forward(s, blobs, dl.dense, x_o, h_bits, idx_in=idx, w_in=w.astype(np.float64))
-    assert_outputs_close(h_dev, h_ref, "h_out")
-    assert_outputs_close(y_dev, y_ref, "y_norm")
+    # h_out carries the residual stream (magnitudes up to ~100 here) and
+    # y_norm its normalised form (up to ~30 on the 8x channels): their bf16
+    # rounding is part of the bound
+    assert_outputs_close(h_dev, h_ref, "h_out", round_rel=2.0 ** -8)
+    assert_outputs_close(y_dev, y_ref, "y_norm", round_rel=2.0 ** -8)
     return x_dev
 
 
