@@ -62,6 +62,8 @@ def parse_args(argv=None):
                    help="streaming store: pinned host memory, or a file read with parallel pread")
     p.add_argument("--direct-io", action="store_true", help="file store: O_DIRECT reads (bypass the page cache)")
     p.add_argument("--store-path", default="/tmp/moe_expert_store.bin")
+    p.add_argument("--stream-resolve", default="device", choices=("device", "host"),
+                   help="streaming: resolve the routing on the GPU (no host round trip) or on the host")
     p.add_argument("--predictor", default="next_router", choices=("next_router", "temporal", "none"),
                    help="streaming prefetch: the next layer's router on this layer's input, the experts the "
                         "next layer chose for the previous token, or no prefetch")
@@ -656,7 +658,11 @@ def run_streaming(args):
     h = torch.empty((1, s.hidden), dtype=torch.int16, device="cuda")
     y = torch.empty_like(h)
 
-    pred = args.predictor
+    on_device = args.stream_resolve == "device"
+    if on_device and args.store == "file":
+        raise SystemExit("--stream-resolve device needs the pinned store")
+    # device-resolved: no prediction (the routing never reaches the host)
+    pred = "none" if on_device else args.predictor
     last_idx = [None] * L  # experts each layer chose for the previous token (temporal predictor)
 
     def token(record=None):
@@ -664,6 +670,16 @@ def run_streaming(args):
         res = torch.randn((1, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
         for l in range(L):
             d = dense[l]
+            if on_device:
+                # router, device resolve (+ fill of the misses), routed layer: back to back
+                M.moe_router_topk(cfg, x, d["wr"], d["bias"], idx_d[0], w_d[0], logits_out=lg[0])
+                M.moe_stream_resolve_device(cache, l, idx_d[0], table)
+                M.moe_layer_forward_routed(cfg, wts[l], x, res, idx_d[0], w_d[0], h, y, ws)
+                if record is not None:
+                    record.append((l, x.clone(), res.clone(), idx_d[0].clone(), w_d[0].clone(), h.clone(),
+                                   y.clone()))
+                x, res = y.clone(), h.clone()
+                continue
             M.moe_router_topk(cfg, x, d["wr"], d["bias"], idx_d[0], w_d[0], logits_out=lg[0])
             if pred == "next_router" and l + 1 < L:
                 dn = dense[l + 1]
@@ -682,11 +698,41 @@ def run_streaming(args):
             last_idx[l] = idx_h[0].numpy().copy()
             x, res = y.clone(), h.clone()
 
+    # device-resolved: one token through the L layers captured as a CUDA
+    # graph (router, resolve, fill, routed layer per layer; layer outputs in
+    # ping-pong buffers), replayed per token after copying the token's
+    # inputs into its input buffers
+    graph = None
+    use_graph = on_device and not args.no_graph
+    if use_graph:
+        npool = args.stream_steps + 4
+        pool_x = torch.randn((npool, 1, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
+        pool_r = torch.randn((npool, 1, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
+        xin, rin = torch.empty_like(h), torch.empty_like(h)
+        hb = [torch.empty_like(h) for _ in range(2)]
+        yb = [torch.empty_like(h) for _ in range(2)]
+
+        def token_body():
+            xx, rr = xin, rin
+            for l in range(L):
+                d = dense[l]
+                M.moe_router_topk(cfg, xx, d["wr"], d["bias"], idx_d[0], w_d[0], logits_out=lg[0])
+                M.moe_stream_resolve_device(cache, l, idx_d[0], table)
+                M.moe_layer_forward_routed(cfg, wts[l], xx, rr, idx_d[0], w_d[0], hb[l % 2], yb[l % 2], ws)
+                xx, rr = yb[l % 2], hb[l % 2]
+
     checked, mismatches = 0, 0
     try:
         for i in range(args.stream_warmup):
             token()
         torch.cuda.synchronize()
+        if use_graph:
+            cap = torch.cuda.Stream()
+            with torch.cuda.stream(cap):
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=cap):
+                    token_body()
+            torch.cuda.synchronize()
         st0 = M.moe_stream_stats(cache)
         fs0 = M.moe_stream_file_stats(cache) if args.store == "file" else None
         M.moe_stream_copy_timing(cache)  # (enables nothing yet: clears)
@@ -696,7 +742,12 @@ def run_streaming(args):
         wall0 = time.perf_counter()
         t0.record()
         for i in range(args.stream_steps):
-            token()
+            if graph is not None:
+                xin.copy_(pool_x[i], non_blocking=True)
+                rin.copy_(pool_r[i], non_blocking=True)
+                graph.replay()
+            else:
+                token()
         t1.record()
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
@@ -745,7 +796,8 @@ def run_streaming(args):
         "n_gpus": 1, "steps": args.stream_steps, "warmup": args.stream_warmup,
         "ms_per_step": ms / args.stream_steps, "higher_is_better": True, "dtype": "f32", "data": "synthetic",
         "config": {"workload": "%s_x%d_layers" % (s.name, L), "layers": L, "layers_requested": L_req,
-                   "predictor": pred,
+                   "predictor": pred, "resolve": args.stream_resolve,
+                   "copier": "fill kernel over mapped host memory" if on_device else "cudaMemcpyAsync",
                    "host_available_gb": (avail / 1e9) if avail else None, "slots": NS,
                    "slot_bytes": nb, "host_store_gb": L * E * nb / 1e9, "device_cache_gb": NS * nb / 1e9,
                    "tokens_per_step": 1, "router_bias": "zipf1.1, a different permutation per layer"},
@@ -763,9 +815,10 @@ def run_streaming(args):
                  "copy_ms_sum": ct["copy_ms"], "copies": ct["copies"], "bytes": ct["bytes"],
                  "busy_share_of_step": ct["busy_ms"] / ms if ms > 0 else None},
         "ms_per_layer": ms / args.stream_steps / L,
+        "cuda_graph": graph is not None,
         "wall_ms_per_step": wall * 1e3 / args.stream_steps,
         "checked_layers": checked, "mismatched_layers": mismatches,
-        "device_error": err,
+        "device_error": err, "cache_device_error": st1.get("device_error", 0),
     }
     if args.store == "file":
         reads = fs1["reads"] - fs0["reads"]
@@ -781,7 +834,7 @@ def run_streaming(args):
         except OSError:
             pass
     print(json.dumps(line), flush=True)
-    return 0 if (err == 0 and mismatches == 0) else 1
+    return 0 if (err == 0 and mismatches == 0 and st1.get("device_error", 0) == 0) else 1
 
 
 def run_batched(args):

@@ -441,12 +441,38 @@ moe_status moe_stream_prefetch(moe_stream_cache* cache, int layer, const int32_t
 moe_status moe_stream_resolve(moe_stream_cache* cache, int layer, const int32_t* idx_host, int n,
                               const void** expert_ptr_dev, cudaStream_t compute_stream);
 
+/* The same resolve decided on the GPU, for routing that stays on the device:
+ * idx_dev (device int32 [n], n <= 64, typically moe_router_topk's output)
+ * names experts of `layer`.  One kernel looks each distinct id up in a
+ * device-resident slot table (hits touch nothing else), picks for every
+ * miss the slot the host policy would pick (an empty slot, lowest index
+ * first, else the least recently used one not taken by this call), updates
+ * the table, and writes expert_ptr_dev[e] for every id; a second kernel
+ * copies the missed experts from the pinned host store into their slots
+ * with 16-byte loads of mapped host memory (it returns at once when nothing
+ * missed).  Nothing waits on the host and nothing is read back, so a layer's
+ * router, this call and moe_layer_forward_routed can run back to back or be
+ * captured into a CUDA graph; the pages' CPU reads the router output before
+ * its reads (hakusoku "パイプライン概要"), which this call keeps on the GPU.
+ * A cache serves either this call or moe_stream_resolve/moe_stream_prefetch,
+ * whichever is called first (the other then returns MOE_ERR_INVALID_ARG);
+ * MOE_ERR_UNSUPPORTED for a file store or a host store the device cannot map.
+ * Ids outside [0, E) get no table entry (the layer then reports a bad
+ * pointer); more distinct ids than slots leave MOE_ERR_OOM in the cache's
+ * device error word (moe_stream_stats' device_error) and the table
+ * unwritten.  moe_stream_stats and moe_stream_copy_timing read the device
+ * counters back (synchronising); bytes_h2d counts the bytes the fill kernel
+ * copied and the copy timing reports its busy time from device timestamps. */
+moe_status moe_stream_resolve_device(moe_stream_cache* cache, int layer, const int32_t* idx_dev, int n,
+                                     const void** expert_ptr_dev, cudaStream_t stream);
+
 /* Counters since create: resolved experts found resident (hits) or copied
  * on demand (misses), prefetch copies issued, resolved experts that a
  * prefetch had brought in and no resolve had used yet (prefetch_hits),
  * prefetch ids skipped for want of a free slot, and bytes copied. */
 typedef struct {
   uint64_t hits, misses, prefetches, prefetch_hits, prefetch_dropped, bytes_h2d;
+  uint64_t device_error;  /* device-resolved caches: 0, or the first error a resolve kernel met */
 } moe_stream_counters;
 moe_status moe_stream_stats(const moe_stream_cache* cache, moe_stream_counters* out);
 

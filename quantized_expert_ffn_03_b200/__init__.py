@@ -104,6 +104,7 @@ EXPORTS = {
     "moe_stream_prefetch": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p]),
     "moe_stream_resolve": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
     "moe_stream_stats": (C.c_int, [C.c_void_p, C.c_void_p]),
+    "moe_stream_resolve_device": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
     "moe_stream_destroy": (None, [C.c_void_p]),
     "moe_device_error": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
     "moe_noalloc_device_error": (C.c_int, [C.c_void_p, C.c_void_p]),
@@ -344,7 +345,8 @@ def moe_layer_forward_host_packed(cfg, wts, xr, hy, workspace, stream=None):
 
 class MoeStreamCounters(C.Structure):
     _fields_ = [("hits", C.c_uint64), ("misses", C.c_uint64), ("prefetches", C.c_uint64),
-                ("prefetch_hits", C.c_uint64), ("prefetch_dropped", C.c_uint64), ("bytes_h2d", C.c_uint64)]
+                ("prefetch_hits", C.c_uint64), ("prefetch_dropped", C.c_uint64), ("bytes_h2d", C.c_uint64),
+                ("device_error", C.c_uint64)]
 
 
 def moe_stream_create(cfg, n_layers, host_store, n_slots, store_bytes=None):
@@ -395,6 +397,13 @@ def moe_stream_resolve(cache, layer, idx, expert_ptr, stream=None):
     """idx: host ids (numpy / list); expert_ptr: int64 CUDA tensor [E] (written)."""
     a, n = _ids(idx)
     _check(_lib.moe_stream_resolve(cache, int(layer), a.ctypes.data, n, _ptr(expert_ptr), _stream(stream)))
+
+
+def moe_stream_resolve_device(cache, layer, idx, expert_ptr, stream=None):
+    """idx: int32 CUDA tensor of expert ids (any shape, at most 64); expert_ptr:
+    int64 CUDA tensor [E] (written on the device).  Nothing is read back."""
+    _check(_lib.moe_stream_resolve_device(cache, int(layer), _ptr(idx), int(idx.numel()), _ptr(expert_ptr),
+                                          _stream(stream)))
 
 
 def moe_stream_stats(cache):

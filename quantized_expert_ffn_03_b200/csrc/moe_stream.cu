@@ -25,6 +25,13 @@
 //     and must not be called while its stream is being captured into a
 //     CUDA graph.
 //
+// Device-resolved caches (moe_stream_resolve_device) keep the same policy on
+// the GPU instead: a slot table [layer][expert] -> slot, the key and the last
+// use of every slot, and counters, all in device memory, updated by one
+// single-block kernel per call; the misses are then copied by a grid of
+// blocks reading the mapped host store.  The routing never leaves the device
+// and no host thread waits.
+//
 // Failures: a copy that cannot be enqueued (MOE_ERR_IO) leaves its slot
 // empty, and a resolve that fails releases the slots it took, so the next
 // call starts from a consistent cache.  Tests drive these paths with
@@ -143,8 +150,30 @@ constexpr int kFileStage = 16;  // pinned staging buffers of a file-backed store
 
 }  // namespace
 
+namespace moe {
+namespace {
+constexpr int kMaxResolveIds = 64;  // ids of one device-resolved call
+// device counters of a device-resolved cache
+enum { DC_CLOCK = 0, DC_HITS, DC_MISSES, DC_BYTES, DC_FILL_NS, DC_ERROR, DC_FILL_DONE, DC_FILL_T0, DC_FILL_T1,
+       DC_FILLS, DC_N };
+struct DevTables {
+  int32_t* slot_of = nullptr;  // [L * E] -> slot, or -1
+  int32_t* key = nullptr;      // [S] -> layer * E + expert, or -1
+  uint64_t* tick = nullptr;    // [S] last use
+  uint64_t* ctr = nullptr;     // [DC_N]
+  int32_t* jobs = nullptr;     // [2 * kMaxResolveIds]: slot, then key, of each fill
+  int32_t* njobs = nullptr;    // [1]
+};
+}  // namespace
+}  // namespace moe
+
 struct moe_stream_cache {
   int L = 0, E = 0, S = 0;
+  int mode = 0;                        // 0 unused, 1 host-resolved, 2 device-resolved
+  int sms = 0;                         // the device's SM count (fill grid)
+  moe::DevTables dt;                   // device-resolved state (pinned stores only)
+  const uint8_t* host_dev = nullptr;   // the store as the device addresses it
+  uint64_t dev_seen_ns = 0, dev_seen_bytes = 0, dev_seen_fills = 0;  // copy timing already reported
   size_t blob = 0;
   int device = 0;
   const uint8_t* host = nullptr;  // pinned host store, or null for a file store
@@ -219,6 +248,9 @@ void destroy_parts(moe_stream_cache* c) {
     if (c->stage[i]) cudaFreeHost(c->stage[i]);
   }
   if (c->slots) cudaFree(c->slots);
+  void* dts[] = {c->dt.slot_of, c->dt.key, c->dt.tick, c->dt.ctr, c->dt.jobs, c->dt.njobs};
+  for (void* q : dts)
+    if (q) cudaFree(q);
 }
 
 // Enqueue the copy of (layer, e) into slot s on stream st (see the ordering
@@ -371,6 +403,7 @@ moe_status finish_create(moe_stream_cache* c, const moe_config* cfg, int n_layer
   c->blob = blob;
   cudaGetDevice(&c->device);
   c->pol.init(n_layers, cfg->n_experts, n_slots);
+  cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->device);
   bool alloc_fault = false;
   {
     std::lock_guard<std::mutex> lk(g_fault_mu);
@@ -400,8 +433,210 @@ moe_status finish_create(moe_stream_cache* c, const moe_config* cfg, int n_layer
     delete c;
     return failf(MOE_ERR_OOM, "could not create the cache's events or staging buffers");
   }
+  if (c->host) {
+    // the device-resolved state: the tables start empty (all -1), the
+    // counters at zero; and the store's device address, if it is mapped
+    moe::DevTables& t = c->dt;
+    const size_t le = (size_t)n_layers * cfg->n_experts;
+    okk = cudaMalloc(&t.slot_of, 4 * le) == cudaSuccess && cudaMalloc(&t.key, 4ull * n_slots) == cudaSuccess &&
+          cudaMalloc(&t.tick, 8ull * n_slots) == cudaSuccess && cudaMalloc(&t.ctr, 8ull * moe::DC_N) == cudaSuccess &&
+          cudaMalloc(&t.jobs, 8ull * moe::kMaxResolveIds) == cudaSuccess &&
+          cudaMalloc(&t.njobs, 16) == cudaSuccess && cudaMemset(t.slot_of, 0xff, 4 * le) == cudaSuccess &&
+          cudaMemset(t.key, 0xff, 4ull * n_slots) == cudaSuccess &&
+          cudaMemset(t.tick, 0, 8ull * n_slots) == cudaSuccess && cudaMemset(t.njobs, 0, 16) == cudaSuccess;
+    if (okk) {
+      uint64_t c0[moe::DC_N] = {};
+      c0[moe::DC_FILL_T0] = ~0ull;  // a running minimum
+      okk = cudaMemcpy(t.ctr, c0, sizeof(c0), cudaMemcpyHostToDevice) == cudaSuccess &&
+            cudaDeviceSynchronize() == cudaSuccess;
+    }
+    if (!okk) {
+      cudaGetLastError();
+      destroy_parts(c);
+      delete c;
+      return failf(MOE_ERR_OOM, "could not allocate the cache's device tables");
+    }
+    void* hd = nullptr;
+    if (cudaHostGetDevicePointer(&hd, const_cast<uint8_t*>(c->host), 0) == cudaSuccess)
+      c->host_dev = static_cast<const uint8_t*>(hd);
+    else
+      cudaGetLastError();  // not mapped: the device-resolved calls are unavailable
+  }
   *out = c;
   return MOE_OK;
+}
+
+// ---- device-resolved calls -----------------------------------------------------------
+
+// One block: the distinct ids of the call, in order, each looked up in the
+// slot table; a miss takes an empty slot (lowest index) or else the least
+// recently used slot not taken by this call (the same choice as
+// StreamPolicy), found by a block-wide reduction.  Table pointers are
+// written only when every id found a slot.
+__global__ void __launch_bounds__(1024) stream_resolve_kernel(moe::DevTables t, int E, int S, int layer,
+                                                              const int32_t* __restrict__ idx, int n,
+                                                              const void** __restrict__ eptr, uint8_t* slots,
+                                                              size_t blob) {
+  extern __shared__ uint32_t held[];  // [(S + 31) / 32] bits: slots taken by this call
+  __shared__ int s_ids[moe::kMaxResolveIds], s_slot[moe::kMaxResolveIds];
+  __shared__ int s_cur, s_abort, s_nj;
+  __shared__ unsigned long long s_red[32];
+  __shared__ int s_redi[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  const int nwords = (S + 31) / 32;
+  for (int i = tid; i < nwords; i += blockDim.x) held[i] = 0u;
+  if (tid < n) s_ids[tid] = idx[tid];
+  if (tid == 0) {
+    s_abort = 0;
+    s_nj = 0;
+  }
+  __syncthreads();
+  uint64_t* ctr = t.ctr;
+#pragma unroll 1
+  for (int i = 0; i < n; ++i) {
+    if (tid == 0) {
+      const int e = s_ids[i];
+      int sl = -2;  // -2: invalid id
+      if (e >= 0 && e < E) sl = t.slot_of[(size_t)layer * E + e];
+      if (sl >= 0 && !(held[sl >> 5] >> (sl & 31) & 1u)) {
+        held[sl >> 5] |= 1u << (sl & 31);
+        t.tick[sl] = ++ctr[moe::DC_CLOCK];
+        ++ctr[moe::DC_HITS];
+      }
+      s_slot[i] = sl;
+      s_cur = sl;
+    }
+    __syncthreads();
+    if (s_cur != -1) continue;  // a hit, a repeat or an invalid id (uniform)
+    // a miss: the lowest empty slot not taken, else the least recently used
+    int be = 0x7fffffff;
+    unsigned long long bl = ~0ull;
+    for (int j = tid; j < S; j += blockDim.x) {
+      if (held[j >> 5] >> (j & 31) & 1u) continue;
+      if (t.key[j] < 0) {
+        be = min(be, j);
+      } else {
+        const unsigned long long k = ((unsigned long long)t.tick[j] << 24) | (unsigned long long)j;
+        bl = k < bl ? k : bl;
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      be = min(be, __shfl_xor_sync(0xffffffffu, be, o));
+      const unsigned long long ob = __shfl_xor_sync(0xffffffffu, bl, o);
+      bl = ob < bl ? ob : bl;
+    }
+    if (lane == 0) {
+      s_redi[warp] = be;
+      s_red[warp] = bl;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int b = 0x7fffffff;
+      unsigned long long l = ~0ull;
+      for (int w = 0; w < nw; ++w) {
+        b = min(b, s_redi[w]);
+        l = s_red[w] < l ? s_red[w] : l;
+      }
+      const int v = b != 0x7fffffff ? b : (l != ~0ull ? (int)(l & 0xffffffull) : -1);
+      if (v < 0) {
+        s_abort = 1;
+        if (ctr[moe::DC_ERROR] == 0) ctr[moe::DC_ERROR] = MOE_ERR_OOM;
+      } else {
+        const int e = s_ids[i];
+        const int32_t kv = t.key[v];
+        if (kv >= 0) t.slot_of[kv] = -1;
+        t.key[v] = layer * E + e;
+        t.slot_of[(size_t)layer * E + e] = v;
+        held[v >> 5] |= 1u << (v & 31);
+        t.tick[v] = ++ctr[moe::DC_CLOCK];
+        ++ctr[moe::DC_MISSES];
+        t.jobs[s_nj] = v;
+        t.jobs[moe::kMaxResolveIds + s_nj] = layer * E + e;
+        ++s_nj;
+        s_slot[i] = v;
+      }
+    }
+    __syncthreads();
+    if (s_abort) break;
+  }
+  if (tid == 0) {
+    if (s_abort) {
+      // undo this call's assignments: their slots were never filled (the
+      // experts they held before are gone, as on the host)
+      for (int j = 0; j < s_nj; ++j) {
+        t.slot_of[t.jobs[moe::kMaxResolveIds + j]] = -1;
+        t.key[t.jobs[j]] = -1;
+      }
+      ctr[moe::DC_MISSES] -= (uint64_t)s_nj;
+    }
+    *t.njobs = s_abort ? 0 : s_nj;
+  }
+  if (!s_abort && tid < n) {
+    const int e = s_ids[tid];
+    int sl = s_slot[tid];
+    if (sl >= 0 || (e >= 0 && e < E && (sl = t.slot_of[(size_t)layer * E + e]) >= 0))
+      eptr[e] = slots + (size_t)sl * blob;
+  }
+}
+
+// Copies the fills of the last resolve from the mapped host store into their
+// slots, 16 bytes per load, four loads in flight per thread; returns at once
+// when nothing missed.  The last block to finish adds the bytes and the
+// span of the copy (device timestamps) to the counters.
+__global__ void __launch_bounds__(256) stream_fill_kernel(moe::DevTables t, const uint8_t* __restrict__ host,
+                                                          uint8_t* slots, size_t blob) {
+  const int nj = *t.njobs;
+  if (nj == 0) return;
+  uint64_t* ctr = t.ctr;
+  __shared__ int s_last;
+  if (threadIdx.x == 0) {
+    uint64_t now;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+    atomicMin(reinterpret_cast<unsigned long long*>(&ctr[moe::DC_FILL_T0]), (unsigned long long)now);
+  }
+  const size_t per = blob / 16;
+  const size_t total = (size_t)nj * per;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t u0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x; u0 < total; u0 += 4 * stride) {
+    uint4 v[4];
+    size_t dst[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const size_t u = u0 + (size_t)k * stride;
+      if (u < total) {
+        const size_t j = u / per, off = u - j * per;
+        const size_t src = (size_t)t.jobs[moe::kMaxResolveIds + j] * blob + 16 * off;
+        v[k] = *reinterpret_cast<const uint4*>(host + src);
+        dst[k] = (size_t)t.jobs[j] * blob + 16 * off;
+      } else {
+        dst[k] = ~size_t(0);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (dst[k] != ~size_t(0)) *reinterpret_cast<uint4*>(slots + dst[k]) = v[k];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    uint64_t now;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+    atomicMax(reinterpret_cast<unsigned long long*>(&ctr[moe::DC_FILL_T1]), (unsigned long long)now);
+    __threadfence();
+    s_last = atomicAdd(reinterpret_cast<unsigned long long*>(&ctr[moe::DC_FILL_DONE]), 1ull) ==
+             (unsigned long long)gridDim.x - 1ull;
+  }
+  __syncthreads();
+  if (s_last && threadIdx.x == 0) {
+    __threadfence();
+    volatile uint64_t* vc = ctr;
+    vc[moe::DC_FILL_NS] += vc[moe::DC_FILL_T1] - vc[moe::DC_FILL_T0];
+    vc[moe::DC_BYTES] += (uint64_t)nj * blob;
+    vc[moe::DC_FILLS] += 1;
+    vc[moe::DC_FILL_T0] = ~0ull;
+    vc[moe::DC_FILL_T1] = 0;
+    vc[moe::DC_FILL_DONE] = 0;
+  }
 }
 
 }  // namespace
@@ -484,6 +719,8 @@ moe_status moe_stream_file_stats(const moe_stream_cache* c, uint64_t* reads, uin
 moe_status moe_stream_prefetch(moe_stream_cache* c, int layer, const int32_t* ids, int n, cudaStream_t copy_stream) {
   if (!c) return failf(MOE_ERR_INVALID_ARG, "cache is NULL");
   std::lock_guard<std::mutex> lk(c->mu);
+  if (c->mode == 2) return failf(MOE_ERR_INVALID_ARG, "this cache is resolved on the device");
+  c->mode = 1;
   moe_status s = check_ids(c, layer, ids, n);
   if (s != MOE_OK) return s;
   DeviceGuard dg(c->device);
@@ -503,6 +740,8 @@ moe_status moe_stream_resolve(moe_stream_cache* c, int layer, const int32_t* idx
   if (!c) return failf(MOE_ERR_INVALID_ARG, "cache is NULL");
   if (!expert_ptr_dev) return failf(MOE_ERR_INVALID_ARG, "expert_ptr_dev is NULL");
   std::lock_guard<std::mutex> lk(c->mu);
+  if (c->mode == 2) return failf(MOE_ERR_INVALID_ARG, "this cache is resolved on the device");
+  c->mode = 1;
   moe_status s = check_ids(c, layer, idx, n);
   if (s != MOE_OK) return s;
   DeviceGuard dg(c->device);
@@ -555,6 +794,34 @@ moe_status moe_stream_resolve(moe_stream_cache* c, int layer, const int32_t* idx
   return MOE_OK;
 }
 
+moe_status moe_stream_resolve_device(moe_stream_cache* c, int layer, const int32_t* idx_dev, int n,
+                                     const void** expert_ptr_dev, cudaStream_t st) {
+  if (!c) return failf(MOE_ERR_INVALID_ARG, "cache is NULL");
+  if (!expert_ptr_dev || (n > 0 && !idx_dev)) return failf(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (n < 0 || n > moe::kMaxResolveIds)
+    return failf(MOE_ERR_INVALID_ARG, "n = %d: a device resolve takes 0..%d ids", n, moe::kMaxResolveIds);
+  if (layer < 0 || layer >= c->L) return failf(MOE_ERR_INVALID_ARG, "layer %d outside [0, %d)", layer, c->L);
+  std::lock_guard<std::mutex> lk(c->mu);
+  if (!c->host || !c->host_dev)
+    return failf(MOE_ERR_UNSUPPORTED, "device resolves need a pinned host store the device can map");
+  if (c->mode == 1) return failf(MOE_ERR_INVALID_ARG, "this cache is resolved on the host");
+  c->mode = 2;
+  if (n == 0) return MOE_OK;
+  DeviceGuard dg(c->device);
+  const size_t held = 4ull * ((size_t)(c->S + 31) / 32);
+  if (held > 48 * 1024) return failf(MOE_ERR_UNSUPPORTED, "more than %d slots", 48 * 1024 * 8);
+  stream_resolve_kernel<<<1, 1024, held, st>>>(c->dt, c->E, c->S, layer, idx_dev, n, expert_ptr_dev, c->slots,
+                                               c->blob);
+  cudaError_t err = cudaGetLastError();
+  if (err == cudaSuccess) {
+    const int grid = c->sms > 0 ? 4 * c->sms : 256;
+    stream_fill_kernel<<<grid, 256, 0, st>>>(c->dt, c->host_dev, c->slots, c->blob);
+    err = cudaGetLastError();
+  }
+  if (err != cudaSuccess) return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(err));
+  return MOE_OK;
+}
+
 moe_status moe_stream_inject_fault(moe_stream_cache* c, int what, int countdown) {
   if (what == MOE_FAULT_NONE) {
     if (c) {
@@ -595,6 +862,21 @@ moe_status moe_stream_copy_timing(moe_stream_cache* c, moe_stream_copy_times* ou
   if (!c || !out) return failf(MOE_ERR_INVALID_ARG, "NULL pointer");
   std::lock_guard<std::mutex> lk(c->mu);
   DeviceGuard dg(c->device);
+  if (c->mode == 2) {
+    // the fill kernels' own spans and bytes since the last call
+    uint64_t v[moe::DC_N];
+    const cudaError_t err = cudaDeviceSynchronize();
+    if (err != cudaSuccess || cudaMemcpy(v, c->dt.ctr, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+      return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(cudaGetLastError()));
+    out->busy_ms = (double)(v[moe::DC_FILL_NS] - c->dev_seen_ns) * 1e-6;
+    out->copy_ms = out->busy_ms;
+    out->copies = v[moe::DC_FILLS] - c->dev_seen_fills;
+    out->bytes = v[moe::DC_BYTES] - c->dev_seen_bytes;
+    c->dev_seen_ns = v[moe::DC_FILL_NS];
+    c->dev_seen_fills = v[moe::DC_FILLS];
+    c->dev_seen_bytes = v[moe::DC_BYTES];
+    return MOE_OK;
+  }
   std::vector<std::pair<double, double>> iv;
   double sum = 0.0;
   for (auto& pr : c->timed) {
@@ -634,6 +916,20 @@ moe_status moe_stream_copy_timing(moe_stream_cache* c, moe_stream_copy_times* ou
 moe_status moe_stream_stats(const moe_stream_cache* c, moe_stream_counters* out) {
   if (!c || !out) return failf(MOE_ERR_INVALID_ARG, "NULL pointer");
   std::lock_guard<std::mutex> lk(const_cast<moe_stream_cache*>(c)->mu);
+  out->device_error = 0;
+  if (c->mode == 2) {
+    uint64_t v[moe::DC_N];
+    DeviceGuard dg(c->device);
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpy(v, c->dt.ctr, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+      return failf(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(cudaGetLastError()));
+    out->hits = v[moe::DC_HITS];
+    out->misses = v[moe::DC_MISSES];
+    out->prefetches = out->prefetch_hits = out->prefetch_dropped = 0;
+    out->bytes_h2d = v[moe::DC_BYTES];
+    out->device_error = v[moe::DC_ERROR];
+    return MOE_OK;
+  }
   const moe::StreamPolicy& p = c->pol;
   out->hits = p.hits;
   out->misses = p.misses;

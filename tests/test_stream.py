@@ -402,6 +402,104 @@ def test_streaming_overlapped_matches_resident(M):
         M.moe_stream_destroy(cache)
 
 
+# ---- resolved on the device ---------------------------------------------------------------
+
+def _run_device_resolved(M, lay, n_slots, steps, tokens):
+    """Every layer's router, moe_stream_resolve_device and the routed call
+    enqueued back to back on one stream with one synchronisation at the end
+    (the routing never reaches the host); outputs must equal the resident
+    routed call's bit for bit, and the device counters RefCache's (fed the
+    same routing afterwards)."""
+    import torch
+    s, L, E = lay.s, lay.L, lay.s.n_experts
+    plan = []
+    for step in range(steps):
+        for l in range(L):
+            dl = lay.layers[l]
+            x, res = S.activations(s, step=step, tokens=tokens, replica=l)
+            xd, rd = to_dev_bits(x), to_dev_bits(res)
+            idd = torch.empty((tokens, s.top_k), dtype=torch.int32, device="cuda")
+            wd = torch.empty((tokens, s.top_k), dtype=torch.float32, device="cuda")
+            lg = torch.empty((tokens, s.n_experts), dtype=torch.float32, device="cuda")
+            M.moe_router_topk(dl.cfg, xd, dl.wr, dl.bias, idd, wd, logits_out=lg)
+            h1, y1 = torch.empty_like(xd), torch.empty_like(xd)
+            M.moe_layer_forward_routed(lay.cfg, dl.wts, xd, rd, idd, wd, h1, y1, dl.ws)
+            plan.append((l, xd, rd, idd, wd, h1, y1))
+    torch.cuda.synchronize()
+    cache = M.moe_stream_create(lay.cfg, L, lay.store, n_slots)
+    table = torch.zeros(E, dtype=torch.int64, device="cuda")
+    ws = torch.zeros(M.moe_layer_workspace_bytes(lay.cfg, 8), dtype=torch.uint8, device="cuda")
+    M.moe_workspace_init(ws)
+    outs = []
+    try:
+        for l, xd, rd, idd, wd, _, _ in plan:
+            dl = lay.layers[l]
+            M.moe_stream_resolve_device(cache, l, idd, table)
+            wts = M.layer_weights(table, None, None, dl.sg, dl.su, dl.sd, dl.gamma)
+            h2, y2 = torch.empty_like(xd), torch.empty_like(xd)
+            M.moe_layer_forward_routed(lay.cfg, wts, xd, rd, idd, wd, h2, y2, ws)
+            outs.append((h2, y2))
+        torch.cuda.synchronize()
+        assert M.moe_device_error(ws)[0] == 0
+        for i, ((h2, y2), p) in enumerate(zip(outs, plan)):
+            assert np.array_equal(from_dev_bits(h2), from_dev_bits(p[5])), i
+            assert np.array_equal(from_dev_bits(y2), from_dev_bits(p[6])), i
+        ref = RefCache(n_slots)
+        for l, _, _, idd, _, _, _ in plan:
+            ref.resolve(l, idd.cpu().numpy().ravel().tolist())
+        st = M.moe_stream_stats(cache)
+        assert st["device_error"] == 0
+        for k in ("hits", "misses"):
+            assert st[k] == ref.c[k], (k, st, ref.c)
+        assert st["bytes_h2d"] == st["misses"] * lay.nb
+        ct = M.moe_stream_copy_timing(cache)
+        assert ct["bytes"] == st["bytes_h2d"] and (ct["busy_ms"] > 0) == (st["misses"] > 0)
+        # the cache stays bound to device resolves
+        with pytest.raises(M.MoeError):
+            M.moe_stream_resolve(cache, 0, np.array([0], np.int32), table)
+        return st
+    finally:
+        torch.cuda.synchronize()
+        M.moe_stream_destroy(cache)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("tokens", [1, 3])
+def test_device_resolved_streaming_matches_resident_tiny(M, tokens):
+    lay = _Layers(M, replace(S.TINY, tokens=2), n_layers=3)
+    # enough slots that later tokens find some experts resident, too few for
+    # all 3 layers' experts (evictions)
+    st = _run_device_resolved(M, lay, n_slots=7 if tokens == 1 else 20, steps=5, tokens=tokens)
+    assert st["misses"] > 0 and st["hits"] > 0
+
+
+@pytest.mark.gpu
+def test_device_resolved_streaming_h4096(M):
+    s = replace(S.QWEN_4BIT, name="h4096_e64_k4_i1024_4bit", n_experts=64, tokens=1)
+    lay = _Layers(M, s, n_layers=2, device_pack=True)
+    st = _run_device_resolved(M, lay, n_slots=10, steps=4, tokens=1)
+    assert st["misses"] > 0
+
+
+@pytest.mark.gpu
+def test_device_resolve_reports_too_few_slots(M):
+    """More distinct ids in one call than slots: the kernel leaves
+    MOE_ERR_OOM in the device counters and writes no pointer; nothing faults."""
+    import torch
+    s = replace(S.TINY, tokens=2)
+    lay = _Layers(M, s, n_layers=1)
+    cache = M.moe_stream_create(lay.cfg, 1, lay.store, 2)
+    table = torch.zeros(s.n_experts, dtype=torch.int64, device="cuda")
+    try:
+        M.moe_stream_resolve_device(cache, 0, _dev(np.array([1, 2, 3], np.int32)), table)
+        st = M.moe_stream_stats(cache)
+        assert st["device_error"] == M.STATUS_BY_NAME["MOE_ERR_OOM"]
+        assert not table.cpu().numpy().any()
+    finally:
+        torch.cuda.synchronize()
+        M.moe_stream_destroy(cache)
+
+
 # ---- failures injected on the host (no GPU fault) ------------------------------------
 
 @pytest.mark.gpu
