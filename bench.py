@@ -538,7 +538,10 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None,
+        "dtype": ("u4 x i8 -> i32 (4-bit gate/up, x as two int8 limbs), bf16 -> f32 (router, shared, down)"
+                  if args.bits == 4 else "bf16 -> f32"),
+        "data": "synthetic",
         "config": {"workload": s.name, "hidden": s.hidden, "inter": s.inter, "n_experts": s.n_experts,
                    "top_k": s.top_k, "bits": s.bits, "group": s.group, "tokens_per_step": T,
                    "shared_expert": "bf16", "router_bias": "zipf1.1", "replicas": R,

@@ -112,7 +112,8 @@ enum { FLAG_TOPK = NGO, FLAG_SCNT, FLAG_NOSS, FLAG_EPOCH };
 // ---- shared-memory plan ------------------------------------------------------
 // xf: x as mma A fragments, [token][group][t][8 words]; word 2s is the bf16
 //     pair at columns 16s + 2t (+1) of the group, word 2s+1 the pair at 16s + 8 + 2t.
-// xsum: per (token, group) sum of x.
+// xsum: per token, the G group sums of x, then (4-bit experts) the G
+//     power-of-two scales of x's int8 limbs.
 // hf: routed intermediate as A fragments (hi/lo), [pair][group][t][step] x 16 bytes.
 // hx: per (pair, 8-row block of I) sum of hi + lo.
 struct DecodeSmem {
@@ -142,7 +143,7 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int T, int K, int E, int 
   s.xf = pos;
   pos = align_up(pos + 2ull * T * H, 16);
   s.xsum = pos;
-  pos = align_up(pos + 4ull * T * (H / 64), 16);
+  pos = align_up(pos + 8ull * T * (H / 64), 16);
   s.hs = pos;
   pos = align_up(pos + 4ull * T * I, 16);
   s.hf = pos;
@@ -305,6 +306,15 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D += A * B for one m16n8k32 step, unsigned 8-bit A, signed 8-bit B,
+// 32-bit integer accumulators (exact).
+__device__ __forceinline__ void mma_16832_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // B fragments of the four 16-column steps of one block from this lane's
 // code bytes: each 16-bit half becomes the bf16 number 128 + q (exponent of
 // 128 OR-ed over a code in the low mantissa bits).  Code positions: see the
@@ -438,6 +448,106 @@ __device__ __forceinline__ void load_codes<FMT_Q2>(LaneCodes<FMT_Q2>& c, uint32_
 // bsum: GU [group] sums of x; down [16-row block] sums of hi + lo.
 // Returns in res[m][0] / res[m][1] the unit's sums of rows g and g + 8 (every
 // lane of lane group g holds them).
+// A 4-bit gate/up unit on the integer tensor cores: the same 16 rows x one
+// window of 8 groups x gate and up as routed_unit, with the codes expanded to
+// bytes (one AND for the low nibbles of a code word, a shift and an AND for
+// the high ones: the A fragment of an m16n8k32 step is then the 32 columns
+// of two 16-column steps in a fixed permutation that x's limb fragments
+// follow) and x as its two int8 limbs, each an exact integer dot.  Epilogue
+// per group: s * sigma * (256 * D_hi + D_lo) + beta * X, the codes taken as
+// q itself (no 128 offset); bsum holds the token's G group sums, then its G
+// limb scales.
+__device__ __forceinline__ void routed_unit_gu_i8(uint32_t sl, const Seg& sg, int u, const RoutedGeo& geo,
+                                                  uint32_t bfrag, uint32_t bsum, float (&res)[2][2]) {
+  constexpr int GPW = 8;
+  constexpr int BB = 32 * LaneCodes<FMT_Q4>::kBytes;  // code bytes of one 8x64 block
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  const int wa = u * geo.W, wb = min(wa + geo.W, geo.nwin);
+  uint32_t cbase[2][2], sbase[2][2];
+#pragma unroll
+  for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      cbase[mm][h] = sl + sg.off[2 * mm + h] + (uint32_t)(lane * LaneCodes<FMT_Q4>::kBytes) -
+                     (uint32_t)(sg.gbase * BB);
+      sbase[mm][h] = sl + sg.off[4 + 2 * mm + h] + (uint32_t)(g * 4) - (uint32_t)(sg.gbase * 32);
+    }
+  // this lane's B column: group g of the window
+  const int bg = g;
+#pragma unroll 1
+  for (int w = wa; w < wb; ++w) {
+    const int g0 = GPW * w, nv = min(GPW, geo.G - g0);
+    uint32_t xb[8];  // word 4 * st + 2 * limb + b of this lane's group
+    {
+      const uint32_t a = bfrag + (uint32_t)(((g0 + bg) * 4 + t) * 32);
+      uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+      if (bg < nv) {
+        v0 = lds128(a);
+        v1 = lds128(a + 16);
+      }
+      xb[0] = v0.x, xb[1] = v0.y, xb[2] = v0.z, xb[3] = v0.w;
+      xb[4] = v1.x, xb[5] = v1.y, xb[6] = v1.z, xb[7] = v1.w;
+    }
+    int dh[2][4], dl[2][4];
+#pragma unroll
+    for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) dh[mm][k] = dl[mm][k] = 0;
+#pragma unroll
+    for (int j = 0; j < GPW; ++j) {
+      if (j < nv) {
+        uint2 c[2][2];
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) c[mm][h] = lds64(cbase[mm][h] + (uint32_t)((g0 + j) * BB));
+        const bool on = bg == j;
+        uint32_t bm[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) bm[k] = on ? xb[k] : 0u;
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+          for (int st = 0; st < 2; ++st) {
+            const uint32_t w0 = st ? c[mm][0].y : c[mm][0].x, w1 = st ? c[mm][1].y : c[mm][1].x;
+            const uint32_t a0 = w0 & 0x0F0F0F0Fu, a2 = (w0 >> 4) & 0x0F0F0F0Fu;
+            const uint32_t a1 = w1 & 0x0F0F0F0Fu, a3 = (w1 >> 4) & 0x0F0F0F0Fu;
+            mma_16832_u8s8(dh[mm], a0, a1, a2, a3, bm[4 * st], bm[4 * st + 1]);
+            mma_16832_u8s8(dl[mm], a0, a1, a2, a3, bm[4 * st + 2], bm[4 * st + 3]);
+          }
+      }
+    }
+    // epilogue: D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int n = 2 * t + e;
+      if (n < nv) {
+        const float X = lds32f(bsum + 4u * (uint32_t)(g0 + n));
+        const float sig = lds32f(bsum + 4u * (uint32_t)(geo.G + g0 + n));
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t sw = lds32(sbase[mm][h] + (uint32_t)((g0 + n) * 32));
+            const float sc = __uint_as_float(sw << 16), bi = __uint_as_float(sw & 0xffff0000u);
+            const float dot = __int2float_rn(dh[mm][2 * h + e] * 256 + dl[mm][2 * h + e]) * sig;
+            acc[mm][h] = fmaf(sc, dot, fmaf(bi, X, acc[mm][h]));
+          }
+      }
+    }
+  }
+#pragma unroll
+  for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float v = acc[mm][h];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      res[mm][h] = v;
+    }
+}
+
 template <int FMT, bool GU>
 __device__ __forceinline__ void routed_unit(uint32_t sl, const Seg& sg, int u, const RoutedGeo& geo, uint32_t bfrag,
                                             uint32_t bsum, float (&res)[2][2]) {
@@ -1138,27 +1248,67 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       // bf16 pair at columns 16s + 2t (+1) of the group, word 2s + 1 the pair at
       // 16s + 8 + 2t) and its group sums, built by all consumer threads: piece
       // q is 8 columns of one token, its four words go to t = 0..3
+      // 4-bit experts take x as two int8 limbs per column instead: x is
+      // rounded to an integer multiple of the group's power-of-two scale
+      // sigma = 2^(e - 13) (e the exponent of the group's largest |x|), so
+      // |x / sigma| < 2^14, and split as 256 * hi + lo (hi in [-64, 64], lo
+      // in [-128, 127]).  Their fragment words follow the byte order that
+      // the unit's code expansion gives A: [token][group][t][8 words], word
+      // 4 * st + 2 * limb + b holds the limb at the four columns
+      // 32 st + {2t, 16 + 2t, 2t + 1, 17 + 2t} (b = 0) or
+      // 32 st + {8 + 2t, 24 + 2t, 9 + 2t, 25 + 2t} (b = 1).
       const int np = T * H / 8;
+      const int Gx = H / 64;
 #pragma unroll 1
       for (int q0 = 0; q0 < np; q0 += kConsumers) {
         const int q = q0 + tid;
-        float sm = 0.f;
+        float sm = 0.f, mx = 0.f;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        float xx[8];
         if (q < np) {
-          const uint4 v = reinterpret_cast<const uint4*>(xs)[q];
-          const int tg = q >> 3, o8 = q & 7;  // tg = token * Gh + group
-          uint32_t* dst = reinterpret_cast<uint32_t*>(xf) + (size_t)tg * 32 + o8;
-          dst[0] = v.x;
-          dst[8] = v.y;
-          dst[16] = v.z;
-          dst[24] = v.w;
-          float xx[8];
+          v = reinterpret_cast<const uint4*>(xs)[q];
           unpack_bf16x8(v, xx);
           sm = ((xx[0] + xx[1]) + (xx[2] + xx[3])) + ((xx[4] + xx[5]) + (xx[6] + xx[7]));
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(xx[i]));
         }
         sm += __shfl_xor_sync(0xffffffffu, sm, 1);
         sm += __shfl_xor_sync(0xffffffffu, sm, 2);
         sm += __shfl_xor_sync(0xffffffffu, sm, 4);
-        if (q < np && (q & 7) == 0) xsum[q >> 3] = sm;
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        if (q < np) {
+          const int tg = q >> 3, o8 = q & 7;  // tg = token * Gx + group
+          const int tok = tg / Gx, grp = tg - tok * Gx;
+          if constexpr (FMT == FMT_Q4) {
+            const int ex = max(mx > 0.f ? (int)((__float_as_uint(mx) >> 23) & 0xffu) - 127 : -100, -100);
+            const float up = __uint_as_float((uint32_t)(127 + 13 - ex) << 23);  // 1 / sigma
+            uint8_t* dst = reinterpret_cast<uint8_t*>(xf) + (size_t)tg * 128;
+            const int st = o8 >> 2, blk = o8 & 3;
+            const int b = blk & 1, ihi = blk >> 1;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+              const int xi = __float2int_rn(xx[r] * up);
+              const int hi = (xi + 128) >> 8, lo = xi - (hi << 8);
+              const int t4 = r >> 1, i = ihi + 2 * (r & 1);
+              uint8_t* w = dst + t4 * 32 + (4 * st + b) * 4 + i;
+              w[0] = (uint8_t)(int8_t)hi;  // limb 0: hi
+              w[8] = (uint8_t)(int8_t)lo;  // limb 1: lo (two words on)
+            }
+            if (o8 == 0) {
+              xsum[(size_t)tok * 2 * Gx + grp] = sm;
+              xsum[(size_t)tok * 2 * Gx + Gx + grp] = __uint_as_float((uint32_t)(127 + ex - 13) << 23);
+            }
+          } else {
+            uint32_t* dst = reinterpret_cast<uint32_t*>(xf) + (size_t)tg * 32 + o8;
+            dst[0] = v.x;
+            dst[8] = v.y;
+            dst[16] = v.z;
+            dst[24] = v.w;
+            if (o8 == 0) xsum[(size_t)tok * 2 * Gx + grp] = sm;
+          }
+        }
       }
       consumer_sync();
       if (L.sgate) {
@@ -1247,12 +1397,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
               if (tid == 0 && !(probed & pb)) trace_mark<TRACE>(p, gu ? 11 : 13);
               float r[2][2];
               const uint64_t tu0 = TRACE ? globaltimer_ns() : 0;
-              if (gu)
-                routed_unit<FMT, true>(smem_u32(sl), sg, u, gh, smem_u32(xf + (size_t)(sg.pair / L.KP) * gh.G * 8),
-                                       smem_u32(xsum + (size_t)(sg.pair / L.KP) * gh.G), r);
-              else
+              if (gu) {
+                const uint32_t xfa = smem_u32(xf + (size_t)(sg.pair / L.KP) * gh.G * 8);
+                const uint32_t xsa = smem_u32(xsum + (size_t)(sg.pair / L.KP) * 2 * gh.G);
+                if constexpr (FMT == FMT_Q4)
+                  routed_unit_gu_i8(smem_u32(sl), sg, u, gh, xfa, xsa, r);
+                else
+                  routed_unit<FMT, true>(smem_u32(sl), sg, u, gh, xfa, xsa, r);
+              } else {
                 routed_unit<FMT, false>(smem_u32(sl), sg, u, gi, smem_u32(hf_s + (size_t)sg.pair * gi.G * 256),
                                         smem_u32(hx_s + (size_t)sg.pair * (I / kRowBlock)), r);
+              }
               if (TRACE && tid == 0 && !(probed & pb)) p.trace[(size_t)c * kTraceEntries + (gu ? 100 : 102)] = globaltimer_after(r[0][0]);
               if (TRACE && tid == 0 && nunit < 8) {
                 p.trace[(size_t)c * kTraceEntries + 104 + 2 * nunit] = tu0;
