@@ -103,7 +103,7 @@ moe_status device_info(DeviceInfo* out) {
 }
 
 struct WsPlan {
-  size_t logits, hs, hf, hx, ss, total;
+  size_t logits, hs, hf, hx, ss, route, sstot, total;
 };
 
 // Tokens per launch of the fused kernel: at most kMaxTokensFused, and at
@@ -127,9 +127,13 @@ int tokens_per_launch(const Layout& L, int grid, int max_tokens) {
 // words tagged with the launch's epoch.  Their region follows the 256-byte
 // header in every plan (fused and batched), so no other data of either path
 // is ever written where a later launch looks for its epoch words.
+// Words: the router logits [C][E], the blocks' sums of squares
+// [kMaxGrid][C], the routing block 0 publishes [C][K][2] (index, weight) and
+// the total sums of squares it publishes [C].
 size_t epoch_region_bytes(const Layout& L) {
   const size_t C = (size_t)chunk_tokens(L);
-  return round_up_256(sizeof(uint64_t) * C * L.E) + round_up_256(sizeof(uint64_t) * C * kMaxGrid);
+  return round_up_256(sizeof(uint64_t) * C * L.E) + round_up_256(sizeof(uint64_t) * C * kMaxGrid) +
+         round_up_256(sizeof(uint64_t) * C * L.K * 2) + round_up_256(sizeof(uint64_t) * C);
 }
 
 WsPlan ws_plan(const Layout& L, int T) {
@@ -138,6 +142,8 @@ WsPlan ws_plan(const Layout& L, int T) {
   size_t pos = 256;
   w.logits = pos;
   w.ss = round_up_256(pos + sizeof(uint64_t) * C * L.E);
+  w.route = round_up_256(w.ss + sizeof(uint64_t) * C * kMaxGrid);
+  w.sstot = round_up_256(w.route + sizeof(uint64_t) * C * L.K * 2);
   pos = 256 + epoch_region_bytes(L);
   w.hs = pos;
   pos = round_up_256(pos + sizeof(float) * (size_t)T * L.I);
@@ -406,6 +412,8 @@ static moe_status layer_forward_chunk(const moe_config* cfg, const moe_layer_wei
   p.hf = ws + wp.hf;
   p.hx = reinterpret_cast<float*>(ws + wp.hx);
   p.ss = reinterpret_cast<uint64_t*>(ws + wp.ss);
+  p.route = reinterpret_cast<uint64_t*>(ws + wp.route);
+  p.sstot = reinterpret_cast<uint64_t*>(ws + wp.sstot);
   if (trace && trace_entries < (size_t)grid * 128)
     return fail(MOE_ERR_INVALID_ARG, "trace needs %d entries", grid * 128);
   p.timeout_ns = kTimeoutNs;

@@ -1005,13 +1005,42 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
     // the router logits of every block carry this launch's epoch once they
     // are written: polling them is the router barrier and the top-K's loads
     // in one (warp-uniform, so the top-K runs unsplit)
+    // Block 0 alone polls the E logit words and runs the top-K, then
+    // publishes the routing as 2*T*K epoch words; every other block polls
+    // those few words.  (148 blocks all polling all E words took ~4 us per
+    // exchange in a micro kernel, one block polling and the rest polling one
+    // result ~1 us.)
     const uint32_t epoch = (uint32_t)flags[FLAG_EPOCH];
     if (lane == 0) trace_mark<TRACE>(p, 65);
     bool gr = ok;
+    if (blockIdx.x == 0) {
 #pragma unroll 1
-    for (int t = 0; t < T && gr; ++t)
-      gr = warp_topk_poll(p.logits + (size_t)t * E, epoch, E, K, tkbuf, tk_i + t * KP, tk_w + t * KP, &ctr[5], p.err,
-                          to, sp_grid, TRACE ? p.trace + (size_t)blockIdx.x * kTraceEntries + 73 : nullptr);
+      for (int t = 0; t < T && gr; ++t)
+        gr = warp_topk_poll(p.logits + (size_t)t * E, epoch, E, K, tkbuf, tk_i + t * KP, tk_w + t * KP, &ctr[5],
+                            p.err, to, sp_grid, TRACE ? p.trace + 73 : nullptr);
+      gr = __all_sync(0xffffffffu, gr);
+      __syncwarp();
+      if (gr) {
+#pragma unroll 1
+        for (int j = lane; j < T * K; j += 32) {
+          const int t = j / K, k = j - t * K;
+          st_relaxed_gpu_b64(p.route + 2 * j, ((uint64_t)epoch << 32) | (uint32_t)tk_i[t * KP + k]);
+          st_relaxed_gpu_b64(p.route + 2 * j + 1, epoch_word(epoch, tk_w[t * KP + k]));
+        }
+      }
+    } else if (gr) {
+      __shared__ uint32_t rw[2 * kMaxPairsFused];
+      gr = warp_poll_words(p.route, 2 * T * K, epoch, rw, &ctr[5], p.err, to);
+      __syncwarp();
+      if (gr) {
+#pragma unroll 1
+        for (int j = lane; j < T * K; j += 32) {
+          const int t = j / K, k = j - t * K;
+          tk_i[t * KP + k] = (int)rw[2 * j];
+          tk_w[t * KP + k] = __uint_as_float(rw[2 * j + 1]);
+        }
+      }
+    }
     good = __all_sync(0xffffffffu, gr) ? 1 : 0;
     __syncwarp();
     if (lane == 0) trace_mark<TRACE>(p, 66);
@@ -1661,11 +1690,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         if (lane == 0) st_relaxed_gpu_b64(p.ss + (size_t)c * T + warp, epoch_word(epoch, s));
         if (TRACE && lane == 0 && warp == 0) p.trace[(size_t)c * kTraceEntries + 99] = globaltimer_ns();
       }
-      // RMSNorm: every block polls all blocks' sums of squares (the words are
+      // RMSNorm: block 0 polls all blocks' sums of squares (the words are
       // complete once they carry this launch's epoch), sums them in block
-      // order and normalises its own rows of h
+      // order and publishes the total per token; every other block polls that
+      // one word, then all normalise their own rows of h with the same total
       bool got = true;
-      if (warp < T) {
+      if (warp < T && c != 0) {
+        __shared__ uint32_t s_tot[kMaxTokensFused];
+        got = warp_poll_words(p.sstot + warp, 1, epoch, s_tot + warp, &ctr[5], p.err, p.timeout_ns);
+        __syncwarp();
+        if (lane == 0) {
+          inv[warp] = rsqrtf(__fdividef(__uint_as_float(s_tot[warp]), (float)H) + L.eps);
+          if (!got) flags[FLAG_NOSS] = 1;  // the total never came
+        }
+      } else if (warp < T) {
         // lane l holds blocks l, l + 32, ...: every pass loads all the words
         // still missing at once, so a pass costs one round trip
         constexpr int kMaxPer = (kMaxGrid + 31) / 32;
@@ -1722,6 +1760,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         for (int i = 0; i < kMaxPer; ++i) s += v[i];
         s = warp_sum(s);
         if (lane == 0) {
+          if (got) st_relaxed_gpu_b64(p.sstot + warp, epoch_word(epoch, s));
           inv[warp] = rsqrtf(__fdividef(s, (float)H) + L.eps);
           if (!got) flags[FLAG_NOSS] = 1;  // some block's sum of squares never came
         }
@@ -1805,7 +1844,7 @@ uint32_t decode_slot_bytes(const Layout& L, int T, int nrows_max, int* nslots) {
   const size_t need[5] = {2ull * L.H + 16, 4ull * L.H + 32, 2ull * L.I + 16,
                           2ull * 2 * 8 * gh.W * per_group + 64, 2ull * 4 * gi.W * per_group + 64};
   for (int ns = kSlots; ns >= 2; --ns) {
-    const size_t other = decode_smem_plan(T, L.KP, L.E, L.H, L.I, nrows_max, ns, 0, smem_opts(L)).total + 1024;
+    const size_t other = decode_smem_plan(T, L.KP, L.E, L.H, L.I, nrows_max, ns, 0, smem_opts(L)).total + 2048;  // + static shared memory and alignment
     if (other >= limit) return 0;
     size_t slot = (limit - other) / ns;
     slot = slot / 1024 * 1024;

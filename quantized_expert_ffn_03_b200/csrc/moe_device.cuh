@@ -78,6 +78,48 @@ __device__ __forceinline__ uint64_t epoch_word(uint32_t epoch, float v) {
   return ((uint64_t)epoch << 32) | __float_as_uint(v);
 }
 
+// Polls words[0..n) (n <= 128, four per lane, all loads of a pass in
+// flight) until every one carries `epoch`; out[i] gets word i's low 32 bits
+// (out may be shared memory; written by the lane that loaded the word).
+// Warp-uniform.  Gives up, returning false, when *abort_flag is raised or the
+// time limit passes (recording device error 1 and raising the flag).
+__device__ __forceinline__ bool warp_poll_words(const uint64_t* words, int n, uint32_t epoch, uint32_t* out,
+                                                uint32_t* abort_flag, uint32_t* err, uint64_t timeout_ns) {
+  const int lane = threadIdx.x & 31;
+  uint32_t need = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (lane + 32 * i < n) need |= 1u << i;
+  uint64_t t0 = 0;
+#pragma unroll 1
+  for (uint32_t it = 0;; ++it) {
+    uint64_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = (need >> i & 1u) ? ld_relaxed_gpu_b64(words + lane + 32 * i) : 0ull;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if ((need >> i & 1u) && (uint32_t)(w[i] >> 32) == epoch) {
+        need &= ~(1u << i);
+        out[lane + 32 * i] = (uint32_t)w[i];
+      }
+    if (__all_sync(0xffffffffu, need == 0u)) return true;
+    if ((it & 31u) == 31u) {
+      int stop = 0;
+      if (lane == 0) {
+        if (t0 == 0) t0 = globaltimer_ns();
+        if (ld_relaxed_gpu(abort_flag) != 0u) {
+          stop = 1;
+        } else if (globaltimer_ns() - t0 > timeout_ns) {
+          atomicCAS(err, 0u, 1u);
+          atomicExch(abort_flag, 1u);
+          stop = 1;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+    }
+  }
+}
+
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }

@@ -19,6 +19,7 @@ namespace moe {
 constexpr int kMaxUnits = 8;
 constexpr int kRowBlock = 16;  // rows of one routed work unit (the mma's M)
 constexpr int kMaxGrid = 256;  // most blocks of a fused-kernel launch (one per SM)
+constexpr int kMaxPairsFused = 64;  // tokens x K of one fused-kernel launch (tokens <= 64 / K)
 struct RoutedGeo {
   int G, gpw, nwin, W, U;
 };
@@ -74,6 +75,8 @@ struct DecodeParams {
   uint8_t* hf;       // routed intermediate as hi/lo bf16 B fragments, 4*T*K*I bytes
   float* hx;         // [T*K][I/16] sums of hi + lo over 16-row blocks
   uint64_t* ss;      // [grid][T] each block's sum of squares of its rows of h, as epoch words
+  uint64_t* route;   // [T][K][2] the routing block 0 found (expert index, weight bits), as epoch words
+  uint64_t* sstot;   // [T] the total sum of squares block 0 found, as epoch words
   uint64_t timeout_ns;
   uint32_t slot_bytes;  // bytes per shared-memory ring slot
   int nslots;           // ring slots (2..4)
