@@ -366,6 +366,12 @@ def print_trace(M, reps, cfg, xs, rs, h_out, y_out, stream, P, R, calls=16):
     starts = [round(float(np.median(rel[:, :, 88 + k])) / 1e3, 3) for k in range(npass)]
     print("trace top-K poll: pass starts (median us) %s; last pass loads returned at %.3f us" %
           (starts, float(np.median(rel[:, :, 96])) / 1e3), file=sys.stderr, flush=True)
+    lead = [float(np.median(rel[:, 0, k])) / 1e3 for k in (73, 96, 78, 79)]
+    others = rel[:, 1:, 78]
+    print("trace routing: block 0 last poll pass starts %.3f, its loads returned %.3f, top-K done %.3f, "
+          "published %.3f us; other blocks have it: median %.3f max %.3f us" %
+          (tuple(lead) + (float(np.median(np.median(others, axis=1))) / 1e3,
+                          float(np.median(others.max(axis=1))) / 1e3)), file=sys.stderr, flush=True)
     it = [float(np.median(rel[:, :, k])) / 1e3 for k in (75, 76, 77)]
     print("trace warp 0 first shared gate/up row part: start %.3f, dot done %.3f, exchange done %.3f us" % tuple(it),
           file=sys.stderr, flush=True)

@@ -1020,6 +1020,7 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
                             p.err, to, sp_grid, TRACE ? p.trace + 73 : nullptr);
       gr = __all_sync(0xffffffffu, gr);
       __syncwarp();
+      if (TRACE && lane == 0) p.trace[78] = globaltimer_ns();
       if (gr) {
 #pragma unroll 1
         for (int j = lane; j < T * K; j += 32) {
@@ -1028,10 +1029,12 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
           st_relaxed_gpu_b64(p.route + 2 * j + 1, epoch_word(epoch, tk_w[t * KP + k]));
         }
       }
+      if (TRACE && lane == 0) p.trace[79] = globaltimer_ns();
     } else if (gr) {
       __shared__ uint32_t rw[2 * kMaxPairsFused];
       gr = warp_poll_words(p.route, 2 * T * K, epoch, rw, &ctr[5], p.err, to);
       __syncwarp();
+      if (TRACE && lane == 0) p.trace[(size_t)blockIdx.x * kTraceEntries + 78] = globaltimer_ns();
       if (gr) {
 #pragma unroll 1
         for (int j = lane; j < T * K; j += 32) {
