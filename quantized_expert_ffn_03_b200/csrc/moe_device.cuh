@@ -519,8 +519,11 @@ static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, ui
   if (!mbar_try_wait(bar, parity)) {
     const uint64_t t0 = globaltimer_ns();
     for (;; ++it) {
-      if (mbar_try_wait(bar, parity)) break;
-      if ((it & 1023u) == 1023u && globaltimer_ns() - t0 > timeout_ns) {
+      // the hardware may suspend the waiting thread (up to 1 us) until the
+      // phase completes: waiting warps then issue almost nothing and leave
+      // the load/store pipe to the warps that work
+      if (mbar_try_wait_sleep(bar, parity, 1000u)) break;
+      if ((it & 15u) == 15u && globaltimer_ns() - t0 > timeout_ns) {
         ok = false;
         break;
       }
