@@ -542,7 +542,8 @@ def run_ours(args):
     abytes = algorithmic_bytes(s, T)
     achieved = abytes / (ms_per_step * 1e-3) / 1e9
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC if args.bits == 4 else METRIC.replace("4-bit", "2-bit"), "value": value,
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
         "dtype": ("u4 x i8 -> i32 (4-bit gate/up, x as two int8 limbs), bf16 -> f32 (router, shared, down)"

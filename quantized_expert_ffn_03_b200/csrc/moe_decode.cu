@@ -457,10 +457,15 @@ __device__ __forceinline__ void load_codes<FMT_Q2>(LaneCodes<FMT_Q2>& c, uint32_
 // per group: s * sigma * (256 * D_hi + D_lo) + beta * X, the codes taken as
 // q itself (no 128 offset); bsum holds the token's G group sums, then its G
 // limb scales.
+// 2-bit codes: one 32-bit word per lane and 8x64 block expands into four
+// byte registers R_k = (w >> 2k) & 0x03030303; step 0 takes R_0, R_1 and
+// step 1 R_2, R_3 (the 64 columns split into two fixed sets of 32).
+template <int FMT>
 __device__ __forceinline__ void routed_unit_gu_i8(uint32_t sl, const Seg& sg, int u, const RoutedGeo& geo,
                                                   uint32_t bfrag, uint32_t bsum, float (&res)[2][2]) {
   constexpr int GPW = 8;
-  constexpr int BB = 32 * LaneCodes<FMT_Q4>::kBytes;  // code bytes of one 8x64 block
+  constexpr int CB = LaneCodes<FMT>::kBytes;
+  constexpr int BB = 32 * CB;  // code bytes of one 8x64 block
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
   const int wa = u * geo.W, wb = min(wa + geo.W, geo.nwin);
@@ -469,8 +474,7 @@ __device__ __forceinline__ void routed_unit_gu_i8(uint32_t sl, const Seg& sg, in
   for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      cbase[mm][h] = sl + sg.off[2 * mm + h] + (uint32_t)(lane * LaneCodes<FMT_Q4>::kBytes) -
-                     (uint32_t)(sg.gbase * BB);
+      cbase[mm][h] = sl + sg.off[2 * mm + h] + (uint32_t)(lane * CB) - (uint32_t)(sg.gbase * BB);
       sbase[mm][h] = sl + sg.off[4 + 2 * mm + h] + (uint32_t)(g * 4) - (uint32_t)(sg.gbase * 32);
     }
   // this lane's B column: group g of the window
@@ -497,25 +501,44 @@ __device__ __forceinline__ void routed_unit_gu_i8(uint32_t sl, const Seg& sg, in
 #pragma unroll
     for (int j = 0; j < GPW; ++j) {
       if (j < nv) {
-        uint2 c[2][2];
-#pragma unroll
-        for (int mm = 0; mm < 2; ++mm)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) c[mm][h] = lds64(cbase[mm][h] + (uint32_t)((g0 + j) * BB));
         const bool on = bg == j;
         uint32_t bm[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) bm[k] = on ? xb[k] : 0u;
+        if constexpr (FMT == FMT_Q4) {
+          uint2 c[2][2];
 #pragma unroll
-        for (int mm = 0; mm < 2; ++mm)
+          for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
-          for (int st = 0; st < 2; ++st) {
-            const uint32_t w0 = st ? c[mm][0].y : c[mm][0].x, w1 = st ? c[mm][1].y : c[mm][1].x;
-            const uint32_t a0 = w0 & 0x0F0F0F0Fu, a2 = (w0 >> 4) & 0x0F0F0F0Fu;
-            const uint32_t a1 = w1 & 0x0F0F0F0Fu, a3 = (w1 >> 4) & 0x0F0F0F0Fu;
-            mma_16832_u8s8(dh[mm], a0, a1, a2, a3, bm[4 * st], bm[4 * st + 1]);
-            mma_16832_u8s8(dl[mm], a0, a1, a2, a3, bm[4 * st + 2], bm[4 * st + 3]);
-          }
+            for (int h = 0; h < 2; ++h) c[mm][h] = lds64(cbase[mm][h] + (uint32_t)((g0 + j) * BB));
+#pragma unroll
+          for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int st = 0; st < 2; ++st) {
+              const uint32_t w0 = st ? c[mm][0].y : c[mm][0].x, w1 = st ? c[mm][1].y : c[mm][1].x;
+              const uint32_t a0 = w0 & 0x0F0F0F0Fu, a2 = (w0 >> 4) & 0x0F0F0F0Fu;
+              const uint32_t a1 = w1 & 0x0F0F0F0Fu, a3 = (w1 >> 4) & 0x0F0F0F0Fu;
+              mma_16832_u8s8(dh[mm], a0, a1, a2, a3, bm[4 * st], bm[4 * st + 1]);
+              mma_16832_u8s8(dl[mm], a0, a1, a2, a3, bm[4 * st + 2], bm[4 * st + 3]);
+            }
+        } else {
+          uint32_t c[2][2];
+#pragma unroll
+          for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) c[mm][h] = lds32(cbase[mm][h] + (uint32_t)((g0 + j) * BB));
+#pragma unroll
+          for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int st = 0; st < 2; ++st) {
+              const uint32_t a0 = (c[mm][0] >> (4 * st)) & 0x03030303u;
+              const uint32_t a2 = (c[mm][0] >> (4 * st + 2)) & 0x03030303u;
+              const uint32_t a1 = (c[mm][1] >> (4 * st)) & 0x03030303u;
+              const uint32_t a3 = (c[mm][1] >> (4 * st + 2)) & 0x03030303u;
+              mma_16832_u8s8(dh[mm], a0, a1, a2, a3, bm[4 * st], bm[4 * st + 1]);
+              mma_16832_u8s8(dl[mm], a0, a1, a2, a3, bm[4 * st + 2], bm[4 * st + 3]);
+            }
+        }
       }
     }
     // epilogue: D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]
@@ -1276,19 +1299,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       consumer_sync();
     }
     {
-      // x as tensor-core fragments ([token][group][t][8 words]: word 2s is the
-      // bf16 pair at columns 16s + 2t (+1) of the group, word 2s + 1 the pair at
-      // 16s + 8 + 2t) and its group sums, built by all consumer threads: piece
-      // q is 8 columns of one token, its four words go to t = 0..3
-      // 4-bit experts take x as two int8 limbs per column instead: x is
-      // rounded to an integer multiple of the group's power-of-two scale
-      // sigma = 2^(e - 13) (e the exponent of the group's largest |x|), so
-      // |x / sigma| < 2^14, and split as 256 * hi + lo (hi in [-64, 64], lo
-      // in [-128, 127]).  Their fragment words follow the byte order that
-      // the unit's code expansion gives A: [token][group][t][8 words], word
-      // 4 * st + 2 * limb + b holds the limb at the four columns
-      // 32 st + {2t, 16 + 2t, 2t + 1, 17 + 2t} (b = 0) or
-      // 32 st + {8 + 2t, 24 + 2t, 9 + 2t, 25 + 2t} (b = 1).
+      // x as the gate/up units' B fragments, with its group sums and scales,
+      // built by all consumer threads (piece q is 8 columns of one token):
+      // x is rounded to an integer multiple of the group's power-of-two
+      // scale sigma = 2^(e - 13) (e the exponent of the group's largest |x|),
+      // so |x / sigma| < 2^14, and split as 256 * hi + lo (hi in [-64, 64],
+      // lo in [-128, 127]).  The fragment words follow the column order that
+      // the units' code expansion gives A: [token][group][t][8 words], word
+      // 4 * st + 2 * limb + b holds one limb at four columns of step st; for
+      // 4-bit codes 32 st + {2t, 16 + 2t, 2t + 1, 17 + 2t} (b = 0) or
+      // 32 st + {8 + 2t, 24 + 2t, 9 + 2t, 25 + 2t} (b = 1); for 2-bit codes
+      // 16 st + {2t, 32 + 2t, 2t + 1, 33 + 2t} (b = 0) or
+      // 16 st + {8 + 2t, 40 + 2t, 9 + 2t, 41 + 2t} (b = 1).
       const int np = T * H / 8;
       const int Gx = H / 64;
 #pragma unroll 1
@@ -1313,12 +1335,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         if (q < np) {
           const int tg = q >> 3, o8 = q & 7;  // tg = token * Gx + group
           const int tok = tg / Gx, grp = tg - tok * Gx;
-          if constexpr (FMT == FMT_Q4) {
+          {
             const int ex = max(mx > 0.f ? (int)((__float_as_uint(mx) >> 23) & 0xffu) - 127 : -100, -100);
             const float up = __uint_as_float((uint32_t)(127 + 13 - ex) << 23);  // 1 / sigma
             uint8_t* dst = reinterpret_cast<uint8_t*>(xf) + (size_t)tg * 128;
-            const int st = o8 >> 2, blk = o8 & 3;
-            const int b = blk & 1, ihi = blk >> 1;
+            // this piece's step, B register and byte offset in the units'
+            // column permutation (4-bit: steps of 32 consecutive columns;
+            // 2-bit: the 8-column blocks 0, 1, 4, 5 then 2, 3, 6, 7)
+            const int st = FMT == FMT_Q4 ? o8 >> 2 : (o8 >> 1) & 1;
+            const int b = o8 & 1;
+            const int ihi = FMT == FMT_Q4 ? (o8 >> 1) & 1 : o8 >> 2;
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
               const int xi = __float2int_rn(xx[r] * up);
@@ -1332,13 +1358,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
               xsum[(size_t)tok * 2 * Gx + grp] = sm;
               xsum[(size_t)tok * 2 * Gx + Gx + grp] = __uint_as_float((uint32_t)(127 + ex - 13) << 23);
             }
-          } else {
-            uint32_t* dst = reinterpret_cast<uint32_t*>(xf) + (size_t)tg * 32 + o8;
-            dst[0] = v.x;
-            dst[8] = v.y;
-            dst[16] = v.z;
-            dst[24] = v.w;
-            if (o8 == 0) xsum[(size_t)tok * 2 * Gx + grp] = sm;
           }
         }
       }
@@ -1432,10 +1451,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
               if (gu) {
                 const uint32_t xfa = smem_u32(xf + (size_t)(sg.pair / L.KP) * gh.G * 8);
                 const uint32_t xsa = smem_u32(xsum + (size_t)(sg.pair / L.KP) * 2 * gh.G);
-                if constexpr (FMT == FMT_Q4)
-                  routed_unit_gu_i8(smem_u32(sl), sg, u, gh, xfa, xsa, r);
-                else
-                  routed_unit<FMT, true>(smem_u32(sl), sg, u, gh, xfa, xsa, r);
+                routed_unit_gu_i8<FMT>(smem_u32(sl), sg, u, gh, xfa, xsa, r);
               } else {
                 routed_unit<FMT, false>(smem_u32(sl), sg, u, gi, smem_u32(hf_s + (size_t)sg.pair * gi.G * 256),
                                         smem_u32(hx_s + (size_t)sg.pair * (I / kRowBlock)), r);

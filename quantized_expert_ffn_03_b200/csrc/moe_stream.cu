@@ -478,29 +478,45 @@ __global__ void __launch_bounds__(1024) stream_resolve_kernel(moe::DevTables t, 
                                                               const void** __restrict__ eptr, uint8_t* slots,
                                                               size_t blob) {
   extern __shared__ uint32_t held[];  // [(S + 31) / 32] bits: slots taken by this call
-  __shared__ int s_ids[moe::kMaxResolveIds], s_slot[moe::kMaxResolveIds];
+  __shared__ int s_ids[moe::kMaxResolveIds], s_slot[moe::kMaxResolveIds], s_look[moe::kMaxResolveIds];
+  __shared__ unsigned long long s_tick[moe::kMaxResolveIds];
+  __shared__ int s_jobslot[moe::kMaxResolveIds];  // slots this call's misses took
   __shared__ int s_cur, s_abort, s_nj;
-  __shared__ unsigned long long s_red[32];
+  __shared__ unsigned long long s_red[32], s_clock;
   __shared__ int s_redi[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
   const int nwords = (S + 31) / 32;
+  uint64_t* ctr = t.ctr;
   for (int i = tid; i < nwords; i += blockDim.x) held[i] = 0u;
-  if (tid < n) s_ids[tid] = idx[tid];
+  // every id's table entry in one round trip (thread i looks up id i)
+  if (tid < n) {
+    const int e = idx[tid];
+    s_ids[tid] = e;
+    s_look[tid] = (e >= 0 && e < E) ? t.slot_of[(size_t)layer * E + e] : -2;  // -2: invalid id
+    s_tick[tid] = 0ull;
+  }
   if (tid == 0) {
     s_abort = 0;
     s_nj = 0;
+    s_clock = ctr[moe::DC_CLOCK];
   }
   __syncthreads();
-  uint64_t* ctr = t.ctr;
 #pragma unroll 1
   for (int i = 0; i < n; ++i) {
     if (tid == 0) {
       const int e = s_ids[i];
-      int sl = -2;  // -2: invalid id
-      if (e >= 0 && e < E) sl = t.slot_of[(size_t)layer * E + e];
+      int sl = s_look[i];
+      // an id seen earlier in this call may have been mapped by a miss since,
+      // and a slot looked up before the loop may have been taken by one
+      if (sl != -2) {
+        for (int j = 0; j < s_nj; ++j)
+          if (s_jobslot[j] == sl) sl = -1;
+        for (int q = 0; q < i; ++q)
+          if (s_ids[q] == e) sl = s_slot[q];
+      }
       if (sl >= 0 && !(held[sl >> 5] >> (sl & 31) & 1u)) {
         held[sl >> 5] |= 1u << (sl & 31);
-        t.tick[sl] = ++ctr[moe::DC_CLOCK];
+        s_tick[i] = ++s_clock;  // written to the table after the loop
         ++ctr[moe::DC_HITS];
       }
       s_slot[i] = sl;
@@ -548,10 +564,11 @@ __global__ void __launch_bounds__(1024) stream_resolve_kernel(moe::DevTables t, 
         t.key[v] = layer * E + e;
         t.slot_of[(size_t)layer * E + e] = v;
         held[v >> 5] |= 1u << (v & 31);
-        t.tick[v] = ++ctr[moe::DC_CLOCK];
+        t.tick[v] = ++s_clock;
         ++ctr[moe::DC_MISSES];
         t.jobs[s_nj] = v;
         t.jobs[moe::kMaxResolveIds + s_nj] = layer * E + e;
+        s_jobslot[s_nj] = v;
         ++s_nj;
         s_slot[i] = v;
       }
@@ -570,12 +587,15 @@ __global__ void __launch_bounds__(1024) stream_resolve_kernel(moe::DevTables t, 
       ctr[moe::DC_MISSES] -= (uint64_t)s_nj;
     }
     *t.njobs = s_abort ? 0 : s_nj;
+    ctr[moe::DC_CLOCK] = s_clock;
   }
+  __syncthreads();
+  // the hits' new last-use ticks and the pointer table, one id per thread
   if (!s_abort && tid < n) {
     const int e = s_ids[tid];
-    int sl = s_slot[tid];
-    if (sl >= 0 || (e >= 0 && e < E && (sl = t.slot_of[(size_t)layer * E + e]) >= 0))
-      eptr[e] = slots + (size_t)sl * blob;
+    const int sl = s_slot[tid];
+    if (s_tick[tid] != 0ull) t.tick[sl] = s_tick[tid];
+    if (sl >= 0) eptr[e] = slots + (size_t)sl * blob;
   }
 }
 
