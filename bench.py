@@ -354,22 +354,17 @@ def print_trace(M, reps, cfg, xs, rs, h_out, y_out, stream, P, R, calls=16):
              for n in range(8) if b0[104 + 2 * n] > 0]
     print("trace_block0 warp0 routed units (start, duration): %s" % units, file=sys.stderr, flush=True)
     print("trace sync warp (median us): %s" % json.dumps(sync), file=sys.stderr, flush=True)
-    # router logits: each block's last logit write, the start of the sync
-    # warp's last poll pass, and its number of passes
+    # router logits: each block's last logit write; block 0's poll passes
     lw = rel[:, :, 72]
-    lp = rel[:, :, 73]
-    print("trace logits: last write median %.3f max %.3f us; top-K poll last pass starts median %.3f max %.3f us; "
-          "passes median %.0f" % (np.median(np.median(lw, axis=1)) / 1e3, np.median(lw.max(axis=1)) / 1e3,
-                                  np.median(np.median(lp, axis=1)) / 1e3, np.median(lp.max(axis=1)) / 1e3,
-                                  np.median(t[:, :, 74])), file=sys.stderr, flush=True)
-    npass = int(min(8, np.median(t[:, :, 74])))
-    starts = [round(float(np.median(rel[:, :, 88 + k])) / 1e3, 3) for k in range(npass)]
-    print("trace top-K poll: pass starts (median us) %s; last pass loads returned at %.3f us" %
-          (starts, float(np.median(rel[:, :, 96])) / 1e3), file=sys.stderr, flush=True)
-    lead = [float(np.median(rel[:, 0, k])) / 1e3 for k in (73, 96, 78, 79)]
+    starts = [round(float(np.median(rel[:, 0, 88 + k])) / 1e3, 3) for k in range(8)
+              if np.all(t[:, 0, 88 + k] > 0)]
+    print("trace logits: last write median %.3f max %.3f us; block 0's poll passes start at %s us" %
+          (np.median(np.median(lw, axis=1)) / 1e3, np.median(lw.max(axis=1)) / 1e3, starts),
+          file=sys.stderr, flush=True)
+    lead = [float(np.median(rel[:, 0, k])) / 1e3 for k in (73, 96, 74, 78, 79)]
     others = rel[:, 1:, 78]
-    print("trace routing: block 0 last poll pass starts %.3f, its loads returned %.3f, top-K done %.3f, "
-          "published %.3f us; other blocks have it: median %.3f max %.3f us" %
+    print("trace routing: block 0 last poll pass starts %.3f, its loads returned %.3f, all words seen %.3f, "
+          "top-K done %.3f, published %.3f us; other blocks have it: median %.3f max %.3f us" %
           (tuple(lead) + (float(np.median(np.median(others, axis=1))) / 1e3,
                           float(np.median(others.max(axis=1))) / 1e3)), file=sys.stderr, flush=True)
     it = [float(np.median(rel[:, :, k])) / 1e3 for k in (75, 76, 77)]

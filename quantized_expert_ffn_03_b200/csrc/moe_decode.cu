@@ -1037,6 +1037,10 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
     if (lane == 0) trace_mark<TRACE>(p, 65);
     bool gr = ok;
     if (blockIdx.x == 0) {
+      // first pass only once this block's own router rows are written: a
+      // pass issued during the launch's first burst of weight loads came back
+      // ~4 us later and mostly stale, and the next could only start then
+      if (gr) gr = warp_wait(&evt[EVT_R], 0, to, sp_evt);
 #pragma unroll 1
       for (int t = 0; t < T && gr; ++t)
         gr = warp_topk_poll(p.logits + (size_t)t * E, epoch, E, K, tkbuf, tk_i + t * KP, tk_w + t * KP, &ctr[5],

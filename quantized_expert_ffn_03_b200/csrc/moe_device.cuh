@@ -264,30 +264,37 @@ static __device__ __noinline__ void warp_topk_keys(const float* logits, int E, i
     float v[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __ldcg(logits + min(lane + 32 * i, E - 1));
-    uint64_t kr[16];
+    // 32-bit ordered logits (the high word of topk_key; 0 for no expert);
+    // each round: the largest not-yet-taken value (a tree over the lane's
+    // 16, then a warp maximum), then among the lanes holding it the lowest
+    // expert index (a warp minimum); the owner marks it taken.  No 64-bit
+    // compares, no divergent rescan: a short dependent chain per round.
+    uint32_t u[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int e = lane + 32 * i;
-      kr[i] = e < E ? topk_key(v[i], e) : 0ull;
+      u[i] = e < E ? (uint32_t)(topk_key(v[i], e) >> 32) : 0u;
     }
-    uint64_t mine = 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) mine = kr[i] > mine ? kr[i] : mine;
+    uint32_t taken = 0;
 #pragma unroll 1
     for (int k = 0; k < K; ++k) {
-      const uint32_t hi = (uint32_t)(mine >> 32);
-      const uint32_t hmax = __reduce_max_sync(0xffffffffu, hi);
-      const uint32_t lmax = __reduce_max_sync(0xffffffffu, hi == hmax ? (uint32_t)mine : 0u);
-      const uint64_t best = ((uint64_t)hmax << 32) | lmax;
-      if (lane == 0) {
-        idx[k] = (int)~lmax;
-        w[k] = topk_key_value(best);
-      }
-      if (mine == best) {
-        uint64_t m = 0;
+      uint32_t m[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) m = (kr[i] < best && kr[i] > m) ? kr[i] : m;
-        mine = m;
+      for (int i = 0; i < 16; ++i) m[i] = (taken >> i & 1u) ? 0u : u[i];
+#pragma unroll
+      for (int s2 = 8; s2 > 0; s2 >>= 1)
+#pragma unroll
+        for (int i = 0; i < s2; ++i) m[i] = max(m[i], m[i + s2]);
+      const uint32_t hmax = __reduce_max_sync(0xffffffffu, m[0]);
+      uint32_t eq = 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) eq |= (uint32_t)(u[i] == hmax && !(taken >> i & 1u)) << i;
+      const uint32_t mine = eq ? (uint32_t)(lane + 32 * (__ffs(eq) - 1)) : 0xffffffffu;
+      const uint32_t best = __reduce_min_sync(0xffffffffu, mine);
+      if ((int)(best & 31u) == lane) taken |= 1u << (best >> 5);
+      if (lane == 0) {
+        idx[k] = (int)best;
+        w[k] = topk_key_value((uint64_t)hmax << 32);
       }
     }
   } else {
@@ -354,7 +361,6 @@ static __device__ __noinline__ bool warp_topk_poll(const uint64_t* words, uint32
       if (tr && lane == 0) {
         const uint64_t now = globaltimer_ns();
         tr[0] = now;
-        tr[1] = it + 1;
         if (it < 8) tr[15 + it] = now;  // start of each of the first 8 passes
       }
       uint64_t wv[16];
@@ -369,7 +375,10 @@ static __device__ __noinline__ bool warp_topk_poll(const uint64_t* words, uint32
         }
       ++nit;
       if (tr && lane == 0) tr[23] = globaltimer_after(wv[0] + wv[15]);  // this pass's loads returned
-      if (__all_sync(0xffffffffu, have == need)) return true;
+      if (__all_sync(0xffffffffu, have == need)) {
+        if (tr && lane == 0) tr[1] = globaltimer_ns();  // every word present: the top-K starts
+        return true;
+      }
       if ((it & 31u) == 31u) {
         int stop = 0;
         if (lane == 0) {
