@@ -1013,6 +1013,7 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
   uint32_t* sp_evt = spins ? spins + 5 : nullptr;
   uint32_t* sp_grid = spins ? spins + 6 : nullptr;
   bool ok = warp_wait(xbar, 0, to, spins ? spins + 7 : nullptr);
+  const uint32_t epoch = (uint32_t)flags[FLAG_EPOCH];
   int good;
   if (p.idx_in) {
     // the routing is given: no router barrier, no top-K
@@ -1033,7 +1034,6 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
     // those few words.  (148 blocks all polling all E words took ~4 us per
     // exchange in a micro kernel, one block polling and the rest polling one
     // result ~1 us.)
-    const uint32_t epoch = (uint32_t)flags[FLAG_EPOCH];
     if (lane == 0) trace_mark<TRACE>(p, 65);
     bool gr = ok;
     if (blockIdx.x == 0) {
