@@ -39,6 +39,13 @@ FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["moe_decode.cu", "moe_device.cuh", "moe_layout.h", "moe_kernels.h"]
 
 
+def decode_dtype(bits):
+    """Arithmetic of the fused decode kernel: gate/up on the integer tensor
+    cores (codes times x as two int8 limbs), the rest bf16 with fp32 sums."""
+    return (f"u{bits} x i8 -> i32 ({bits}-bit gate/up, x as two int8 limbs), "
+            "bf16 -> f32 (router, shared, down)")
+
+
 def parse_args(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -541,8 +548,7 @@ def run_ours(args):
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
-        "dtype": ("u4 x i8 -> i32 (4-bit gate/up, x as two int8 limbs), bf16 -> f32 (router, shared, down)"
-                  if args.bits == 4 else "bf16 -> f32"),
+        "dtype": decode_dtype(args.bits),
         "data": "synthetic",
         "config": {"workload": s.name, "hidden": s.hidden, "inter": s.inter, "n_experts": s.n_experts,
                    "top_k": s.top_k, "bits": s.bits, "group": s.group, "tokens_per_step": T,
@@ -799,7 +805,7 @@ def run_streaming(args):
         "metric": "streaming tier: tokens/s through %d layers, experts in pinned host memory" % L,
         "value": args.stream_steps / secs, "unit": "tokens/s", "impl": "ours", "mode": "streaming",
         "n_gpus": 1, "steps": args.stream_steps, "warmup": args.stream_warmup,
-        "ms_per_step": ms / args.stream_steps, "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+        "ms_per_step": ms / args.stream_steps, "higher_is_better": True, "dtype": decode_dtype(s.bits), "data": "synthetic",
         "config": {"workload": "%s_x%d_layers" % (s.name, L), "layers": L, "layers_requested": L_req,
                    "predictor": pred, "resolve": args.stream_resolve,
                    "copier": "fill kernel over mapped host memory" if on_device else "cudaMemcpyAsync",
@@ -906,7 +912,8 @@ def run_batched(args):
                 line = {"metric": "batched MoE-layer tokens/s (T tokens per step)", "value": T / (ms * 1e-3),
                         "unit": "tokens/s", "impl": "ours", "mode": "batched", "path": path, "n_gpus": 1,
                         "steps": steps, "warmup": 3, "ms_per_step": ms, "higher_is_better": True,
-                        "dtype": "f16 x f16 -> f32 (routed), bf16 (shared, router)" if path == "batched" else "f32",
+                        "dtype": ("f16 x f16 -> f32 (routed), bf16 (shared, router)" if path == "batched"
+                                  else decode_dtype(s.bits)),
                         "data": "synthetic",
                         "config": {"workload": "%s_T%d_%s" % (s.name, T, routing), "tokens_per_step": T,
                                    "routing": routing, "replicas": R, "cuda_graph": True},
