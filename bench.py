@@ -69,8 +69,10 @@ def parse_args(argv=None):
                    help="streaming store: pinned host memory, or a file read with parallel pread")
     p.add_argument("--direct-io", action="store_true", help="file store: O_DIRECT reads (bypass the page cache)")
     p.add_argument("--store-path", default="/tmp/moe_expert_store.bin")
-    p.add_argument("--stream-resolve", default="device", choices=("device", "host"),
-                   help="streaming: resolve the routing on the GPU (no host round trip) or on the host")
+    p.add_argument("--stream-resolve", default="fused", choices=("fused", "device", "host"),
+                   help="streaming: each layer as one launch that routes, looks its experts up in the cache and "
+                        "copies the misses (fused), the router, a resolve kernel and the routed layer as "
+                        "separate launches (device), or the routing resolved on the host (host)")
     p.add_argument("--predictor", default="next_router", choices=("next_router", "temporal", "none"),
                    help="streaming prefetch: the next layer's router on this layer's input, the experts the "
                         "next layer chose for the previous token, or no prefetch")
@@ -597,7 +599,12 @@ def run_streaming(args):
     their event-timed intervals), against a 1 GiB pinned copy on the same
     box.  After timing, a few more tokens are checked: every layer's outputs
     must equal, bit for bit, the routed call on the same experts copied
-    straight from the store."""
+    straight from the store.  --stream-resolve device keeps the routing on
+    the GPU: per layer the router, moe_stream_resolve_device (a resolve and a
+    fill kernel) and the routed layer; --stream-resolve fused runs each layer
+    as one moe_layer_forward_streamed launch (routing, cache lookup, copy of
+    the misses by the layer's own blocks, the layer).  Both are captured as a
+    CUDA graph per token and have no prediction."""
     import torch
     import quantized_expert_ffn_03_b200 as M
 
@@ -669,9 +676,12 @@ def run_streaming(args):
     h = torch.empty((1, s.hidden), dtype=torch.int16, device="cuda")
     y = torch.empty_like(h)
 
-    on_device = args.stream_resolve == "device"
+    fused = args.stream_resolve == "fused"
+    on_device = args.stream_resolve in ("device", "fused")
     if on_device and args.store == "file":
-        raise SystemExit("--stream-resolve device needs the pinned store")
+        raise SystemExit("--stream-resolve %s needs the pinned store" % args.stream_resolve)
+    # fused: each layer's weights with its router (the expert table is the cache)
+    wts_f = [M.layer_weights(None, d["wr"], d["bias"], d["sg"], d["su"], d["sd"], d["gamma"]) for d in dense]
     # device-resolved: no prediction (the routing never reaches the host)
     pred = "none" if on_device else args.predictor
     last_idx = [None] * L  # experts each layer chose for the previous token (temporal predictor)
@@ -681,6 +691,15 @@ def run_streaming(args):
         res = torch.randn((1, s.hidden), generator=gen, device="cuda").to(torch.bfloat16).view(torch.int16)
         for l in range(L):
             d = dense[l]
+            if fused:
+                # one launch: route, look the experts up, copy the misses, the layer
+                M.moe_layer_forward_streamed(cfg, wts_f[l], x, res, h, y, cache, l, ws, idx_out=idx_d[0],
+                                             w_out=w_d[0])
+                if record is not None:
+                    record.append((l, x.clone(), res.clone(), idx_d[0].clone(), w_d[0].clone(), h.clone(),
+                                   y.clone()))
+                x, res = y.clone(), h.clone()
+                continue
             if on_device:
                 # router, device resolve (+ fill of the misses), routed layer: back to back
                 M.moe_router_topk(cfg, x, d["wr"], d["bias"], idx_d[0], w_d[0], logits_out=lg[0])
@@ -727,9 +746,12 @@ def run_streaming(args):
             xx, rr = xin, rin
             for l in range(L):
                 d = dense[l]
-                M.moe_router_topk(cfg, xx, d["wr"], d["bias"], idx_d[0], w_d[0], logits_out=lg[0])
-                M.moe_stream_resolve_device(cache, l, idx_d[0], table)
-                M.moe_layer_forward_routed(cfg, wts[l], xx, rr, idx_d[0], w_d[0], hb[l % 2], yb[l % 2], ws)
+                if fused:
+                    M.moe_layer_forward_streamed(cfg, wts_f[l], xx, rr, hb[l % 2], yb[l % 2], cache, l, ws)
+                else:
+                    M.moe_router_topk(cfg, xx, d["wr"], d["bias"], idx_d[0], w_d[0], logits_out=lg[0])
+                    M.moe_stream_resolve_device(cache, l, idx_d[0], table)
+                    M.moe_layer_forward_routed(cfg, wts[l], xx, rr, idx_d[0], w_d[0], hb[l % 2], yb[l % 2], ws)
                 xx, rr = yb[l % 2], hb[l % 2]
 
     checked, mismatches = 0, 0
@@ -808,7 +830,9 @@ def run_streaming(args):
         "ms_per_step": ms / args.stream_steps, "higher_is_better": True, "dtype": decode_dtype(s.bits), "data": "synthetic",
         "config": {"workload": "%s_x%d_layers" % (s.name, L), "layers": L, "layers_requested": L_req,
                    "predictor": pred, "resolve": args.stream_resolve,
-                   "copier": "fill kernel over mapped host memory" if on_device else "cudaMemcpyAsync",
+                   "copier": ("every block of the layer kernel over mapped host memory" if fused else
+                              "fill kernel over mapped host memory" if on_device else "cudaMemcpyAsync"),
+                   "launches_per_layer": 1 if fused else (5 if on_device else 3 + 2 * (pred == "next_router")),
                    "host_available_gb": (avail / 1e9) if avail else None, "slots": NS,
                    "slot_bytes": nb, "host_store_gb": L * E * nb / 1e9, "device_cache_gb": NS * nb / 1e9,
                    "tokens_per_step": 1, "router_bias": "zipf1.1, a different permutation per layer"},

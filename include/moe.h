@@ -466,6 +466,37 @@ moe_status moe_stream_resolve(moe_stream_cache* cache, int layer, const int32_t*
 moe_status moe_stream_resolve_device(moe_stream_cache* cache, int layer, const int32_t* idx_dev, int n,
                                      const void** expert_ptr_dev, cudaStream_t stream);
 
+/* One streamed layer in one launch: moe_layer_forward (router, top-K, the
+ * chosen experts' SwiGLU FFNs, shared expert, combine, residual, RMSNorm;
+ * same arguments, outputs and workspace) with the routed experts taken from
+ * `cache` (layer `layer`) instead of wts->expert_ptr, which is ignored.
+ * Inside the launch, the block that finds the routing applies the device
+ * resolve's policy to the T*K chosen experts (hits touch their slots; a miss
+ * takes the lowest empty slot not held by this call, else the least
+ * recently used one, and is mapped to it), then every block copies its
+ * share of the missed blobs from the pinned host store (mapped host memory,
+ * 16-byte loads) into their slots and waits for the others before the
+ * routed weights are read.  So the stand-alone router, the resolve and the
+ * fill launches of moe_stream_resolve_device are not needed, and the
+ * routing never leaves the GPU (hakusoku "パイプライン概要" reads the GPU's
+ * routing on the CPU before its expert reads; blog.cecily.jp on BigMoeOnEdge
+ * streams the routed experts of each layer on demand).  The cache follows
+ * the same rules as moe_stream_resolve_device (this call and that one may
+ * share a cache); it must have at most 32767 slots and at most 64 per
+ * expert of a layer, and E <= 65535 (MOE_ERR_UNSUPPORTED otherwise), and
+ * must live on the current device with blobs of this layer's shape
+ * (MOE_ERR_INVALID_ARG).  Counters: as moe_stream_resolve_device (hits,
+ * misses, bytes_h2d; no copy timing).  More distinct experts in one launch
+ * than slots: MOE_ERR_OOM in the cache's device error word, the call's
+ * assignments undone, and the layer's device error word (moe_device_error)
+ * reports a bad expert pointer; its outputs are then not written.  Tokens
+ * beyond one launch's limit (64 / K) run in successive launches, each
+ * resolving its own experts. */
+moe_status moe_layer_forward_streamed(const moe_config* cfg, const moe_layer_weights* wts, const void* x_bf16,
+                                      const void* residual_bf16, int T, void* h_out_bf16, void* y_norm_bf16,
+                                      int32_t* idx_out, float* w_out, moe_stream_cache* cache, int layer,
+                                      void* workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Counters since create: resolved experts found resident (hits) or copied
  * on demand (misses), prefetch copies issued, resolved experts that a
  * prefetch had brought in and no resolve had used yet (prefetch_hits),

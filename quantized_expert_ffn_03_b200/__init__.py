@@ -105,6 +105,9 @@ EXPORTS = {
     "moe_stream_resolve": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
     "moe_stream_stats": (C.c_int, [C.c_void_p, C.c_void_p]),
     "moe_stream_resolve_device": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
+    "moe_layer_forward_streamed": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                             C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                             C.c_int, C.c_void_p, C.c_size_t, C.c_void_p]),
     "moe_stream_destroy": (None, [C.c_void_p]),
     "moe_device_error": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
     "moe_noalloc_device_error": (C.c_int, [C.c_void_p, C.c_void_p]),
@@ -404,6 +407,17 @@ def moe_stream_resolve_device(cache, layer, idx, expert_ptr, stream=None):
     int64 CUDA tensor [E] (written on the device).  Nothing is read back."""
     _check(_lib.moe_stream_resolve_device(cache, int(layer), _ptr(idx), int(idx.numel()), _ptr(expert_ptr),
                                           _stream(stream)))
+
+
+def moe_layer_forward_streamed(cfg, wts, x, residual, h_out, y_norm, cache, layer, workspace, idx_out=None,
+                               w_out=None, stream=None):
+    """One streamed layer in one launch: the routed experts come from the
+    device-resolved cache `cache` (layer `layer`); wts' expert_ptr is ignored."""
+    T = x.shape[0]
+    _check(_lib.moe_layer_forward_streamed(C.byref(cfg), C.byref(wts), _ptr(x), _ptr(residual), T, _ptr(h_out),
+                                           _ptr(y_norm), _ptr(idx_out), _ptr(w_out), cache, int(layer),
+                                           _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                           _stream(stream)))
 
 
 def moe_stream_stats(cache):

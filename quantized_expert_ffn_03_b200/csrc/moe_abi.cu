@@ -13,6 +13,9 @@
 #include "moe_kernels.h"
 
 namespace moe {
+// The kernel's view of a device-resolved streaming cache (moe_stream.cu).
+moe_status stream_view(moe_stream_cache* c, int layer, int E, uint64_t blob_bytes, StreamView* v);
+
 void pack_host(const Layout& L, const float* wg, const float* wu, const float* wd, int e_begin,
                int e_count, uint8_t* out);
 }
@@ -343,7 +346,7 @@ static moe_status layer_forward_chunk(const moe_config* cfg, const moe_layer_wei
                                       float* w_out, void* workspace, size_t ws_bytes,
                                       void* trace, size_t trace_entries, cudaStream_t stream,
                                       const int32_t* idx_in, const float* w_in, const void* gamma_pre = nullptr,
-                                      void* x_out = nullptr) {
+                                      void* x_out = nullptr, const StreamView* sv = nullptr) {
   Layout L;
   moe_status s = check_cfg(cfg, &L);
   if (s != MOE_OK) return s;
@@ -354,8 +357,8 @@ static moe_status layer_forward_chunk(const moe_config* cfg, const moe_layer_wei
     return fail(MOE_ERR_INVALID_ARG, "bf16 arrays must be 16-byte aligned");
   const bool given = idx_in != nullptr;  // routing given: the router weights are not read
   if (given && !w_in) return fail(MOE_ERR_INVALID_ARG, "NULL routing weights");
-  if (!wts || !wts->expert_ptr || (!given && !wts->router_w) || !wts->gamma || !x_bf16 || !residual_bf16 ||
-      !h_out_bf16 || !y_norm_bf16)
+  if (!wts || (!wts->expert_ptr && !sv) || (!given && !wts->router_w) || !wts->gamma || !x_bf16 ||
+      !residual_bf16 || !h_out_bf16 || !y_norm_bf16)
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
   if (L.has_shared && !L.spacked && (!wts->shared_gate || !wts->shared_up || !wts->shared_down))
     return fail(MOE_ERR_INVALID_ARG, "has_shared=1 but a shared-expert pointer is NULL");
@@ -383,10 +386,12 @@ static moe_status layer_forward_chunk(const moe_config* cfg, const moe_layer_wei
   const size_t smem = decode_smem_bytes(L, T, nrows_max, nslots, slot_bytes);
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  DecodeParams p;
+  DecodeParams p = {};
   p.L = L;
   p.T = T;
-  p.expert_ptr = wts->expert_ptr;
+  p.expert_ptr = sv ? nullptr : wts->expert_ptr;
+  p.streamed = sv ? 1 : 0;
+  if (sv) p.sv = *sv;
   p.wr = static_cast<const uint16_t*>(wts->router_w);
   p.bias = wts->router_bias;
   p.sg = static_cast<const uint16_t*>(wts->shared_gate);
@@ -605,7 +610,8 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
                                      void* h_out_bf16, void* y_norm_bf16, int32_t* idx_out,
                                      float* w_out, void* workspace, size_t ws_bytes,
                                      void* trace, size_t trace_entries, cudaStream_t stream,
-                                     const int32_t* idx_in = nullptr, const float* w_in = nullptr) {
+                                     const int32_t* idx_in = nullptr, const float* w_in = nullptr,
+                                     const StreamView* sv = nullptr) {
   Layout L;
   moe_status s = check_cfg(cfg, &L);
   if (s != MOE_OK) return s;
@@ -616,8 +622,8 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
     return fail(MOE_ERR_UNSUPPORTED, "a traced call takes at most %d tokens", chunk_tokens(L));
   const bool given = idx_in != nullptr;
   if (given && !w_in) return fail(MOE_ERR_INVALID_ARG, "NULL routing weights");
-  if (!wts || !wts->expert_ptr || (!given && !wts->router_w) || !wts->gamma || !x_bf16 || !residual_bf16 ||
-      !h_out_bf16 || !y_norm_bf16)
+  if (!wts || (!wts->expert_ptr && !sv) || (!given && !wts->router_w) || !wts->gamma || !x_bf16 ||
+      !residual_bf16 || !h_out_bf16 || !y_norm_bf16)
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
   weight_opts(wts, &L);
   DeviceInfo di;
@@ -627,7 +633,8 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
     return fail(MOE_ERR_UNSUPPORTED, "shape does not fit the fused kernel's shared memory (H=%d, I=%d)", L.H, L.I);
   if (T <= C)
     return layer_forward_chunk(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out,
-                               workspace, ws_bytes, trace, trace_entries, stream, idx_in, w_in);
+                               workspace, ws_bytes, trace, trace_entries, stream, idx_in, w_in, nullptr, nullptr,
+                               sv);
   if (trace) return fail(MOE_ERR_UNSUPPORTED, "a traced call takes at most %d tokens", C);
   const size_t row = 2ull * (size_t)L.H;
   for (int t0 = 0; t0 < T; t0 += C) {
@@ -637,7 +644,7 @@ static moe_status layer_forward_impl(const moe_config* cfg, const moe_layer_weig
                             static_cast<const uint8_t*>(residual_bf16) + o, n, static_cast<uint8_t*>(h_out_bf16) + o,
                             static_cast<uint8_t*>(y_norm_bf16) + o, idx_out ? idx_out + ok_ : nullptr,
                             w_out ? w_out + ok_ : nullptr, workspace, ws_bytes, nullptr, 0, stream,
-                            idx_in ? idx_in + ok_ : nullptr, w_in ? w_in + ok_ : nullptr);
+                            idx_in ? idx_in + ok_ : nullptr, w_in ? w_in + ok_ : nullptr, nullptr, nullptr, sv);
     if (s != MOE_OK) return s;
   }
   return ok();
@@ -686,6 +693,26 @@ moe_status moe_layer_forward_routed(const moe_config* cfg, const moe_layer_weigh
   if (T > 0 && (!idx || !w)) return fail(MOE_ERR_INVALID_ARG, "NULL routing");
   return layer_forward_impl(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, nullptr, nullptr,
                             workspace, ws_bytes, nullptr, 0, stream, idx, w);
+}
+
+moe_status moe_layer_forward_streamed(const moe_config* cfg, const moe_layer_weights* wts, const void* x_bf16,
+                                      const void* residual_bf16, int T, void* h_out_bf16, void* y_norm_bf16,
+                                      int32_t* idx_out, float* w_out, moe_stream_cache* cache, int layer,
+                                      void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  Layout L;
+  moe_status s = check_cfg(cfg, &L);
+  if (s != MOE_OK) return s;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+  if (!cache) return fail(MOE_ERR_INVALID_ARG, "cache is NULL");
+  if (L.E > kStreamMaxExperts) return fail(MOE_ERR_UNSUPPORTED, "a streamed call takes at most %d experts", kStreamMaxExperts);
+  StreamView v;
+  if ((s = stream_view(cache, layer, L.E, L.blob_bytes, &v)) != MOE_OK) return s;
+  if (v.S > kStreamMaxSlots || v.S > 64 * L.E)
+    return fail(MOE_ERR_UNSUPPORTED, "a streamed call takes at most %d slots (and 64 per expert of a layer)",
+                kStreamMaxSlots);
+  if (T == 0) return ok();
+  return layer_forward_impl(cfg, wts, x_bf16, residual_bf16, T, h_out_bf16, y_norm_bf16, idx_out, w_out,
+                            workspace, ws_bytes, nullptr, 0, stream, nullptr, nullptr, &v);
 }
 
 moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* wts,

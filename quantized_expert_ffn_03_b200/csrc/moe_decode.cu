@@ -44,6 +44,7 @@
 
 #include <mutex>
 
+#include "../../include/moe.h"
 #include "moe_kernels.h"
 #include "moe_device.cuh"
 
@@ -902,7 +903,151 @@ __device__ __forceinline__ void emit_rows(Producer& pr, int type, const uint8_t*
 // buffer, which the register top-K for E <= 512 leaves unused) when it is
 // small and 16-byte aligned.
 __device__ __forceinline__ bool ptab_in_smem(const DecodeParams& p) {
-  return p.L.E <= 512 && (p.L.E & 1) == 0 && (reinterpret_cast<uintptr_t>(p.expert_ptr) & 15u) == 0;
+  return p.expert_ptr != nullptr && p.L.E <= 512 && (p.L.E & 1) == 0 &&
+         (reinterpret_cast<uintptr_t>(p.expert_ptr) & 15u) == 0;
+}
+
+// ---- streamed calls: the expert cache -----------------------------------------------
+// A pair's cache slot as block 0 publishes it (the high half of its index
+// word): the slot, kSlotMiss when its blob is still to be copied in, or
+// kNoSlot when the call found no slot (the cache had too few).
+constexpr uint32_t kSlotMiss = 0x8000u;
+constexpr uint32_t kNoSlot = 0x7fffu;
+
+// Block 0's sync warp, streamed calls: the device resolve's cache policy over
+// the call's T*K chosen experts, in order.  A hit marks its slot held and
+// touches it; a repeat of an expert already held is neither; a miss takes
+// the lowest empty slot that the call does not hold, else the least
+// recently used one it does not hold, unmaps that slot's old expert and maps
+// the new one.  code[j] gets pair j's slot (| kSlotMiss for a miss).  If no
+// slot is left, the call's assignments are undone, MOE_ERR_OOM goes to the
+// cache's error counter and every code is kNoSlot.  held: at least S bits of
+// shared memory.  Returns false on that failure.  Warp-uniform.  (Fields
+// are passed one by one: a reference to the kernel's parameters would make
+// the whole kernel keep them in local memory.)
+__device__ __noinline__ bool warp_stream_resolve(int32_t* slot_of_, int32_t* key_, uint64_t* tick_, uint64_t* dctr_,
+                                                 int S, int layer, int E, uint64_t blob, const int* tk_i, int T,
+                                                 int K, int KP, uint32_t* held, uint32_t* code) {
+  const int lane = threadIdx.x & 31, n = T * K;
+  volatile int32_t* slot_of = slot_of_;
+  volatile int32_t* key = key_;
+  volatile uint64_t* tick = tick_;
+  for (int i = lane; i < (S + 31) / 32; i += 32) held[i] = 0u;
+  // every pair's table entry and the use clock in one round trip (lane q
+  // looks up pairs q and q + 32); entries are read again only after a miss
+  // of this call has changed the table
+  auto pair_key = [&](int j) { return layer * E + tk_i[(j / K) * KP + j % K]; };
+  const int look0 = lane < n ? slot_of[pair_key(lane)] : -1;
+  const int look1 = lane + 32 < n ? slot_of[pair_key(lane + 32)] : -1;
+  uint64_t clock = reinterpret_cast<volatile uint64_t*>(dctr_)[DC_CLOCK];
+  __syncwarp();
+  int nj = 0, nh = 0, j = 0;
+  bool fail = false;
+#pragma unroll 1
+  for (; j < n; ++j) {
+    const int kv = pair_key(j);
+    int sl = __shfl_sync(0xffffffffu, j < 32 ? look0 : look1, j & 31);
+    if (nj > 0) sl = slot_of[kv];
+    if (sl >= 0) {  // a hit, or a repeat of an expert this call holds
+      if (lane == 0) {
+        if (!(held[sl >> 5] >> (sl & 31) & 1u)) {
+          held[sl >> 5] |= 1u << (sl & 31);
+          tick[sl] = ++clock;
+          ++nh;
+        }
+        code[j] = (uint32_t)sl;
+      }
+      __syncwarp();
+      continue;
+    }
+    int be = 0x7fffffff;
+    unsigned long long bl = ~0ull;
+#pragma unroll 1
+    for (int q = lane; q < S; q += 32) {
+      if (held[q >> 5] >> (q & 31) & 1u) continue;
+      if (key[q] < 0) {
+        be = min(be, q);
+      } else {
+        const unsigned long long kk = ((unsigned long long)tick[q] << 24) | (unsigned long long)q;
+        bl = kk < bl ? kk : bl;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      be = min(be, __shfl_xor_sync(0xffffffffu, be, o));
+      const unsigned long long ob = __shfl_xor_sync(0xffffffffu, bl, o);
+      bl = ob < bl ? ob : bl;
+    }
+    const int vs = be != 0x7fffffff ? be : (bl != ~0ull ? (int)(bl & 0xffffffull) : -1);
+    if (vs < 0) {
+      fail = true;
+      break;
+    }
+    if (lane == 0) {
+      const int old = key[vs];
+      if (old >= 0) slot_of[old] = -1;
+      key[vs] = kv;
+      slot_of[kv] = vs;
+      held[vs >> 5] |= 1u << (vs & 31);
+      tick[vs] = ++clock;
+      code[j] = (uint32_t)vs | kSlotMiss;
+    }
+    ++nj;
+    __syncwarp();
+  }
+  if (lane == 0) {
+    if (fail) {
+      // undo: the slots this call took were never filled (the experts they
+      // held before are gone, as with the resolve kernel)
+      for (int q = 0; q < j; ++q)
+        if (code[q] & kSlotMiss) {
+          slot_of[pair_key(q)] = -1;
+          key[code[q] & kNoSlot] = -1;
+        }
+      nj = 0;
+      atomicCAS(reinterpret_cast<unsigned long long*>(&dctr_[DC_ERROR]), 0ull, (unsigned long long)MOE_ERR_OOM);
+      for (int q = 0; q < n; ++q) code[q] = kNoSlot;
+    }
+    // the counters: added, not waited for (the next call's clock read is
+    // ordered by the kernel boundary)
+    atomicAdd(reinterpret_cast<unsigned long long*>(&dctr_[DC_HITS]), (unsigned long long)nh);
+    if (nj > 0) {
+      atomicAdd(reinterpret_cast<unsigned long long*>(&dctr_[DC_MISSES]), (unsigned long long)nj);
+      atomicAdd(reinterpret_cast<unsigned long long*>(&dctr_[DC_BYTES]), (unsigned long long)nj * blob);
+      atomicAdd(reinterpret_cast<unsigned long long*>(&dctr_[DC_FILLS]), 1ull);
+    }
+    reinterpret_cast<volatile uint64_t*>(dctr_)[DC_CLOCK] = clock;
+  }
+  __syncwarp();
+  return !fail;
+}
+
+// Every block's sync warp, streamed calls with misses: this block's share
+// (1/G of each blob, in 16-byte pieces, four loads in flight per lane) of
+// the missed blobs, from the store (host memory the device maps) into their
+// slots.
+__device__ __noinline__ void warp_fill_share(const uint8_t* host, uint8_t* slots, int layer, int E, uint64_t blob,
+                                             const int* tk_i, const uint32_t* code, int T, int K, int KP) {
+  const int lane = threadIdx.x & 31, G = gridDim.x, c = blockIdx.x;
+  const uint64_t per = blob / 16;  // blob is a multiple of 256
+  const uint64_t a = per * (uint64_t)c / (uint64_t)G, b = per * (uint64_t)(c + 1) / (uint64_t)G;
+#pragma unroll 1
+  for (int j = 0; j < T * K; ++j) {
+    if (!(code[j] & kSlotMiss) || code[j] == kNoSlot) continue;
+    const int e = tk_i[(j / K) * KP + j % K];
+    const uint4* src = reinterpret_cast<const uint4*>(host + (uint64_t)(layer * E + e) * blob);
+    uint4* dst = reinterpret_cast<uint4*>(slots + (uint64_t)(code[j] & kNoSlot) * blob);
+#pragma unroll 1
+    for (uint64_t u = a + lane; u < b; u += 4 * 32) {
+      uint4 w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (u + 32 * k < b) w[k] = src[u + 32 * k];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (u + 32 * k < b) dst[u + 32 * k] = w[k];
+    }
+  }
 }
 
 template <bool TRACE>
@@ -951,6 +1096,9 @@ __device__ void run_producer(const DecodeParams& p, Producer& pr, uint16_t* xs, 
   if (pr.ok) {
     if (mbar_wait(topkbar, 0, p.timeout_ns, pr.spins ? pr.spins + 1 : nullptr)) {
       routed = flags[FLAG_TOPK] != 0;
+      // streamed calls: other blocks may have just written the blobs these
+      // copies read (their stores, seen through the fill barrier)
+      if (p.streamed) fence_proxy_async_global();
     } else {
       pr.ok = false;
       atomicCAS(p.err, 0u, 1u);
@@ -1010,6 +1158,7 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
   const int T = p.T, K = L.K, KP = L.KP, E = L.E, G = gridDim.x;
   uint32_t* ctr = p.ctr;
   const uint64_t to = p.timeout_ns;
+  __shared__ uint32_t s_code[kMaxPairsFused];  // streamed calls: each pair's cache slot code
   uint32_t* sp_evt = spins ? spins + 5 : nullptr;
   uint32_t* sp_grid = spins ? spins + 6 : nullptr;
   bool ok = warp_wait(xbar, 0, to, spins ? spins + 7 : nullptr);
@@ -1048,11 +1197,18 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
       gr = __all_sync(0xffffffffu, gr);
       __syncwarp();
       if (TRACE && lane == 0) p.trace[78] = globaltimer_ns();
+      // a streamed call: the chosen experts' cache slots (the key buffer is
+      // free once the top-K is done; it holds the slots' bitmap); a call
+      // that finds too few slots still publishes, with no slot for any pair
+      if (gr && p.streamed)
+        warp_stream_resolve(p.sv.slot_of, p.sv.key, p.sv.tick, p.sv.dctr, p.sv.S, p.sv.layer, E, L.blob_bytes, tk_i,
+                            T, K, KP, reinterpret_cast<uint32_t*>(tkbuf), s_code);
       if (gr) {
 #pragma unroll 1
         for (int j = lane; j < T * K; j += 32) {
           const int t = j / K, k = j - t * K;
-          st_relaxed_gpu_b64(p.route + 2 * j, ((uint64_t)epoch << 32) | (uint32_t)tk_i[t * KP + k]);
+          const uint32_t hi = p.streamed ? s_code[j] << 16 : 0u;
+          st_relaxed_gpu_b64(p.route + 2 * j, ((uint64_t)epoch << 32) | hi | (uint32_t)tk_i[t * KP + k]);
           st_relaxed_gpu_b64(p.route + 2 * j + 1, epoch_word(epoch, tk_w[t * KP + k]));
         }
       }
@@ -1066,8 +1222,9 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
 #pragma unroll 1
         for (int j = lane; j < T * K; j += 32) {
           const int t = j / K, k = j - t * K;
-          tk_i[t * KP + k] = (int)rw[2 * j];
+          tk_i[t * KP + k] = p.streamed ? (int)(rw[2 * j] & 0xffffu) : (int)rw[2 * j];
           tk_w[t * KP + k] = __uint_as_float(rw[2 * j + 1]);
+          if (p.streamed) s_code[j] = rw[2 * j] >> 16;
         }
       }
     }
@@ -1087,10 +1244,12 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
         tk_w[j] = 1.f;
       }
       const int e = shp ? 0 : tk_i[j];
+      const uint32_t sc = p.streamed && !shp ? s_code[t * K + k] & kNoSlot : 0u;
       const void* bp = shp ? reinterpret_cast<const void*>(p.spacked)
-                           : (e >= 0 && e < E) ? (ptab_in_smem(p) ? reinterpret_cast<const void*>(tkbuf[e])
-                                                                  : p.expert_ptr[e])
-                                               : nullptr;
+                       : !(e >= 0 && e < E) ? nullptr
+                       : p.streamed ? (sc == kNoSlot ? nullptr : p.sv.slots + (uint64_t)sc * L.blob_bytes)
+                       : ptab_in_smem(p) ? reinterpret_cast<const void*>(tkbuf[e])
+                                         : p.expert_ptr[e];
       if (bp == nullptr || (reinterpret_cast<uintptr_t>(bp) & 255u)) {
         atomicCAS(p.err, 0u, 2u);
         atomicExch(&ctr[5], 1u);
@@ -1104,6 +1263,24 @@ __device__ void run_sync(const DecodeParams& p, uint64_t* xbar, uint64_t* xfbar,
       }
     }
     good = __all_sync(0xffffffffu, good != 0) ? 1 : 0;
+  }
+  // a streamed call with misses: every block copies its share of the missed
+  // blobs into their slots and waits until every block has (its routed
+  // tiles read them next; the producer orders its copies after this)
+  if (p.streamed && good) {
+    bool miss = false;
+    for (int j = 0; j < T * K; ++j) miss = miss || (s_code[j] & kSlotMiss) != 0u;
+    if (miss) {
+      warp_fill_share(p.sv.host, p.sv.slots, p.sv.layer, E, L.blob_bytes, tk_i, s_code, T, K, KP);
+      __syncwarp();
+      int gf = 1;
+      if (lane == 0) {
+        __threadfence();
+        red_release_add(&ctr[7], 1u);
+        gf = grid_wait_thread(&ctr[7], G, &ctr[5], p.err, to, sp_grid) ? 1 : 0;
+      }
+      good = __shfl_sync(0xffffffffu, gf, 0) ? good : 0;
+    }
   }
   // every lane's eptr store must precede lane 0's release to the producer
   __syncwarp();
@@ -1813,6 +1990,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       volatile uint32_t* vc = reinterpret_cast<volatile uint32_t*>(ctr);
       for (int k = 0; k < 6; ++k) vc[k] = 0u;
       vc[6] = (uint32_t)flags[FLAG_EPOCH];
+      vc[7] = 0u;
     }
   }
   if (tid == 0) trace_mark<TRACE>(p, 8);

@@ -23,6 +23,34 @@ constexpr int kMaxPairsFused = 64;  // tokens x K of one fused-kernel launch (to
 struct RoutedGeo {
   int G, gpw, nwin, W, U;
 };
+
+// Device counters of a device-resolved expert-streaming cache: the use
+// clock, hits, misses, bytes copied, copy time, the error code, and the fill
+// kernel's bookkeeping (blocks done, first and last timestamps, fills).
+enum StreamCounter {
+  DC_CLOCK = 0, DC_HITS, DC_MISSES, DC_BYTES, DC_FILL_NS, DC_ERROR, DC_FILL_DONE, DC_FILL_T0, DC_FILL_T1,
+  DC_FILLS, DC_N
+};
+
+// A device-resolved cache as a streamed layer call sees it: the slot table
+// [L][E] -> slot (or -1), each slot's key (layer * E + expert, or -1) and
+// last use, the counters, the pinned store as the device addresses it
+// ([L][E] blobs), and the slots (one blob each).
+struct StreamView {
+  int32_t* slot_of;
+  int32_t* key;
+  uint64_t* tick;
+  uint64_t* dctr;
+  const uint8_t* host;
+  uint8_t* slots;
+  int S;      // slots
+  int layer;  // the layer of this call
+};
+// A streamed call publishes each pair's slot in 15 bits beside a 16-bit
+// expert index, and keeps the slots it holds as a bitmap in the 8 * E bytes
+// of the top-K key buffer: S <= 32767, S <= 64 * E, E <= 65535.
+constexpr int kStreamMaxSlots = 32767;
+constexpr int kStreamMaxExperts = 65535;
 __host__ __device__ inline RoutedGeo routed_geo(int cols, int gpw) {
   RoutedGeo g;
   g.G = cols / 64;
@@ -45,7 +73,8 @@ __host__ __device__ inline int decode_rows_max(int H, int G) { return 16 * ((H /
 // intermediates.  ctr[1] shared gate/up, [2] routed gate/up, [3] blocks that
 // finished, [5] abort flag of the running launch, [6] the last launch's
 // epoch (each launch publishes its router logits and sums of squares as
-// 64-bit words tagged with its own epoch, ctr[6] + 1).
+// 64-bit words tagged with its own epoch, ctr[6] + 1), [7] blocks done
+// copying a streamed call's missed experts.
 struct DecodeParams {
   Layout L;
   int T;
@@ -75,12 +104,17 @@ struct DecodeParams {
   uint8_t* hf;       // routed intermediate as hi/lo bf16 B fragments, 4*T*K*I bytes
   float* hx;         // [T*K][I/16] sums of hi + lo over 16-row blocks
   uint64_t* ss;      // [grid][T] each block's sum of squares of its rows of h, as epoch words
-  uint64_t* route;   // [T][K][2] the routing block 0 found (expert index, weight bits), as epoch words
+  uint64_t* route;   // [T][K][3] the routing block 0 found (expert index, weight bits, cache slot), as epoch words
   uint64_t* sstot;   // [T] the total sum of squares block 0 found, as epoch words
   uint64_t timeout_ns;
   uint32_t slot_bytes;  // bytes per shared-memory ring slot
   int nslots;           // ring slots (2..4)
   uint64_t* trace;      // optional [grid][64] phase timestamps (ns), or null
+  // streamed layer call (expert_ptr null): block 0 looks the chosen experts
+  // up in the cache, takes slots for the misses, and every block copies its
+  // share of the missed blobs from the store before the routed tiles
+  int streamed;
+  StreamView sv;
 };
 
 constexpr int kDecodeBlockThreads = 512;  // 14 consumer warps, a producer warp, a sync warp

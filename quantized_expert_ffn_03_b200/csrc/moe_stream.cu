@@ -59,6 +59,7 @@
 #include <vector>
 
 #include "../../include/moe.h"
+#include "moe_kernels.h"
 #include "moe_stream_policy.h"
 
 namespace moe {
@@ -153,9 +154,6 @@ constexpr int kFileStage = 16;  // pinned staging buffers of a file-backed store
 namespace moe {
 namespace {
 constexpr int kMaxResolveIds = 64;  // ids of one device-resolved call
-// device counters of a device-resolved cache
-enum { DC_CLOCK = 0, DC_HITS, DC_MISSES, DC_BYTES, DC_FILL_NS, DC_ERROR, DC_FILL_DONE, DC_FILL_T0, DC_FILL_T1,
-       DC_FILLS, DC_N };
 struct DevTables {
   int32_t* slot_of = nullptr;  // [L * E] -> slot, or -1
   int32_t* key = nullptr;      // [S] -> layer * E + expert, or -1
@@ -971,3 +969,37 @@ void moe_stream_destroy(moe_stream_cache* c) {
 }
 
 }  // extern "C"
+
+namespace moe {
+
+// The fused kernel's view of a device-resolved cache for one streamed layer
+// call (moe_layer_forward_streamed): the cache must hold a pinned store the
+// device maps, serve the device-resolved protocol (an unused cache becomes
+// device-resolved), live on the current device and hold blobs of
+// `blob_bytes` for `E` experts per layer.
+moe_status stream_view(moe_stream_cache* c, int layer, int E, uint64_t blob_bytes, StreamView* v) {
+  if (!c || !v) return failf(MOE_ERR_INVALID_ARG, "cache is NULL");
+  if (layer < 0 || layer >= c->L) return failf(MOE_ERR_INVALID_ARG, "layer %d outside [0, %d)", layer, c->L);
+  std::lock_guard<std::mutex> lk(c->mu);
+  if (!c->host || !c->host_dev || !c->dt.slot_of)
+    return failf(MOE_ERR_UNSUPPORTED, "streamed layer calls need a pinned host store the device can map");
+  if (c->mode == 1) return failf(MOE_ERR_INVALID_ARG, "this cache is resolved on the host");
+  if (c->E != E || c->blob != blob_bytes)
+    return failf(MOE_ERR_INVALID_ARG, "the cache holds %d experts of %zu bytes per layer, the layer %d of %llu",
+                 c->E, c->blob, E, (unsigned long long)blob_bytes);
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != c->device) return failf(MOE_ERR_INVALID_ARG, "the cache lives on device %d, not %d", c->device, dev);
+  c->mode = 2;
+  v->slot_of = c->dt.slot_of;
+  v->key = c->dt.key;
+  v->tick = c->dt.tick;
+  v->dctr = c->dt.ctr;
+  v->host = c->host_dev;
+  v->slots = c->slots;
+  v->S = c->S;
+  v->layer = layer;
+  return MOE_OK;
+}
+
+}  // namespace moe

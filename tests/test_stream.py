@@ -500,6 +500,113 @@ def test_device_resolve_reports_too_few_slots(M):
         M.moe_stream_destroy(cache)
 
 
+# ---- streamed layer calls (lookup, fill and layer in one launch) --------------------
+
+def _run_streamed(M, lay, n_slots, steps, tokens):
+    """moe_layer_forward_streamed for every layer of every step, back to back
+    on one stream with one synchronisation at the end: outputs and routing
+    must equal the resident fused call's bit for bit (the same kernel routes
+    both; only where the expert bytes come from differs), and the device
+    counters RefCache's fed the same routing."""
+    import torch
+    s, L, E = lay.s, lay.L, lay.s.n_experts
+    plan = []
+    for step in range(steps):
+        for l in range(L):
+            dl = lay.layers[l]
+            x, res = S.activations(s, step=step, tokens=tokens, replica=l)
+            xd, rd = to_dev_bits(x), to_dev_bits(res)
+            h1, y1 = torch.empty_like(xd), torch.empty_like(xd)
+            i1 = torch.empty((tokens, s.top_k), dtype=torch.int32, device="cuda")
+            w1 = torch.empty((tokens, s.top_k), dtype=torch.float32, device="cuda")
+            M.moe_layer_forward(lay.cfg, dl.wts, xd, rd, h1, y1, i1, w1, dl.ws)
+            plan.append((l, xd, rd, h1, y1, i1, w1))
+    torch.cuda.synchronize()
+    cache = M.moe_stream_create(lay.cfg, L, lay.store, n_slots)
+    ws = torch.zeros(M.moe_layer_workspace_bytes(lay.cfg, 8), dtype=torch.uint8, device="cuda")
+    M.moe_workspace_init(ws)
+    outs = []
+    try:
+        for l, xd, rd, _, _, _, _ in plan:
+            dl = lay.layers[l]
+            wts = M.layer_weights(None, dl.wr, dl.bias, dl.sg, dl.su, dl.sd, dl.gamma)
+            h2, y2 = torch.empty_like(xd), torch.empty_like(xd)
+            i2 = torch.empty((tokens, s.top_k), dtype=torch.int32, device="cuda")
+            w2 = torch.empty((tokens, s.top_k), dtype=torch.float32, device="cuda")
+            M.moe_layer_forward_streamed(lay.cfg, wts, xd, rd, h2, y2, cache, l, ws, idx_out=i2, w_out=w2)
+            outs.append((h2, y2, i2, w2))
+        torch.cuda.synchronize()
+        assert M.moe_device_error(ws)[0] == 0
+        for i, ((h2, y2, i2, w2), p) in enumerate(zip(outs, plan)):
+            assert np.array_equal(i2.cpu().numpy(), p[5].cpu().numpy()), i
+            assert np.array_equal(w2.cpu().numpy(), p[6].cpu().numpy()), i
+            assert np.array_equal(from_dev_bits(h2), from_dev_bits(p[3])), i
+            assert np.array_equal(from_dev_bits(y2), from_dev_bits(p[4])), i
+        ref = RefCache(n_slots)
+        for (l, *_), (_, _, i2, _) in zip(plan, outs):
+            ref.resolve(l, i2.cpu().numpy().ravel().tolist())
+        st = M.moe_stream_stats(cache)
+        assert st["device_error"] == 0
+        for k in ("hits", "misses"):
+            assert st[k] == ref.c[k], (k, st, ref.c)
+        assert st["bytes_h2d"] == st["misses"] * lay.nb
+        # the same cache also serves the separate device resolve
+        table = torch.zeros(E, dtype=torch.int64, device="cuda")
+        M.moe_stream_resolve_device(cache, 0, outs[0][2], table)
+        torch.cuda.synchronize()
+        assert M.moe_stream_stats(cache)["device_error"] == 0
+        return st
+    finally:
+        torch.cuda.synchronize()
+        M.moe_stream_destroy(cache)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("tokens", [1, 3])
+def test_streamed_layer_matches_resident_tiny(M, tokens):
+    lay = _Layers(M, replace(S.TINY, tokens=2), n_layers=3)
+    st = _run_streamed(M, lay, n_slots=7 if tokens == 1 else 20, steps=5, tokens=tokens)
+    assert st["misses"] > 0 and st["hits"] > 0
+
+
+@pytest.mark.gpu
+def test_streamed_layer_h4096(M):
+    s = replace(S.QWEN_4BIT, name="h4096_e64_k4_i1024_4bit", n_experts=64, tokens=1)
+    lay = _Layers(M, s, n_layers=2, device_pack=True)
+    st = _run_streamed(M, lay, n_slots=10, steps=4, tokens=1)
+    assert st["misses"] > 0
+
+
+@pytest.mark.gpu
+def test_streamed_layer_reports_too_few_slots(M):
+    """More distinct experts in one launch than slots: MOE_ERR_OOM in the
+    cache's counters, a bad expert pointer in the layer's error word, the
+    call's assignments undone; nothing faults or waits out."""
+    import torch
+    s = replace(S.TINY, tokens=3)
+    lay = _Layers(M, s, n_layers=1)
+    cache = M.moe_stream_create(lay.cfg, 1, lay.store, 1)
+    dl = lay.layers[0]
+    ws = torch.zeros(M.moe_layer_workspace_bytes(lay.cfg, 8), dtype=torch.uint8, device="cuda")
+    M.moe_workspace_init(ws)
+    try:
+        x, res = S.activations(s, step=0, tokens=3, replica=0)
+        xd, rd = to_dev_bits(x), to_dev_bits(res)
+        h, y = torch.empty_like(xd), torch.empty_like(xd)
+        i2 = torch.empty((3, s.top_k), dtype=torch.int32, device="cuda")
+        wts = M.layer_weights(None, dl.wr, dl.bias, dl.sg, dl.su, dl.sd, dl.gamma)
+        M.moe_layer_forward_streamed(lay.cfg, wts, xd, rd, h, y, cache, 0, ws, idx_out=i2)
+        torch.cuda.synchronize()
+        assert len(set(i2.cpu().numpy().ravel().tolist())) > 1
+        st = M.moe_stream_stats(cache)
+        assert st["device_error"] == M.STATUS_BY_NAME["MOE_ERR_OOM"]
+        assert st["misses"] == 0
+        assert M.moe_device_error(ws)[0] == M.STATUS_BY_NAME["MOE_ERR_DEVICE"]
+    finally:
+        torch.cuda.synchronize()
+        M.moe_stream_destroy(cache)
+
+
 # ---- failures injected on the host (no GPU fault) ------------------------------------
 
 @pytest.mark.gpu
