@@ -39,8 +39,14 @@ namespace moe {
 
 namespace {
 
-constexpr int kGThreads = 160;   // 4 producer/epilogue warps + the MMA warp
-constexpr int kProducers = 128;
+// 4 owner warps (producers and epilogue), the MMA warp (warp 4), 4 helper
+// warps (producers only): each of the tile's 128 rows has an owner thread
+// and a helper thread, which split its copies and dequantisation (the
+// dequantisation of the codes, not the MMA or the bytes, sets the time of
+// the packed GEMMs at a few tokens per expert)
+constexpr int kGThreads = 288;
+constexpr int kProducers = 256;
+constexpr int kMmaWarp = 4;
 constexpr int kTileM = 128;      // output rows per tile (the MMA's M)
 constexpr int kTileN = 128;      // columns (tokens / slots) per tile at most
 constexpr int kKB = 64;          // reduction columns per k-block (one quantisation group)
@@ -191,7 +197,7 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_gemm_kernel(const GemmPa
     bar_init(fin, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc::tmem_alloc(smem_addr((const void*)tmem_slot), kTmemCols);
     tc::tmem_relinquish();
   }
@@ -211,9 +217,18 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_gemm_kernel(const GemmPa
   uint32_t kb_global = 0;  // k-blocks consumed by this CTA so far (stage / phase counter)
   uint32_t tile_iter = 0;
 
-  if (warp < 4) {
-    // ================= producers and epilogue =================
-    const uint32_t row = (uint32_t)tid;  // this thread's A row and TMEM lane
+  if (warp != kMmaWarp) {
+    // ================= producers (and, for the owners, the epilogue) =================
+    // this thread's A row (and, for an owner, its TMEM lane: warp w reaches
+    // lanes 32 (w % 4) ..); half 0 = owner, 1 = helper.  With two A
+    // matrices half h copies and dequantises matrix h; with one, the
+    // k-blocks g (counted over the CTA's tiles, which also picks their code
+    // slot, an even number of them) of parity h, so a helper that runs
+    // ahead into the next tile never writes a slot its owner still reads.
+    // Each half copies half of every k-block's B rows.
+    const uint32_t row = 32u * (uint32_t)(warp & 3) + (uint32_t)lane;
+    const int half = warp > kMmaWarp ? 1 : 0;
+    auto mine = [&](int a, uint32_t g) { return NA == 2 ? a == half : (int)(g & 1u) == half; };
 #pragma unroll 1
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tile_iter) {
       const int chunk = tile / MT, mt = tile - chunk * MT;
@@ -231,11 +246,11 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_gemm_kernel(const GemmPa
       const uint8_t* blob = kPacked ? static_cast<const uint8_t*>(p.expert_ptr[e]) : nullptr;
       // this thread's B rows: chunk id = row + 128 q -> tile row 16 q + row / 8, chunk row % 8
       const int bc = (int)(row & 7u);
-      int brow_src[kTileN / 16];
+      int brow_src[kTileN / 32];  // the B rows of this half: q = half * kTileN / 32 + qq
 #pragma unroll
-      for (int q = 0; q < kTileN / 16; ++q) {
-        const int r = 16 * q + (int)(row >> 3);
-        brow_src[q] = r < n ? (p.b_rows ? p.b_rows[c0 + r] : c0 + r) : -1;
+      for (int qq = 0; qq < kTileN / 32; ++qq) {
+        const int r = 16 * (half * (kTileN / 32) + qq) + (int)(row >> 3);
+        brow_src[qq] = r < n ? (p.b_rows ? p.b_rows[c0 + r] : c0 + r) : -1;
       }
       const uint32_t gbase = kb_global;
       // issue the copies of k-block kb (B and dense A) into its stage
@@ -247,16 +262,18 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_gemm_kernel(const GemmPa
         const int kbb = kb % KB1;
         const uint16_t* bsrc = (kb >= KB1) ? p.b2 : p.b;
 #pragma unroll
-        for (int q = 0; q < kTileN / 16; ++q) {
+        for (int qq = 0; qq < kTileN / 32; ++qq) {
+          const int q = half * (kTileN / 32) + qq;
           const int r = 16 * q + (int)(row >> 3);
           const uint32_t dst = st + L.b0 + tc::sw128((uint32_t)r, (uint32_t)bc);
-          const int src_row = brow_src[q];
+          const int src_row = brow_src[qq];
           const uint16_t* src = bsrc + (size_t)(src_row < 0 ? 0 : src_row) * p.K + kbb * kKB + 8 * bc;
           tc::cp16(dst, src, src_row < 0 ? 0u : 16u);
         }
         if constexpr (!kPacked) {
 #pragma unroll
           for (int a = 0; a < NA; ++a) {
+            if (!mine(a, gbase + (uint32_t)kb)) continue;
             const uint16_t* arow = p.a_dense[a] + (size_t)(row_ok ? m0 + (int)row : 0) * p.K + kbb * kKB;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
@@ -274,6 +291,7 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_gemm_kernel(const GemmPa
             const int CB = AK == 4 ? 32 : 16;  // code bytes of one row in one group
 #pragma unroll
             for (int a = 0; a < NA; ++a) {
+              if (!mine(a, gbase + (uint32_t)kb)) continue;
               const uint8_t* cp = blob + p.off_codes[a] + blk * (size_t)(8 * CB) + (size_t)(grow & 7) * CB;
               const uint32_t dst = cs + (uint32_t)a * kTileM * 36u + row * 32u;
               tc::cp16(dst, cp, 16u);
@@ -308,6 +326,7 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_gemm_kernel(const GemmPa
           const uint32_t cs = sbase + L.code0 + (g % (uint32_t)L.SC) * L.code_stage;
 #pragma unroll
           for (int a = 0; a < NA; ++a) {
+            if (!mine(a, gbase + (uint32_t)kb)) continue;
             const uint32_t arow = st + L.a0 + a * kATile + row * 128u;
             if (row_ok) {
               uint32_t sw;
@@ -327,6 +346,7 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_gemm_kernel(const GemmPa
       tc::cp_wait<0>();
       kb_global += (uint32_t)KB;
       if (!ok) break;
+      if (half) continue;  // helpers: on to the next tile's copies
       // ---- epilogue: wait for the tile's accumulators ----
       ok = gwait(accfull, tile_iter & 1u, p, t0);
       if (!ok) break;
@@ -403,7 +423,7 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_gemm_kernel(const GemmPa
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
