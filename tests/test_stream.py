@@ -247,7 +247,7 @@ class _Layers:
     and experts (replica = layer), resident on the device, and the pinned host
     store [layer][expert] of the packed experts."""
 
-    def __init__(self, M, s, n_layers, device_pack=False):
+    def __init__(self, M, s, n_layers, device_pack=False, **layer_kw):
         import torch
         self.M, self.s, self.L = M, s, n_layers
         self.cfg = mcfg(s)
@@ -265,7 +265,7 @@ class _Layers:
                 torch.cuda.synchronize()
                 dl = self._resident(l, blobs)
             else:
-                dl = DeviceLayer(s, replica=l)
+                dl = DeviceLayer(s, replica=l, **layer_kw)
                 blobs = dl.pool[:E]
             self.store[l * E:(l + 1) * E].copy_(blobs.cpu())
             self.layers.append(dl)
@@ -529,7 +529,10 @@ def _run_streamed(M, lay, n_slots, steps, tokens):
     try:
         for l, xd, rd, _, _, _, _ in plan:
             dl = lay.layers[l]
-            wts = M.layer_weights(None, dl.wr, dl.bias, dl.sg, dl.su, dl.sd, dl.gamma)
+            spacked, sgate = getattr(dl, "spacked", None), getattr(dl, "sgate", None)
+            bf = spacked is None  # the shared expert's form as in the resident layer
+            wts = M.layer_weights(None, dl.wr, dl.bias, dl.sg if bf else None, dl.su if bf else None,
+                                  dl.sd if bf else None, dl.gamma, shared_out_gate=sgate, shared_packed=spacked)
             h2, y2 = torch.empty_like(xd), torch.empty_like(xd)
             i2 = torch.empty((tokens, s.top_k), dtype=torch.int32, device="cuda")
             w2 = torch.empty((tokens, s.top_k), dtype=torch.float32, device="cuda")
@@ -542,9 +545,14 @@ def _run_streamed(M, lay, n_slots, steps, tokens):
             assert np.array_equal(w2.cpu().numpy(), p[6].cpu().numpy()), i
             assert np.array_equal(from_dev_bits(h2), from_dev_bits(p[3])), i
             assert np.array_equal(from_dev_bits(y2), from_dev_bits(p[4])), i
+        # one resolve per launch: tokens beyond one launch's limit run in
+        # successive launches, each looking up its own experts
+        chunk = M.moe_layer_tokens_per_launch(lay.cfg)
         ref = RefCache(n_slots)
         for (l, *_), (_, _, i2, _) in zip(plan, outs):
-            ref.resolve(l, i2.cpu().numpy().ravel().tolist())
+            ids = i2.cpu().numpy()
+            for t0 in range(0, ids.shape[0], chunk):
+                ref.resolve(l, ids[t0:t0 + chunk].ravel().tolist())
         st = M.moe_stream_stats(cache)
         assert st["device_error"] == 0
         for k in ("hits", "misses"):
@@ -567,6 +575,28 @@ def test_streamed_layer_matches_resident_tiny(M, tokens):
     lay = _Layers(M, replace(S.TINY, tokens=2), n_layers=3)
     st = _run_streamed(M, lay, n_slots=7 if tokens == 1 else 20, steps=5, tokens=tokens)
     assert st["misses"] > 0 and st["hits"] > 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("form", ["2bit", "more_tokens_than_one_launch", "packed_shared_gated"])
+def test_streamed_layer_forms(M, form):
+    """The streamed call with 2-bit experts; with more tokens than one
+    launch takes (successive launches, each resolving its own experts); and
+    with the shared expert packed like the routed ones (its pair is not
+    looked up in the cache) behind a sigmoid gate."""
+    if form == "2bit":
+        lay = _Layers(M, replace(S.TINY, bits=2, tokens=2), n_layers=2)
+        st = _run_streamed(M, lay, n_slots=7, steps=4, tokens=2)
+    elif form == "more_tokens_than_one_launch":
+        lay = _Layers(M, replace(S.TINY, tokens=12), n_layers=2, max_tokens=12)
+        assert M.moe_layer_tokens_per_launch(lay.cfg) < 12
+        st = _run_streamed(M, lay, n_slots=24, steps=3, tokens=12)
+    else:
+        s = replace(S.TINY, tokens=2)
+        g = S.rng(s.seed, 0, "shared_out_gate", s.hidden).standard_normal(s.hidden).astype(np.float32)
+        lay = _Layers(M, s, n_layers=2, shared_packed=True, shared_out_gate=S.f32_to_bf16_bits(g * np.float32(0.1)))
+        st = _run_streamed(M, lay, n_slots=7, steps=4, tokens=2)
+    assert st["misses"] > 0
 
 
 @pytest.mark.gpu
