@@ -491,7 +491,9 @@ moe_status moe_stream_resolve_device(moe_stream_cache* cache, int layer, const i
  * assignments undone, and the layer's device error word (moe_device_error)
  * reports a bad expert pointer; its outputs are then not written.  Tokens
  * beyond one launch's limit (64 / K) run in successive launches, each
- * resolving its own experts. */
+ * resolving its own experts.  A launch changes the cache's tables and slots:
+ * calls that share a cache (this one, moe_stream_resolve_device and the
+ * layers reading its slots) must be ordered, e.g. on one stream. */
 moe_status moe_layer_forward_streamed(const moe_config* cfg, const moe_layer_weights* wts, const void* x_bf16,
                                       const void* residual_bf16, int T, void* h_out_bf16, void* y_norm_bf16,
                                       int32_t* idx_out, float* w_out, moe_stream_cache* cache, int layer,
