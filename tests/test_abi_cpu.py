@@ -123,6 +123,13 @@ def test_argument_checks_without_gpu():
     # T == 0 is a no-op that touches nothing
     st = lib.moe_layer_forward(C.byref(good), None, None, None, 0, None, None, None, None, None, 0, None)
     assert st == 0
+    # the streamed call refuses a bad shape or a NULL cache before any device work
+    st = lib.moe_layer_forward_streamed(C.byref(bad), C.byref(wts), 16, 16, 1, 16, 16, None, None, None, 0, 256,
+                                        1 << 20, None)
+    assert st == 2
+    st = lib.moe_layer_forward_streamed(C.byref(good), C.byref(wts), 16, 16, 1, 16, 16, None, None, None, 0, 256,
+                                        1 << 20, None)
+    assert st == 1 and "cache" in M.last_error()
     k_gt_e = M.config(256, 128, 4, 8)
     st = lib.moe_layer_forward(C.byref(k_gt_e), C.byref(wts), 16, 16, 1, 16, 16, None, None, 256, 1 << 20, None)
     assert st == 2
